@@ -1,0 +1,189 @@
+"""CPU oracle for the symmetric INT4 GPTQ W4A16 linear layer.
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's CPU
+baseline leg may import this package; the library and its Python binding never
+do.  The arithmetic lives in ``gptq_oracle.c`` (plain C, binary64, one element
+at a time); this module only compiles it with gcc and marshals numpy arrays.
+
+Definition (GPTQ-Pro README, "Runtime contract"; GPTQModel wiki "Installation
+and Quickstart", "Defaults and compatibility decisions"):
+    q[k,n] = (uint32(qweight[k//8, n]) >> 4*(k%8)) & 0xF
+    W[k,n] = fp16_RNE((q[k,n] - 8) * scales[k//G, n])
+    Y[m,n] = sum_k x[m,k] * W[k,n]            (binary64, k ascending)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gptq_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+_p = ctypes.c_void_p
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, no fast-math) into oracle/_build."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or \
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".{os.getpid()}.tmp"
+        subprocess.run(["gcc", "-O2", "-fno-fast-math", "-std=c11", "-shared", "-fPIC",
+                        "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.oracle_half_to_double.restype = ctypes.c_double
+            lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
+            lib.oracle_double_to_half.restype = ctypes.c_uint16
+            lib.oracle_double_to_half.argtypes = [ctypes.c_double]
+            lib.oracle_round_to_half.argtypes = [_p, _i64, _p]
+            lib.oracle_unpack.argtypes = [_p, _i64, _i64, _p]
+            lib.oracle_pack.argtypes = [_p, _i64, _i64, _p]
+            lib.oracle_num_groups.restype = _i64
+            lib.oracle_num_groups.argtypes = [_i64, _i32]
+            lib.oracle_dequant.argtypes = [_p, _p, _i64, _i64, _i32, _p]
+            lib.oracle_gemm.restype = ctypes.c_int
+            lib.oracle_gemm.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32, _p]
+            lib.oracle_gemm_entries.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32,
+                                                _i64, _p, _p, _p]
+            lib.oracle_gemm_rows.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32,
+                                             _i64, _p, _p]
+            _lib = lib
+    return _lib
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a)
+    if a.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {a.dtype}")
+    return a
+
+
+def _ptr(a):
+    return a.ctypes.data_as(_p)
+
+
+def _bits16(a):
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float16:
+        return a.view(np.uint16)
+    return _c(a, np.uint16)
+
+
+def half_to_double(h: int) -> float:
+    return _load().oracle_half_to_double(int(h))
+
+
+def double_to_half_bits(v: float) -> int:
+    return int(_load().oracle_double_to_half(float(v)))
+
+
+def round_to_half(v: np.ndarray) -> np.ndarray:
+    """binary64 -> binary16 (round to nearest, ties to even), as float16."""
+    v = _c(np.asarray(v, dtype=np.float64), np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    _load().oracle_round_to_half(_ptr(v), v.size, _ptr(out))
+    return out.view(np.float16)
+
+
+def num_groups(K: int, group: int) -> int:
+    return int(_load().oracle_num_groups(K, group))
+
+
+def unpack(qweight: np.ndarray) -> np.ndarray:
+    """int32 [K/8, N] -> uint8 codes [K, N]."""
+    qw = _c(qweight, np.int32)
+    K, N = qw.shape[0] * 8, qw.shape[1]
+    codes = np.empty((K, N), dtype=np.uint8)
+    _load().oracle_unpack(_ptr(qw), K, N, _ptr(codes))
+    return codes
+
+
+def pack(codes: np.ndarray) -> np.ndarray:
+    """uint8 codes [K, N] (values 0..15) -> int32 [K/8, N]."""
+    c = _c(codes, np.uint8)
+    K, N = c.shape
+    if K % 8:
+        raise ValueError("K must be a multiple of 8")
+    qw = np.empty((K // 8, N), dtype=np.int32)
+    _load().oracle_pack(_ptr(c), K, N, _ptr(qw))
+    return qw
+
+
+def dequant(qweight: np.ndarray, scales: np.ndarray, group: int) -> np.ndarray:
+    """W = fp16((q - 8) * s) as float16 [K, N]."""
+    qw = _c(qweight, np.int32)
+    s = _bits16(scales)
+    K, N = qw.shape[0] * 8, qw.shape[1]
+    if s.shape != (num_groups(K, group), N):
+        raise ValueError(f"scales shape {s.shape} does not match K={K}, group={group}")
+    w = np.empty((K, N), dtype=np.uint16)
+    _load().oracle_dequant(_ptr(qw), _ptr(s), K, N, group, _ptr(w))
+    return w.view(np.float16)
+
+
+def gemm(x: np.ndarray, qweight: np.ndarray, scales: np.ndarray, group: int) -> np.ndarray:
+    """Y = x . W in binary64, float64 [M, N]."""
+    xb = _bits16(x)
+    qw = _c(qweight, np.int32)
+    s = _bits16(scales)
+    M, K = xb.shape
+    N = qw.shape[1]
+    if qw.shape[0] * 8 != K:
+        raise ValueError("x and qweight disagree on K")
+    y = np.empty((M, N), dtype=np.float64)
+    if _load().oracle_gemm(_ptr(xb), _ptr(qw), _ptr(s), M, K, N, group, _ptr(y)):
+        raise MemoryError("oracle_gemm could not allocate its dequantised copy")
+    return y
+
+
+def gemm_entries(x, qweight, scales, group, ms, ns) -> np.ndarray:
+    """Y[ms[i], ns[i]] in binary64, for sampled checks on large problems."""
+    xb = _bits16(x)
+    qw = _c(qweight, np.int32)
+    s = _bits16(scales)
+    M, K = xb.shape
+    N = qw.shape[1]
+    ms = _c(np.asarray(ms, dtype=np.int64), np.int64)
+    ns = _c(np.asarray(ns, dtype=np.int64), np.int64)
+    if ms.shape != ns.shape:
+        raise ValueError("ms and ns must have the same length")
+    if ms.size and (ms.min() < 0 or ms.max() >= M or ns.min() < 0 or ns.max() >= N):
+        raise IndexError("sample index out of range")
+    out = np.empty(ms.shape, dtype=np.float64)
+    _load().oracle_gemm_entries(_ptr(xb), _ptr(qw), _ptr(s), M, K, N, group,
+                                ms.size, _ptr(ms), _ptr(ns), _ptr(out))
+    return out
+
+
+def gemm_rows(x, qweight, scales, group, ms) -> np.ndarray:
+    """Full rows Y[ms, :] in binary64, float64 [len(ms), N]."""
+    xb = _bits16(x)
+    qw = _c(qweight, np.int32)
+    s = _bits16(scales)
+    M, K = xb.shape
+    N = qw.shape[1]
+    ms = _c(np.asarray(ms, dtype=np.int64), np.int64)
+    if ms.size and (ms.min() < 0 or ms.max() >= M):
+        raise IndexError("row index out of range")
+    out = np.empty((ms.size, N), dtype=np.float64)
+    _load().oracle_gemm_rows(_ptr(xb), _ptr(qw), _ptr(s), M, K, N, group,
+                             ms.size, _ptr(ms), _ptr(out))
+    return out
