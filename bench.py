@@ -1,0 +1,431 @@
+"""Benchmark of the B200 W4A16 GPTQ linear (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode_up] [--no-sweep]
+
+A step is one call of gptq_w4a16_gemm (validate, dispatch, kernel) on the
+headline workload: the decode GEMV of the FFN up-projection shape, M=1,
+K=5120, N=17408, group 128 (46.0 MB of algorithmic traffic per call).  The
+metric is achieved GB/s of algorithmic bytes (packed weights + scales + X + Y,
+each moved once).  Inputs are resident in HBM; consecutive steps rotate over
+enough distinct copies of the weights that every step reads from HBM, not L2.
+
+With N > 1 (torchrun), every rank runs an independent replica on its own GPU
+(the layer needs no exchange between GPUs): value = all ranks' bytes / the
+slowest rank's time.  `--impl reference` times the CPU oracle instead (rank 0
+only) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from int4_weight_only_gptq_b200 import workloads as W  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode_up")
+    ap.add_argument("--no-sweep", action="store_true")
+    return ap.parse_args()
+
+
+WORKLOADS = {
+    "decode_up": (lambda: W.decode_up(), "decode GEMV, FFN up-projection: M=1, K=5120, N=17408, group=128"),
+}
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def traffic_record(kernel_file: str, key: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (matching hash); else None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    src = os.path.join(ROOT, "int4_weight_only_gptq_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(src)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(src, name), "rb") as f:
+                h.update(f.read())
+    digest = h.hexdigest()[:16]
+    try:
+        with open(path) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 3 and parts[0] == key and parts[1] == digest:
+                    return float(parts[2])
+    except OSError:
+        pass
+    return None
+
+
+# ---- clocks --------------------------------------------------------------
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, index: int, uuid: str | None = None, period_s: float = 0.01):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = None
+            if uuid:
+                try:
+                    self.h = pynvml.nvmlDeviceGetHandleByUUID(
+                        uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+                except Exception:
+                    self.h = None
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---- GPU arm -------------------------------------------------------------
+
+def to_device(p, torch, copies: int):
+    x = torch.from_numpy(p.x.view(np.int16)).view(torch.float16).cuda()
+    qw0 = torch.from_numpy(p.qweight).cuda()
+    s0 = torch.from_numpy(p.scales.view(np.int16)).view(torch.float16).cuda()
+    sets = []
+    for i in range(copies):
+        qw = qw0 if i == 0 else qw0.clone()
+        s = s0 if i == 0 else s0.clone()
+        xi = x if i == 0 else x.clone()
+        y = torch.empty((p.M, p.N), dtype=torch.float16, device="cuda")
+        sets.append((xi, qw, s, y))
+    return sets
+
+
+def copies_for(p, l2_bytes: int) -> int:
+    per = p.K * p.N // 2 + p.scales.size * 2 + p.M * p.K * 2 + p.M * p.N * 2
+    return max(1, math.ceil(2 * l2_bytes / per) + 1)
+
+
+def time_gemm(lib, torch, p, steps, warmup, kernel=0, stream=None, l2_bytes=0):
+    """Device time per call (ms) of back-to-back calls through the C ABI."""
+    copies = copies_for(p, l2_bytes) if l2_bytes else 1
+    sets = to_device(p, torch, copies)
+    stream = stream or torch.cuda.current_stream()
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    fn = lib.gptq_w4a16_gemm if kernel == 0 else lib.gptq_w4a16_gemm_kernel
+    argv = []
+    for (x, qw, s, y) in sets:
+        a = (ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(qw.data_ptr()),
+             ctypes.c_void_p(s.data_ptr()), p.M, p.K, p.N, p.group, ctypes.c_void_p(y.data_ptr()), sh)
+        argv.append(a if kernel == 0 else a + (kernel,))
+    for i in range(warmup):
+        st = fn(*argv[i % copies])
+        if st:
+            raise RuntimeError(f"gemm status {st}")
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        fn(*argv[i % copies])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, copies
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from int4_weight_only_gptq_b200 import binding
+
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    lib = binding.load()
+    props = torch.cuda.get_device_properties(local_rank)
+    l2 = props.L2_cache_size
+    make, desc = WORKLOADS[args.workload]
+    p = make()
+    bytes_per_step = p.algorithmic_bytes
+    copies = copies_for(p, l2)
+    sets = to_device(p, torch, copies)
+    stream = torch.cuda.current_stream()
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    argv = [(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(qw.data_ptr()),
+             ctypes.c_void_p(s.data_ptr()), p.M, p.K, p.N, p.group,
+             ctypes.c_void_p(y.data_ptr()), sh) for (x, qw, s, y) in sets]
+    fn = lib.gptq_w4a16_gemm
+    for i in range(max(3, args.warmup)):
+        st = fn(*argv[i % copies])
+        if st:
+            raise RuntimeError(f"gptq_w4a16_gemm returned {st}: {binding.status_string(st)}")
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank, str(getattr(props, "uuid", "")) or None) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            fn(*argv[i % copies])
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    if binding.device_error() != 0:
+        raise RuntimeError("a kernel reported a bounded-wait timeout")
+    ms = elapsed_ms / args.steps
+    value = bytes_per_step * world / (ms * 1e-3) / 1e9
+    per_gpu = bytes_per_step / (ms * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers: pinned X in, Y out
+    xh = torch.from_numpy(p.x.view(np.int16)).view(torch.float16).pin_memory()
+    yh = torch.empty((p.M, p.N), dtype=torch.float16).pin_memory()
+    xd, qw, s, yd = sets[0]
+    e2 = []
+    for rep in range(2):
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(10, min(args.steps, 500))
+        a0.record(stream)
+        for i in range(n_e2e):
+            xs, qws, ss, ys = sets[i % copies]
+            xs.copy_(xh, non_blocking=True)
+            binding.gemm(xs, qws, ss, p.group, out=ys, stream=stream)
+            yh.copy_(ys, non_blocking=True)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e2.append(a0.elapsed_time(a1) / n_e2e)
+    e2e_ms = min(e2)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    hbm, tf, src = peaks()
+    out = None
+    if rank == 0:
+        clocks = clk.summary()
+        kernel_id, split = binding.select(p.M, p.K, p.N, p.group)
+        traffic = traffic_record("decode.cu", f"{args.workload}")
+        out = {
+            "metric": "W4A16 GEMM decode GB/s (algorithmic bytes: packed weights + scales + X + Y)",
+            "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": round(ms, 6),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp16 x int4 -> fp32 acc -> fp16", "data": "synthetic (seeded, PCG64 seed 0)",
+            "config": {"workload": desc, "M": p.M, "K": p.K, "N": p.N, "group": p.group,
+                       "bytes_per_step": bytes_per_step,
+                       "l2": f"rotating {copies} input copies ({copies * bytes_per_step / 1e6:.0f} MB > 2x L2 {l2 / 1e6:.0f} MB)",
+                       "parallelism": f"replicas x{world} (no exchange)",
+                       "kernel": {1: "decode", 2: "prefill"}.get(kernel_id, kernel_id),
+                       "split_k_ctas": split},
+            "roofline": {"bound": "hbm", "achieved": round(per_gpu, 1), "peak": hbm,
+                         "unit": "GB/s", "frac": round(per_gpu / hbm, 4),
+                         "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6.65 TB/s",
+                         "traffic": traffic},
+            "e2e": {"value": round(bytes_per_step * world / (e2e_ms * 1e-3) / 1e9, 1),
+                    "unit": "GB/s", "ms_per_step": round(e2e_ms, 6),
+                    "h2d_bytes_per_step": int(p.M * p.K * 2),
+                    "d2h_bytes_per_step": int(p.M * p.N * 2),
+                    "note": "pinned host X -> device, gptq_w4a16_gemm, device Y -> pinned host; weights resident"},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+        }
+    if not args.no_sweep and world == 1:
+        sweep = run_sweep(lib, torch, l2, hbm, tf)
+        if rank == 0:
+            out["sweep"] = sweep
+    if rank == 0:
+        out["cpu_baseline"] = cpu_baseline(p, bytes_per_step)
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_sweep(lib, torch, l2, hbm, tf):
+    """The other workloads, one line each: decode GB/s, prefill TFLOP/s."""
+    res = {}
+
+    def hbm_case(name, p, steps=300):
+        ms, copies = time_gemm(lib, torch, p, steps, 20, l2_bytes=l2)
+        gbs = p.algorithmic_bytes / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 5), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
+
+    def tc_case(name, p, steps=30):
+        ms, _ = time_gemm(lib, torch, p, steps, 5)
+        tfl = p.flops / (ms * 1e-3) / 1e12
+        res[name] = {"ms": round(ms, 4), "TFLOP/s": round(tfl, 1), "frac_tensor": round(tfl / tf, 3)}
+
+    for M in (1, 2, 4, 8, 16):
+        hbm_case(f"decode_down_M{M}", W.decode_down(M))
+    for M in (512, 2048, 8192):
+        tc_case(f"prefill_M{M}", W.prefill(M))
+    for g in W.GROUP_SIZES:
+        hbm_case(f"square_g{g}_M1", W.group_sweep(g, 1))
+        hbm_case(f"square_g{g}_M16", W.group_sweep(g, 16))
+        tc_case(f"square_g{g}_M4096", W.group_sweep(g, 4096))
+    for name, K, N, count in W.LAYER_LINEARS:
+        for M in (1, 16):
+            hbm_case(f"layer_{name}_M{M}", W.layer_linear(name, M))
+        tc_case(f"layer_{name}_M4096", W.layer_linear(name, 4096))
+    for M in (1, 16, 4096):
+        key = "ms"
+        total = sum(res[f"layer_{n}_M{M}"][key] * c for n, _, _, c in W.LAYER_LINEARS)
+        res[f"layer_total_M{M}_ms"] = round(total, 4)
+    return res
+
+
+# ---- CPU oracle ----------------------------------------------------------
+
+def cpu_baseline(p, bytes_per_step, budget_s: float = 10.0):
+    """The oracle as it stands, single-threaded, on whole calls of the same
+    workload (M=1 computes every output), repeated for about budget_s."""
+    import oracle
+    oracle.build()
+    threads = oracle.get_threads()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.gemm_rows(p.x, p.qweight, p.scales, p.group, list(range(p.M)))
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 1000:
+            break
+    per = el / n
+    return {"value": round(bytes_per_step / per / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{n} whole call(s) of the workload ({el:.1f} s, {threads} OpenMP threads over output columns)",
+            "s_per_call": round(per, 4)}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: rank 0 only, each step one oracle call
+    on a column slice of the workload (every k, every row), so that a step
+    takes a fraction of a second; GB/s counts the slice's share of the bytes."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    make, desc = WORKLOADS[args.workload]
+    p = make()
+    import oracle
+    oracle.build()
+    threads = oracle.get_threads()
+    n_cols = 1088  # N / 16 for the up-projection
+    frac = n_cols / p.N
+    rows = np.repeat(np.arange(p.M, dtype=np.int64), n_cols)
+    warm = min(max(3, args.warmup), 3)
+    times = []
+    for i in range(warm + args.steps):
+        c0 = (i * n_cols) % (p.N - n_cols + 1)
+        cols = np.tile(np.arange(c0, c0 + n_cols, dtype=np.int64), p.M)
+        t0 = time.perf_counter()
+        oracle.gemm_entries(p.x, p.qweight, p.scales, p.group, rows, cols)
+        if i >= warm:
+            times.append(time.perf_counter() - t0)
+        if sum(times) > 90:
+            break
+    ms = 1e3 * sum(times) / len(times)
+    v = frac * p.algorithmic_bytes / (ms * 1e-3) / 1e9
+    sample = (f"{len(times)} steps, each all {p.M} row(s) x {n_cols} of {p.N} columns "
+              f"(1/16 of the workload), {threads} OpenMP threads over output entries")
+    print(json.dumps({
+        "impl": "reference", "metric": "W4A16 GEMM decode GB/s (algorithmic bytes: packed weights + scales + X + Y)",
+        "value": round(v, 4), "unit": "GB/s", "n_gpus": world, "steps": len(times),
+        "warmup": warm, "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+        "data": "synthetic (seeded, PCG64 seed 0)",
+        "config": {"workload": desc, "M": p.M, "K": p.K, "N": p.N, "group": p.group},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

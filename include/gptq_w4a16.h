@@ -1,0 +1,146 @@
+/*
+ * gptq_w4a16.h — C ABI of the B200 (sm_100a) symmetric INT4 GPTQ W4A16 linear.
+ *
+ *   Y[M,N] = X[M,K] . W[K,N],   W[k,n] = fp16_RNE((q[k,n] - 8) * scales[k/G, n])
+ *   q[k,n] = (uint32(qweight[k/8, n]) >> (4*(k%8))) & 0xF
+ *
+ * Source of the operation: GPTQ-Pro README, "Runtime contract" (symmetric GPTQ
+ * INT4, FP16 activations, desc_act=False, native int32 qweight, group sizes
+ * -1/16/32/64/128/256/512/1024, input features divisible by 16, output
+ * features divisible by 8) and "Ampere kernel architecture" (a small-M fused
+ * decode path, a tensor-core prefill path, FP32 accumulation, deterministic
+ * split-K; all paths read the original int32 qweight); GPTQModel wiki
+ * "Installation and Quickstart", "Defaults and compatibility decisions" (sym
+ * True, pack_dtype int32).  The pages do not state the nibble order; this
+ * library reads the lowest nibble as the lowest k.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named x, qweight, scales, y, w_out are DEVICE pointers on the
+ *    current CUDA device, dense and row-major.  FP16 values travel as their
+ *    16-bit patterns (uint16_t).  All must be 16-byte aligned.
+ *  - The caller owns every buffer.  The library allocates no device memory,
+ *    keeps no dequantised or repacked copy of the weights, and holds no state
+ *    between calls other than a per-device attribute cache and a device-side
+ *    error word (see gptq_device_error).
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *    stream-ordered and asynchronous: they enqueue work and return without
+ *    synchronising.
+ *  - Arguments are checked before anything is enqueued.  A failed check
+ *    returns a gptq_status and enqueues nothing; there is no fallback path.
+ *  - Results are deterministic: the same inputs give bitwise-identical outputs.
+ *  - The library is reentrant; concurrent calls on different streams are safe.
+ */
+#ifndef GPTQ_W4A16_H
+#define GPTQ_W4A16_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GPTQ_API __attribute__((visibility("default")))
+#else
+#define GPTQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GPTQ_OK = 0,
+    GPTQ_ERR_NULL = 1,     /* a required pointer is NULL                              */
+    GPTQ_ERR_SHAPE = 2,    /* M < 0, K <= 0, N <= 0, K % 16, N % 8, or a size limit    */
+    GPTQ_ERR_GROUP = 3,    /* group not in {-1,16,32,64,128,256,512,1024}              */
+    GPTQ_ERR_ALIGN = 4,    /* a pointer is not 16-byte aligned                        */
+    GPTQ_ERR_DEVICE = 5,   /* no current device, or it is not compute capability 10.0 */
+    GPTQ_ERR_CUDA = 6,     /* the CUDA runtime reported an error at launch             */
+    GPTQ_ERR_TIMEOUT = 7,  /* a kernel gave up a bounded wait (see gptq_device_error)  */
+    GPTQ_ERR_ALIAS = 8,    /* the output overlaps an input                            */
+    GPTQ_ERR_KERNEL = 9    /* kernel_id names no kernel, or one that cannot take M     */
+} gptq_status;
+
+/* Kernel identifiers reported by gptq_w4a16_select and accepted by
+ * gptq_w4a16_gemm_kernel. */
+#define GPTQ_KERNEL_AUTO 0
+#define GPTQ_KERNEL_DECODE 1   /* M <= 16: streams qweight, split-K, warp MMA      */
+#define GPTQ_KERNEL_PREFILL 2  /* any M: TMA + tcgen05 MMA with TMEM accumulators  */
+
+/* Size limits (inclusive). */
+#define GPTQ_MAX_K 1048576
+#define GPTQ_MAX_N 1048576
+#define GPTQ_MAX_M 8388608
+#define GPTQ_DECODE_MAX_M 16
+
+/*
+ * Y = X . dequant(qweight, scales).
+ *   x       [M, K]          FP16 bits    (may be NULL only when M == 0)
+ *   qweight [K/8, N]        int32, eight 4-bit codes along K, lowest nibble = lowest k
+ *   scales  [n_groups, N]   FP16 bits, n_groups = 1 if group == -1 or group >= K,
+ *                           else ceil(K / group); the last group may be ragged
+ *   y       [M, N]          FP16 bits, written (may be NULL only when M == 0);
+ *                           must not overlap x, qweight or scales
+ * Accumulation is FP32; each output is rounded once to FP16 (nearest-even).
+ * M == 0 returns GPTQ_OK and enqueues nothing.  The kernel is chosen by
+ * gptq_w4a16_select.
+ */
+GPTQ_API int gptq_w4a16_gemm(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                    int64_t M, int64_t K, int64_t N, int32_t group,
+                    uint16_t* y, void* stream);
+
+/*
+ * As gptq_w4a16_gemm, with the kernel forced: kernel_id is one of the
+ * GPTQ_KERNEL_* values (AUTO behaves exactly like gptq_w4a16_gemm).  DECODE
+ * accepts M <= GPTQ_DECODE_MAX_M only (else GPTQ_ERR_KERNEL).  Meant for tests
+ * and benchmarks that compare the kernels on the same shape.
+ */
+GPTQ_API int gptq_w4a16_gemm_kernel(const uint16_t* x, const int32_t* qweight,
+                           const uint16_t* scales, int64_t M, int64_t K, int64_t N,
+                           int32_t group, uint16_t* y, void* stream, int32_t kernel_id);
+
+/*
+ * As gptq_w4a16_gemm_kernel with GPTQ_KERNEL_DECODE, with the number of CTAs
+ * that split K within one column block fixed to `splits` (1..8) instead of
+ * chosen from the shape.  Any split gives a correct, deterministic result;
+ * the choice only moves performance.  Meant for tuning sweeps and tests.
+ */
+GPTQ_API int gptq_w4a16_gemm_decode_splits(const uint16_t* x, const int32_t* qweight,
+                                           const uint16_t* scales, int64_t M, int64_t K,
+                                           int64_t N, int32_t group, uint16_t* y, void* stream,
+                                           int32_t splits);
+
+/*
+ * W[K, N] = dequant(qweight, scales) as FP16 bits, each value rounded once from
+ * the exact (q - 8) * s (a debugging and verification entry; the GEMM never
+ * materialises W).  w_out must not overlap qweight or scales.
+ */
+GPTQ_API int gptq_dequant(const int32_t* qweight, const uint16_t* scales, int64_t K, int64_t N,
+                 int32_t group, uint16_t* w_out, void* stream);
+
+/*
+ * The dispatcher, observable: which kernel gptq_w4a16_gemm would launch for
+ * this shape and with how many K-splits (1 when the kernel does not split K).
+ * Validates the shape and group like the GEMM (not the pointers); needs a
+ * current CUDA device of compute capability 10.0 (the split depends on its SM
+ * count).  Either output pointer may be NULL.
+ */
+GPTQ_API int gptq_w4a16_select(int64_t M, int64_t K, int64_t N, int32_t group,
+                      int32_t* kernel_id, int32_t* split_k);
+
+/* Static, human-readable name of a gptq_status value. */
+GPTQ_API const char* gptq_status_string(int status);
+
+/*
+ * Reads and clears the device-side error word of the current device: 0 when
+ * no kernel gave up a bounded wait since the last call, else GPTQ_ERR_TIMEOUT.
+ * Synchronises the current device.  Kernels never trap: a wait that exceeds
+ * its bound records the error here, abandons the output tile and exits.
+ */
+GPTQ_API int gptq_device_error(void);
+
+/* Library version as "major.minor.patch". */
+GPTQ_API const char* gptq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_W4A16_H */

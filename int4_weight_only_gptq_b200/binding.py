@@ -1,0 +1,182 @@
+"""Python binding of libgptq_w4a16.so (ctypes; argument marshalling only).
+
+Every step of the layer runs in the library's CUDA kernels.  PyTorch supplies
+device memory and the current stream; this module checks tensor dtypes and
+devices, passes raw pointers, and turns status codes into exceptions.  There is
+no CPU path: if the library is missing or the device is not sm_100, calls
+raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libgptq_w4a16.so")
+
+KERNEL_AUTO, KERNEL_DECODE, KERNEL_PREFILL = 0, 1, 2
+DECODE_MAX_M = 16
+GROUP_SIZES = (-1, 16, 32, 64, 128, 256, 512, 1024)
+
+STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_NULL", 2: "GPTQ_ERR_SHAPE", 3: "GPTQ_ERR_GROUP",
+          4: "GPTQ_ERR_ALIGN", 5: "GPTQ_ERR_DEVICE", 6: "GPTQ_ERR_CUDA",
+          7: "GPTQ_ERR_TIMEOUT", 8: "GPTQ_ERR_ALIAS", 9: "GPTQ_ERR_KERNEL"}
+
+# Every entry point declared in include/gptq_w4a16.h.
+EXPORTS = ("gptq_w4a16_gemm", "gptq_w4a16_gemm_kernel", "gptq_w4a16_gemm_decode_splits",
+           "gptq_dequant", "gptq_w4a16_select", "gptq_status_string", "gptq_device_error",
+           "gptq_version")
+
+
+class GptqError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+_lock = threading.Lock()
+_lib = None
+
+_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the library once (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    f"CUDA library not built: {path} is missing "
+                    "(run `python -m int4_weight_only_gptq_b200.build`)")
+            lib = ctypes.CDLL(path)
+            gemm_args = [_p, _p, _p, _i64, _i64, _i64, _i32, _p, _p]
+            lib.gptq_w4a16_gemm.argtypes = gemm_args
+            lib.gptq_w4a16_gemm_kernel.argtypes = gemm_args + [_i32]
+            lib.gptq_w4a16_gemm_decode_splits.argtypes = gemm_args + [_i32]
+            lib.gptq_dequant.argtypes = [_p, _p, _i64, _i64, _i32, _p, _p]
+            lib.gptq_w4a16_select.argtypes = [_i64, _i64, _i64, _i32,
+                                              ctypes.POINTER(_i32), ctypes.POINTER(_i32)]
+            lib.gptq_status_string.restype = ctypes.c_char_p
+            lib.gptq_status_string.argtypes = [ctypes.c_int]
+            lib.gptq_device_error.argtypes = []
+            lib.gptq_version.restype = ctypes.c_char_p
+            for name in ("gptq_w4a16_gemm", "gptq_w4a16_gemm_kernel",
+                         "gptq_w4a16_gemm_decode_splits", "gptq_dequant",
+                         "gptq_w4a16_select", "gptq_device_error"):
+                getattr(lib, name).restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().gptq_status_string(int(status)).decode()
+
+
+def _check(status: int):
+    if status != 0:
+        raise GptqError(status, status_string(status))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _as_bits16(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype == torch.float16:
+        return t
+    if t.dtype in (torch.int16, torch.uint16):
+        return t
+    raise TypeError(f"expected a float16 tensor, got {t.dtype}")
+
+
+def _require(t: torch.Tensor, name: str, dtype_ok, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+    if not dtype_ok(t.dtype):
+        raise TypeError(f"{name} has dtype {t.dtype}")
+
+
+def gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, group: int,
+         out: torch.Tensor | None = None, stream=None, kernel: int = KERNEL_AUTO,
+         decode_splits: int = 0) -> torch.Tensor:
+    """Y[M, N] = x[M, K] . dequant(qweight[K/8, N], scales[n_groups, N]) (FP16)."""
+    lib = load()
+    dev = qweight.device
+    _require(qweight, "qweight", lambda d: d == torch.int32, None)
+    _require(scales, "scales", lambda d: d == torch.float16, dev)
+    _require(x, "x", lambda d: d == torch.float16, dev)
+    if x.dim() != 2 or qweight.dim() != 2 or scales.dim() != 2:
+        raise ValueError("x, qweight and scales must be 2-D")
+    M, K = x.shape
+    N = qweight.shape[1]
+    if qweight.shape[0] * 8 != K:
+        raise ValueError(f"qweight rows {qweight.shape[0]} do not match K={K}")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=dev)
+    else:
+        _require(out, "out", lambda d: d == torch.float16, dev)
+        if tuple(out.shape) != (M, N):
+            raise ValueError(f"out has shape {tuple(out.shape)}, expected {(M, N)}")
+    s = _stream_handle(stream, dev)
+    args = (_ptr(x), _ptr(qweight), _ptr(scales), M, K, N, group, _ptr(out), s)
+    if decode_splits:
+        _check(lib.gptq_w4a16_gemm_decode_splits(*args, decode_splits))
+    elif kernel == KERNEL_AUTO:
+        _check(lib.gptq_w4a16_gemm(*args))
+    else:
+        _check(lib.gptq_w4a16_gemm_kernel(*args, kernel))
+    return out
+
+
+def dequant(qweight: torch.Tensor, scales: torch.Tensor, group: int,
+            out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """W[K, N] = fp16((q - 8) * s): the debugging entry."""
+    lib = load()
+    dev = qweight.device
+    _require(qweight, "qweight", lambda d: d == torch.int32, None)
+    _require(scales, "scales", lambda d: d == torch.float16, dev)
+    K, N = qweight.shape[0] * 8, qweight.shape[1]
+    if out is None:
+        out = torch.empty((K, N), dtype=torch.float16, device=dev)
+    else:
+        _require(out, "out", lambda d: d == torch.float16, dev)
+    _check(lib.gptq_dequant(_ptr(qweight), _ptr(scales), K, N, group, _ptr(out),
+                            _stream_handle(stream, dev)))
+    return out
+
+
+def select(M: int, K: int, N: int, group: int) -> tuple[int, int]:
+    """(kernel_id, split_k) the dispatcher picks for this shape."""
+    lib = load()
+    k, s = _i32(-1), _i32(-1)
+    _check(lib.gptq_w4a16_select(M, K, N, group, ctypes.byref(k), ctypes.byref(s)))
+    return k.value, s.value
+
+
+def device_error() -> int:
+    """Read and clear the device error word (synchronises the device)."""
+    return int(load().gptq_device_error())
+
+
+def version() -> str:
+    return load().gptq_version().decode()

@@ -1,0 +1,235 @@
+// C ABI of the W4A16 GPTQ library: argument checks (fail-closed, before any
+// launch), the shape-driven dispatcher, and the per-device state.
+//
+// The checks restate the runtime contract of the GPTQ-Pro README ("Runtime
+// contract": group sizes -1/16/32/64/128/256/512/1024, input features
+// divisible by 16, output features divisible by 8; unsupported combinations
+// are rejected, never silently routed elsewhere).
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/gptq_w4a16.h"
+#include "kernels.h"
+
+namespace gptq {
+namespace {
+
+// One error word per device, written only by kernels that give up a wait.
+__device__ int g_error_word;
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_dev_once[kMaxDevices];
+DeviceInfo g_dev[kMaxDevices];
+int g_dev_status[kMaxDevices];
+
+int query_device(const DeviceInfo** out) {
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) {
+    cudaGetLastError();
+    return GPTQ_ERR_DEVICE;
+  }
+  std::call_once(g_dev_once[d], [d] {
+    DeviceInfo info;
+    info.device = d;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, d) != cudaSuccess) {
+      cudaGetLastError();
+      g_dev_status[d] = GPTQ_ERR_DEVICE;
+      return;
+    }
+    info.num_sms = prop.multiProcessorCount;
+    info.cc_major = prop.major;
+    info.cc_minor = prop.minor;
+    info.smem_optin = (int)prop.sharedMemPerBlockOptin;
+    info.l2_bytes = prop.l2CacheSize;
+    if (info.cc_major != 10 || info.cc_minor != 0) {
+      g_dev_status[d] = GPTQ_ERR_DEVICE;
+      return;
+    }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) {
+      cudaGetLastError();
+      g_dev_status[d] = GPTQ_ERR_DEVICE;
+      return;
+    }
+    info.error_word = static_cast<int*>(p);
+    g_dev[d] = info;
+    g_dev_status[d] = GPTQ_OK;
+  });
+  if (g_dev_status[d] != GPTQ_OK) return g_dev_status[d];
+  *out = &g_dev[d];
+  return GPTQ_OK;
+}
+
+bool valid_group(int32_t g) {
+  switch (g) {
+    case -1: case 16: case 32: case 64: case 128: case 256: case 512: case 1024:
+      return true;
+    default:
+      return false;
+  }
+}
+
+int check_shape(int64_t M, int64_t K, int64_t N, int32_t group) {
+  if (M < 0 || K <= 0 || N <= 0) return GPTQ_ERR_SHAPE;
+  if (K % 16 != 0 || N % 8 != 0) return GPTQ_ERR_SHAPE;
+  if (K > GPTQ_MAX_K || N > GPTQ_MAX_N || M > GPTQ_MAX_M) return GPTQ_ERR_SHAPE;
+  if (!valid_group(group)) return GPTQ_ERR_GROUP;
+  return GPTQ_OK;
+}
+
+int64_t num_groups(int64_t K, int32_t group) {
+  if (group == -1 || group >= K) return 1;
+  return (K + group - 1) / group;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, int64_t abytes, const void* b, int64_t bbytes) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + (uintptr_t)bbytes && b0 < a0 + (uintptr_t)abytes;
+}
+
+int select_kernel(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev, int32_t* split) {
+  if (M <= GPTQ_DECODE_MAX_M) {
+    if (split) *split = decode_pick_splits(M, K, N, dev);
+    return GPTQ_KERNEL_DECODE;
+  }
+  if (split) *split = 1;
+  return GPTQ_KERNEL_PREFILL;
+}
+
+int gemm_impl(const uint16_t* x, const int32_t* qweight, const uint16_t* scales, int64_t M,
+              int64_t K, int64_t N, int32_t group, uint16_t* y, void* stream, int32_t kernel_id,
+              int32_t splits) {
+  int st = check_shape(M, K, N, group);
+  if (st != GPTQ_OK) return st;
+  if (kernel_id < GPTQ_KERNEL_AUTO || kernel_id > GPTQ_KERNEL_PREFILL) return GPTQ_ERR_KERNEL;
+  if (kernel_id == GPTQ_KERNEL_DECODE && M > GPTQ_DECODE_MAX_M) return GPTQ_ERR_KERNEL;
+  if (splits < 0 || splits > 8) return GPTQ_ERR_KERNEL;
+  if (!qweight || !scales) return GPTQ_ERR_NULL;
+  if (M == 0) return GPTQ_OK;
+  if (!x || !y) return GPTQ_ERR_NULL;
+  if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(y))
+    return GPTQ_ERR_ALIGN;
+  const int64_t ybytes = M * N * 2;
+  if (overlaps(y, ybytes, x, M * K * 2) || overlaps(y, ybytes, qweight, K / 8 * N * 4) ||
+      overlaps(y, ybytes, scales, num_groups(K, group) * N * 2))
+    return GPTQ_ERR_ALIAS;
+  const DeviceInfo* dev = nullptr;
+  st = query_device(&dev);
+  if (st != GPTQ_OK) return st;
+  if (kernel_id == GPTQ_KERNEL_AUTO) kernel_id = select_kernel(M, K, N, *dev, nullptr);
+  const int gs = group_shift_of(group);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (kernel_id == GPTQ_KERNEL_DECODE)
+    e = launch_decode(x, qweight, scales, y, M, K, N, gs, splits, s, *dev);
+  else
+    e = launch_prefill(x, qweight, scales, y, M, K, N, gs, s, *dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  return GPTQ_OK;
+}
+
+}  // namespace
+}  // namespace gptq
+
+using namespace gptq;
+
+extern "C" {
+
+int gptq_w4a16_gemm(const uint16_t* x, const int32_t* qweight, const uint16_t* scales, int64_t M,
+                    int64_t K, int64_t N, int32_t group, uint16_t* y, void* stream) {
+  return gemm_impl(x, qweight, scales, M, K, N, group, y, stream, GPTQ_KERNEL_AUTO, 0);
+}
+
+int gptq_w4a16_gemm_kernel(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                           int64_t M, int64_t K, int64_t N, int32_t group, uint16_t* y,
+                           void* stream, int32_t kernel_id) {
+  return gemm_impl(x, qweight, scales, M, K, N, group, y, stream, kernel_id, 0);
+}
+
+int gptq_w4a16_gemm_decode_splits(const uint16_t* x, const int32_t* qweight,
+                                  const uint16_t* scales, int64_t M, int64_t K, int64_t N,
+                                  int32_t group, uint16_t* y, void* stream, int32_t splits) {
+  if (splits < 1) return GPTQ_ERR_KERNEL;
+  return gemm_impl(x, qweight, scales, M, K, N, group, y, stream, GPTQ_KERNEL_DECODE, splits);
+}
+
+int gptq_dequant(const int32_t* qweight, const uint16_t* scales, int64_t K, int64_t N,
+                 int32_t group, uint16_t* w_out, void* stream) {
+  int st = check_shape(0, K, N, group);
+  if (st != GPTQ_OK) return st;
+  if (!qweight || !scales || !w_out) return GPTQ_ERR_NULL;
+  if (!aligned16(qweight) || !aligned16(scales) || !aligned16(w_out)) return GPTQ_ERR_ALIGN;
+  const int64_t wbytes = K * N * 2;
+  if (overlaps(w_out, wbytes, qweight, K / 8 * N * 4) ||
+      overlaps(w_out, wbytes, scales, num_groups(K, group) * N * 2))
+    return GPTQ_ERR_ALIAS;
+  const DeviceInfo* dev = nullptr;
+  st = query_device(&dev);
+  if (st != GPTQ_OK) return st;
+  cudaError_t e = launch_dequant(qweight, scales, K, N, group_shift_of(group), w_out,
+                                 static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  return GPTQ_OK;
+}
+
+int gptq_w4a16_select(int64_t M, int64_t K, int64_t N, int32_t group, int32_t* kernel_id,
+                      int32_t* split_k) {
+  int st = check_shape(M, K, N, group);
+  if (st != GPTQ_OK) return st;
+  const DeviceInfo* dev = nullptr;
+  st = query_device(&dev);
+  if (st != GPTQ_OK) return st;
+  int32_t split = 1;
+  const int k = select_kernel(M, K, N, *dev, &split);
+  if (kernel_id) *kernel_id = k;
+  if (split_k) *split_k = split;
+  return GPTQ_OK;
+}
+
+const char* gptq_status_string(int status) {
+  switch (status) {
+    case GPTQ_OK: return "ok";
+    case GPTQ_ERR_NULL: return "null pointer";
+    case GPTQ_ERR_SHAPE: return "invalid shape (need M >= 0, K > 0 and K % 16 == 0, N > 0 and N % 8 == 0, within the size limits)";
+    case GPTQ_ERR_GROUP: return "unsupported group size (need -1, 16, 32, 64, 128, 256, 512 or 1024)";
+    case GPTQ_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case GPTQ_ERR_DEVICE: return "no current CUDA device of compute capability 10.0";
+    case GPTQ_ERR_CUDA: return "CUDA launch error";
+    case GPTQ_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    case GPTQ_ERR_ALIAS: return "output overlaps an input";
+    case GPTQ_ERR_KERNEL: return "kernel id or split count not valid for this call";
+    default: return "unknown status";
+  }
+}
+
+int gptq_device_error(void) {
+  const DeviceInfo* dev = nullptr;
+  int st = query_device(&dev);
+  if (st != GPTQ_OK) return st;
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  int v = 0;
+  const int zero = 0;
+  if (cudaMemcpy(&v, dev->error_word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(dev->error_word, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  return v;
+}
+
+const char* gptq_version(void) { return "0.1.0"; }
+
+}  // extern "C"

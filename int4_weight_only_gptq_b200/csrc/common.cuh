@@ -1,0 +1,194 @@
+// Device helpers shared by the sm_100a kernels of the W4A16 GPTQ library.
+//
+// The dequantisation primitive follows the layer's definition exactly
+// (GPTQ-Pro README, "Runtime contract": symmetric INT4, zero point 8, FP16):
+// a code q becomes the FP16 value 1024 + q by OR-ing it into the mantissa of
+// 1024.0 (exponent bits 0x6400), (1024 + q) - 1032 = q - 8 is exact, and the
+// product (q - 8) * s is rounded once to FP16 (round to nearest even).  The
+// arithmetic is written with explicit .rn modifiers so that the compiler cannot
+// contract it into a fused multiply-add with a different rounding.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace gptq {
+
+constexpr uint32_t kMagic1024 = 0x64006400u;   // half2(1024, 1024)
+constexpr uint32_t kMinus1032 = 0x64086408u;   // half2(1032, 1032) (subtracted)
+constexpr uint32_t kOneSixteenth = 0x2C002C00u; // half2(1/16, 1/16)
+constexpr uint32_t kMinus72 = 0xD480D480u;      // half2(-72, -72)
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;  // (a & b) | c
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t hsub2_rn(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t hmul2_rn(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t hfma2_rn(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// Eight codes of one qweight word -> four half2 (q - 8), paired (k, k+4):
+//   p[0] = (k0, k4), p[1] = (k1, k5), p[2] = (k2, k6), p[3] = (k3, k7)
+// (low half first).  All four are exact small integers.
+__device__ __forceinline__ void unpack_centered(uint32_t w, uint32_t p[4]) {
+  const uint32_t w8 = w >> 8;  // logical shift: the word is unsigned here
+  p[0] = hsub2_rn(lop3_and_or(w, 0x000F000Fu, kMagic1024), kMinus1032);
+  p[1] = hfma2_rn(lop3_and_or(w, 0x00F000F0u, kMagic1024), kOneSixteenth, kMinus72);
+  p[2] = hsub2_rn(lop3_and_or(w8, 0x000F000Fu, kMagic1024), kMinus1032);
+  p[3] = hfma2_rn(lop3_and_or(w8, 0x00F000F0u, kMagic1024), kOneSixteenth, kMinus72);
+}
+
+// Dequantised weights of one word, paired (k, k+4) as above: one rounding.
+__device__ __forceinline__ void dequant_word_paired(uint32_t w, uint32_t s2, uint32_t p[4]) {
+  unpack_centered(w, p);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) p[j] = hmul2_rn(p[j], s2);
+}
+
+// Same, in natural k order: n[j] = (k_{2j}, k_{2j+1}).
+__device__ __forceinline__ void dequant_word_natural(uint32_t w, uint32_t s2, uint32_t n[4]) {
+  uint32_t p[4];
+  dequant_word_paired(w, s2, p);
+  n[0] = prmt(p[0], p[1], 0x5410);  // (k0, k1)
+  n[1] = prmt(p[2], p[3], 0x5410);  // (k2, k3)
+  n[2] = prmt(p[0], p[1], 0x7632);  // (k4, k5)
+  n[3] = prmt(p[2], p[3], 0x7632);  // (k6, k7)
+}
+
+__device__ __forceinline__ uint32_t half2_broadcast(uint16_t h) {
+  return (uint32_t)h | ((uint32_t)h << 16);
+}
+
+// ---- global loads ----------------------------------------------------------
+
+// Streaming 16-byte load: read-only path, not kept in L1.
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint2 ld_nc_v2(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t ld_nc_u32(const void* p) {
+  uint32_t r;
+  asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint16_t ld_nc_u16(const void* p) {
+  uint16_t r;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));
+  return r;
+}
+
+// ---- warp-level MMA (m16n8k16, FP16 inputs, FP32 accumulate) ------------------
+
+__device__ __forceinline__ void mma_m16n8k16(float d[4], const uint32_t a[4], uint32_t b0,
+                                             uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// ---- shared memory / cluster ------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared variable in another CTA of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// ---- mbarrier (bounded waits) ------------------------------------------------
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbarrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+}  // namespace gptq

@@ -1,0 +1,46 @@
+// Internal interface between the C ABI (api.cu) and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gptq {
+
+struct DeviceInfo {
+  int device = -1;
+  int num_sms = 0;
+  int cc_major = 0;
+  int cc_minor = 0;
+  int smem_optin = 0;   // max dynamic shared memory per block (opt-in)
+  int l2_bytes = 0;
+  int* error_word = nullptr;  // device address of this device's error word
+};
+
+// Error codes written to the device error word (match gptq_status values).
+constexpr int kDeviceErrTimeout = 7;
+
+// log2(group), or 62 for group == -1 (then (8*i) >> 62 == 0 for every row).
+inline int group_shift_of(int32_t group) {
+  if (group == -1) return 62;
+  int s = 0;
+  while ((1 << s) < group) ++s;
+  return s;
+}
+
+cudaError_t launch_dequant(const int32_t* qweight, const uint16_t* scales, int64_t K, int64_t N,
+                           int group_shift, uint16_t* w_out, cudaStream_t stream,
+                           const DeviceInfo& dev);
+
+// Decode (M <= 16).  splits = number of CTAs that share one column block along
+// K (the cluster size, 1..8); 0 picks it from the shape.
+int decode_pick_splits(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev);
+cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                          uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
+                          int splits, cudaStream_t stream, const DeviceInfo& dev);
+
+// Prefill (any M >= 1): TMA + tcgen05 with TMEM accumulators.
+cudaError_t launch_prefill(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                           uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
+                           cudaStream_t stream, const DeviceInfo& dev);
+
+}  // namespace gptq

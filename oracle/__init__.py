@@ -38,8 +38,8 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_LIB_PATH) or \
             os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".{os.getpid()}.tmp"
-        subprocess.run(["gcc", "-O2", "-fno-fast-math", "-std=c11", "-shared", "-fPIC",
-                        "-o", tmp, _SRC, "-lm"], check=True)
+        subprocess.run(["gcc", "-O2", "-fno-fast-math", "-std=c11", "-fopenmp", "-shared",
+                        "-fPIC", "-o", tmp, _SRC, "-lm"], check=True)
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
 
@@ -49,6 +49,8 @@ def _load():
     with _lock:
         if _lib is None:
             lib = ctypes.CDLL(build())
+            lib.oracle_set_threads.argtypes = [ctypes.c_int]
+            lib.oracle_get_threads.restype = ctypes.c_int
             lib.oracle_half_to_double.restype = ctypes.c_double
             lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
             lib.oracle_double_to_half.restype = ctypes.c_uint16
@@ -85,6 +87,15 @@ def _bits16(a):
     if a.dtype == np.float16:
         return a.view(np.uint16)
     return _c(a, np.uint16)
+
+
+def set_threads(n: int) -> None:
+    """Threads used to split independent outputs (results do not change)."""
+    _load().oracle_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(_load().oracle_get_threads())
 
 
 def half_to_double(h: int) -> float:

@@ -24,11 +24,35 @@
  * rounding, closed forms, brute force on tiny shapes, round trips).
  *
  * Every routine here is deliberately plain: one element at a time, no
- * blocking, no vectorisation, no threads.
+ * blocking, no vectorisation; OpenMP threads only split independent outputs.
  */
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Threads split the independent outputs (columns or listed entries) only;
+ * every output's sum over k is still formed by one thread in ascending k, so
+ * the result does not depend on the thread count. */
+void oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+int oracle_get_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
 
 /* ---- IEEE 754-2008 binary16: 1 sign bit, 5 exponent bits (bias 15),
  *      10 fraction bits.  emin = -14, precision p = 11. ---------------------- */
@@ -146,6 +170,7 @@ static uint16_t dequant_at(const int32_t* qweight, const uint16_t* scales,
 void oracle_dequant(const int32_t* qweight, const uint16_t* scales, int64_t K,
                     int64_t N, int32_t group, uint16_t* w)
 {
+    #pragma omp parallel for schedule(static)
     for (int64_t k = 0; k < K; ++k)
         for (int64_t n = 0; n < N; ++n)
             w[k * N + n] = dequant_at(qweight, scales, N, group, k, n);
@@ -160,6 +185,7 @@ int oracle_gemm(const uint16_t* x, const int32_t* qweight, const uint16_t* scale
     uint16_t* w = (uint16_t*)malloc((size_t)(K * N) * sizeof(uint16_t));
     if (!w) return 1;
     oracle_dequant(qweight, scales, K, N, group, w);
+    #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n) {
             double acc = 0.0;
@@ -179,6 +205,7 @@ void oracle_gemm_entries(const uint16_t* x, const int32_t* qweight,
                          const int64_t* ns, double* out)
 {
     (void)M;
+    #pragma omp parallel for schedule(dynamic, 16)
     for (int64_t i = 0; i < count; ++i) {
         int64_t m = ms[i], n = ns[i];
         double acc = 0.0;
@@ -189,18 +216,20 @@ void oracle_gemm_entries(const uint16_t* x, const int32_t* qweight,
     }
 }
 
-/* Y rows ms[0..count) in full: out is binary64 [count, N]. */
+/* Y rows ms[0..count) in full: out is binary64 [count, N].  Column n's
+ * weights are dequantised once and used for every listed row. */
 void oracle_gemm_rows(const uint16_t* x, const int32_t* qweight,
                       const uint16_t* scales, int64_t M, int64_t K, int64_t N,
                       int32_t group, int64_t count, const int64_t* ms, double* out)
 {
     (void)M;
-    for (int64_t n = 0; n < N; ++n)
+    #pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t n = 0; n < N; ++n) {
         for (int64_t i = 0; i < count; ++i) out[i * N + n] = 0.0;
-    for (int64_t k = 0; k < K; ++k)
-        for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
             double w = oracle_half_to_double(dequant_at(qweight, scales, N, group, k, n));
             for (int64_t i = 0; i < count; ++i)
                 out[i * N + n] += oracle_half_to_double(x[ms[i] * K + k]) * w;
         }
+    }
 }

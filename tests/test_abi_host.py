@@ -1,0 +1,121 @@
+"""The C ABI on the host (no GPU needed): the library loads, exports every
+entry point declared in include/*.h, and rejects bad arguments with the right
+status before touching a device.  No call here launches a kernel."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from int4_weight_only_gptq_b200 import binding
+from int4_weight_only_gptq_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load()
+
+
+def declared_entry_points():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names += re.findall(r"GPTQ_API\s+[\w\s\*]*?\b(gptq_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_entry_points()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(binding.EXPORTS)
+
+
+def test_version_and_status_strings(lib):
+    assert binding.version() == "0.1.0"
+    for st in range(10):
+        assert binding.status_string(st)
+    assert binding.status_string(12345) == "unknown status"
+
+
+# fake, aligned device-looking addresses: never dereferenced because every
+# call below fails a host-side check first (or returns early for M == 0)
+X, QW, S, Y = 0x10000, 0x200000, 0x400000, 0x800000
+
+
+def call(lib, x=X, qw=QW, s=S, M=4, K=512, N=256, g=128, y=Y, kernel=None):
+    args = (ctypes.c_void_p(x), ctypes.c_void_p(qw), ctypes.c_void_p(s), M, K, N, g,
+            ctypes.c_void_p(y), None)
+    if kernel is None:
+        return lib.gptq_w4a16_gemm(*args)
+    return lib.gptq_w4a16_gemm_kernel(*args, kernel)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(M=-1), 2), (dict(K=0), 2), (dict(K=-16), 2), (dict(N=0), 2),
+    (dict(K=520), 2), (dict(N=252), 2), (dict(K=16 * (1 << 20) + 16), 2),
+    (dict(N=(1 << 20) + 8), 2), (dict(M=(1 << 23) + 1), 2),
+    (dict(g=0), 3), (dict(g=8), 3), (dict(g=100), 3), (dict(g=2048), 3), (dict(g=-2), 3),
+    (dict(qw=0), 1), (dict(s=0), 1), (dict(x=0), 1), (dict(y=0), 1),
+    (dict(x=X + 2), 4), (dict(qw=QW + 4), 4), (dict(s=S + 8), 4), (dict(y=Y + 2), 4),
+    (dict(y=X), 8), (dict(y=QW + 16), 8), (dict(y=S), 8),
+    (dict(kernel=3), 9), (dict(kernel=-1), 9), (dict(kernel=1, M=17), 9),
+])
+def test_gemm_argument_checks(lib, kw, status):
+    assert call(lib, **kw) == status
+
+
+def test_empty_m_is_a_no_op(lib):
+    # M == 0: success without a device and without x / y
+    assert call(lib, M=0, x=0, y=0) == 0
+    assert call(lib, M=0, x=0, y=0, kernel=2) == 0
+
+
+def test_no_device_is_reported(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert call(lib) == 5
+    k, s = ctypes.c_int32(), ctypes.c_int32()
+    assert lib.gptq_w4a16_select(1, 512, 256, 128, ctypes.byref(k), ctypes.byref(s)) == 5
+
+
+def test_dequant_and_select_checks(lib):
+    v = ctypes.c_void_p
+    assert lib.gptq_dequant(v(QW), v(S), 520, 256, 128, v(Y), None) == 2
+    assert lib.gptq_dequant(v(QW), v(S), 512, 256, 7, v(Y), None) == 3
+    assert lib.gptq_dequant(None, v(S), 512, 256, 128, v(Y), None) == 1
+    assert lib.gptq_dequant(v(QW), v(S), 512, 256, 128, None, None) == 1
+    assert lib.gptq_dequant(v(QW), v(S), 512, 256, 128, v(Y + 2), None) == 4
+    assert lib.gptq_dequant(v(QW), v(S), 512, 256, 128, v(QW), None) == 8
+    assert lib.gptq_w4a16_select(1, 512, 250, 128, None, None) == 2
+    assert lib.gptq_w4a16_select(1, 512, 256, 3, None, None) == 3
+    assert lib.gptq_w4a16_gemm_decode_splits(v(X), v(QW), v(S), 1, 512, 256, 128, v(Y),
+                                             None, 0) == 9
+    assert lib.gptq_w4a16_gemm_decode_splits(v(X), v(QW), v(S), 1, 512, 256, 128, v(Y),
+                                             None, 9) == 9
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 512, dtype=torch.float16)
+    qw = torch.zeros(64, 256, dtype=torch.int32)
+    s = torch.zeros(4, 256, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        binding.gemm(x, qw, s, 128)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="not built"):
+        binding.load.__wrapped__ if hasattr(binding.load, "__wrapped__") else None
+        saved = binding._lib
+        binding._lib = None
+        try:
+            binding.load(str(tmp_path / "nope.so"))
+        finally:
+            binding._lib = saved

@@ -1,0 +1,254 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bars (written here):
+  * dequantised weights: bit-exact;
+  * Y: max |y_gpu - y_ref| / (1 + |y_ref|) <= 1e-2 against the binary64
+    oracle, and every reported error is printed;
+  * integer work that floating point cannot blur (one-hot X, all codes 8,
+    integer-exact inputs): bitwise equal;
+  * determinism: two runs give bitwise-identical Y.
+Full-size problems are compared on sampled rows (every column of those rows).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from int4_weight_only_gptq_b200 import binding as B
+from int4_weight_only_gptq_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from int4_weight_only_gptq_b200.build import build
+    build()
+    B.load()
+    assert B.device_error() == 0
+    yield
+    assert B.device_error() == 0
+
+
+def dev(p):
+    x = torch.from_numpy(p.x.view(np.int16)).view(torch.float16).cuda()
+    qw = torch.from_numpy(p.qweight).cuda()
+    s = torch.from_numpy(p.scales.view(np.int16)).view(torch.float16).cuda()
+    return x, qw, s
+
+
+def rel_err(y_gpu, y_ref):
+    y = y_gpu.astype(np.float64)
+    return float(np.max(np.abs(y - y_ref) / (1.0 + np.abs(y_ref)))) if y.size else 0.0
+
+
+def run(p, kernel=B.KERNEL_AUTO, splits=0):
+    x, qw, s = dev(p)
+    y = B.gemm(x, qw, s, p.group, kernel=kernel, decode_splits=splits)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+def check_rows(p, y, rows, label):
+    ref = oracle.gemm_rows(p.x, p.qweight, p.scales, p.group, rows)
+    err = rel_err(y[rows], ref)
+    print(f"[parity] {label}: max rel err {err:.3e} over {len(rows)} rows x {p.N} cols")
+    assert np.all(np.isfinite(y[rows]))
+    assert err <= TOL, f"{label}: {err}"
+    return err
+
+
+def sample_rows(M, n=4, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = {0, M - 1}
+    rows.update(int(r) for r in rng.integers(0, M, size=max(0, n - 2)))
+    return sorted(rows)
+
+
+# ---- dequantisation: bit-exact ----------------------------------------------
+
+@pytest.mark.parametrize("K,N,G", [(512, 256, 128), (528, 24, 128), (64, 8, 16), (48, 40, 32),
+                                   (5120, 5120, -1), (1024, 136, 1024), (160, 64, 64)])
+def test_dequant_bit_exact(K, N, G):
+    p = W.make_problem(1, K, N, G, seed=K + N)
+    _, qw, s = dev(p)
+    w = B.dequant(qw, s, G)
+    torch.cuda.synchronize()
+    ref = oracle.dequant(p.qweight, p.scales, G)
+    assert np.array_equal(w.cpu().numpy().view(np.uint16), ref.view(np.uint16))
+
+
+def test_dequant_bit_exact_full_size_up_projection():
+    p = W.decode_up()
+    _, qw, s = dev(p)
+    w = B.dequant(qw, s, p.group).cpu().numpy()
+    ref = oracle.dequant(p.qweight, p.scales, p.group)
+    assert np.array_equal(w.view(np.uint16), ref.view(np.uint16))
+
+
+def test_dequant_every_code_and_scale():
+    """All 16 codes x every finite FP16 scale, bit-exact."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    bits = bits[(bits & 0x7C00) != 0x7C00]
+    N = (bits.size // 8) * 8
+    scales = bits[:N].view(np.float16).reshape(1, N)
+    qw = np.empty((2, N), dtype=np.int32)
+    qw[0] = np.int32(0x76543210)
+    qw[1] = np.uint32(0xFEDCBA98).view(np.int32)
+    w = B.dequant(torch.from_numpy(qw).cuda(),
+                  torch.from_numpy(scales.view(np.int16)).view(torch.float16).cuda(), -1)
+    ref = oracle.dequant(qw, scales, -1)
+    assert np.array_equal(w.cpu().numpy().view(np.uint16), ref.view(np.uint16))
+
+
+# ---- the GEMM on the tiny workload, both kernels ----------------------------
+
+@pytest.mark.parametrize("M", [1, 4])
+@pytest.mark.parametrize("kernel", [B.KERNEL_AUTO, B.KERNEL_DECODE, B.KERNEL_PREFILL])
+def test_tiny(M, kernel):
+    p = W.tiny(M)
+    y = run(p, kernel)
+    ref = oracle.gemm(p.x, p.qweight, p.scales, p.group)
+    err = rel_err(y, ref)
+    print(f"[parity] tiny M={M} kernel={kernel}: max rel err {err:.3e}")
+    assert err <= TOL
+
+
+# ---- ragged and edge shapes -----------------------------------------------
+
+EDGE = [  # (M, K, N, G)
+    (1, 16, 8, -1), (3, 48, 40, 16), (5, 528, 24, 128), (7, 96, 72, 32), (8, 160, 264, 64),
+    (9, 64, 8, 16), (13, 1040, 136, 1024), (16, 272, 520, 16), (2, 5120, 8, 512),
+]
+
+
+@pytest.mark.parametrize("M,K,N,G", EDGE)
+@pytest.mark.parametrize("kernel", [B.KERNEL_DECODE, B.KERNEL_PREFILL])
+def test_edge_shapes_small_m(M, K, N, G, kernel):
+    p = W.make_problem(M, K, N, G, seed=M * 7 + K + N)
+    y = run(p, kernel)
+    ref = oracle.gemm(p.x, p.qweight, p.scales, G)
+    err = rel_err(y, ref)
+    print(f"[parity] edge M={M} K={K} N={N} G={G} kernel={kernel}: {err:.3e}")
+    assert err <= TOL
+
+
+@pytest.mark.parametrize("M,K,N,G", [(17, 64, 8, 16), (129, 528, 136, 128), (300, 96, 264, 32),
+                                     (257, 1040, 128, -1), (513, 160, 392, 64)])
+def test_edge_shapes_prefill(M, K, N, G):
+    p = W.make_problem(M, K, N, G, seed=M + K + N)
+    y = run(p)
+    ref = oracle.gemm(p.x, p.qweight, p.scales, G)
+    err = rel_err(y, ref)
+    print(f"[parity] prefill M={M} K={K} N={N} G={G}: {err:.3e}")
+    assert err <= TOL
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_decode_every_split(splits):
+    p = W.make_problem(6, 2048, 200, 32, seed=splits)
+    y = run(p, splits=splits)
+    ref = oracle.gemm(p.x, p.qweight, p.scales, 32)
+    assert rel_err(y, ref) <= TOL
+
+
+# ---- closed forms and exact cases -----------------------------------------
+
+@pytest.mark.parametrize("kernel", [B.KERNEL_DECODE, B.KERNEL_PREFILL])
+def test_all_codes_eight_gives_exact_zero(kernel):
+    p = W.make_problem(16, 512, 256, 128, seed=3)
+    p.qweight[:] = np.uint32(0x88888888).view(np.int32)
+    y = run(p, kernel)
+    assert np.all(y.astype(np.float64) == 0.0)
+
+
+@pytest.mark.parametrize("kernel", [B.KERNEL_DECODE, B.KERNEL_PREFILL])
+def test_one_hot_x_reproduces_dequantised_rows_bitwise(kernel):
+    p = W.make_problem(16, 1024, 264, 32, seed=4)
+    ks = [0, 1, 7, 8, 100, 511, 512, 777, 1000, 1023, 64, 65, 3, 300, 900, 31]
+    p.x[:] = 0
+    for m, k in enumerate(ks):
+        p.x[m, k] = 1
+    y = run(p, kernel)
+    w = oracle.dequant(p.qweight, p.scales, 32)
+    for m, k in enumerate(ks):
+        assert np.array_equal(y[m].view(np.uint16), w[k].view(np.uint16)), (m, k)
+
+
+@pytest.mark.parametrize("kernel", [B.KERNEL_DECODE, B.KERNEL_PREFILL])
+@pytest.mark.parametrize("M", [1, 5, 16])
+def test_integer_exact_inputs_match_bitwise(kernel, M):
+    """x in {-4..4}, scales 2^-6: every product and partial sum is exact in
+    FP32, so any summation order gives the oracle's value exactly."""
+    rng = np.random.default_rng(M)
+    p = W.make_problem(M, 2048, 136, 64, seed=M)
+    p.x[:] = rng.integers(-4, 5, size=p.x.shape).astype(np.float16)
+    p.scales[:] = np.float16(2.0 ** -6)
+    y = run(p, kernel)
+    ref = oracle.round_to_half(oracle.gemm(p.x, p.qweight, p.scales, 64))
+    assert np.array_equal(y.view(np.uint16), ref.view(np.uint16))
+
+
+@pytest.mark.parametrize("kernel,M", [(B.KERNEL_DECODE, 1), (B.KERNEL_DECODE, 16),
+                                      (B.KERNEL_PREFILL, 300)])
+def test_deterministic(kernel, M):
+    p = W.make_problem(M, 5120, 1024, 128, seed=9)
+    a, b = run(p, kernel), run(p, kernel)
+    assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+
+
+def test_empty_m():
+    p = W.make_problem(1, 512, 256, 128)
+    _, qw, s = dev(p)
+    x = torch.empty((0, 512), dtype=torch.float16, device="cuda")
+    y = B.gemm(x, qw, s, 128)
+    assert y.shape == (0, 256)
+
+
+def test_maximum_k_and_n():
+    p = W.make_problem(2, 1 << 20, 8, 1024, seed=11)
+    y = run(p, B.KERNEL_DECODE)
+    check_rows(p, y, [0, 1], "max K decode")
+    y = run(p, B.KERNEL_PREFILL)
+    check_rows(p, y, [0, 1], "max K prefill")
+    q = W.make_problem(1, 16, 1 << 20, -1, seed=12)
+    y = run(q)
+    ref = oracle.gemm(q.x, q.qweight, q.scales, -1)
+    assert rel_err(y, ref) <= TOL
+
+
+# ---- the workloads at full size (sampled rows, every column) --------------------
+
+def test_decode_up_projection_full():
+    p = W.decode_up()
+    assert B.select(1, 5120, 17408, 128)[0] == B.KERNEL_DECODE
+    check_rows(p, run(p), [0], "decode up-projection M=1")
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 16])
+def test_decode_down_projection_sweep(M):
+    p = W.decode_down(M)
+    assert B.select(M, 17408, 5120, 32)[0] == B.KERNEL_DECODE
+    check_rows(p, run(p), sample_rows(M, 3), f"decode down-projection M={M}")
+
+
+@pytest.mark.parametrize("M", [512, 2048, 8192])
+def test_prefill_full(M):
+    p = W.prefill(M)
+    assert B.select(M, 5120, 17408, 128)[0] == B.KERNEL_PREFILL
+    check_rows(p, run(p), sample_rows(M, 3), f"prefill M={M}")
+
+
+@pytest.mark.parametrize("G", W.GROUP_SIZES)
+@pytest.mark.parametrize("M", [1, 16, 4096])
+def test_group_sweep(G, M):
+    p = W.group_sweep(G, M)
+    check_rows(p, run(p), sample_rows(M, 2), f"square G={G} M={M}")
+
+
+@pytest.mark.parametrize("which", [n for n, _, _, _ in W.LAYER_LINEARS])
+@pytest.mark.parametrize("M", [1, 16, 4096])
+def test_layer_linears(which, M):
+    p = W.layer_linear(which, M)
+    check_rows(p, run(p), sample_rows(M, 2), f"layer {which} M={M}")
