@@ -65,7 +65,7 @@ typedef enum {
 #define GPTQ_KERNEL_PREFILL 2  /* any M: TMA + tcgen05 MMA with TMEM accumulators  */
 
 /* Size limits (inclusive). */
-#define GPTQ_MAX_K 1048576
+#define GPTQ_MAX_K 65536
 #define GPTQ_MAX_N 1048576
 #define GPTQ_MAX_M 8388608
 #define GPTQ_DECODE_MAX_M 16

@@ -9,7 +9,7 @@
 
 #include <mutex>
 
-#include "../../include/gptq_w4a16.h"
+#include "gptq_w4a16.h"
 #include "kernels.h"
 
 namespace gptq {

@@ -2,246 +2,450 @@
 //
 // Operation: GPTQ-Pro README, "Runtime contract" and "Ampere kernel
 // architecture" (fused small-M decode that reads the native int32 qweight,
-// keeps scales close, and reduces split-K partial sums deterministically).
+// keeps scales resident, and reduces split-K partial sums deterministically).
 // The Ampere design (four-warp output tiles, M <= 4) is prior art only; this
-// kernel is laid out for sm_100a:
+// kernel is laid out for sm_100a, where a memory-bound kernel is limited by
+// the bytes it keeps in flight:
 //
-// * Work unit: a "row quad" (four packed rows = 32 k) by 32 or 64 columns per
-//   warp.  Lane (q = lane/4, c = lane%4) loads the 16-byte qweight vector of
-//   packed row 4r+c, columns n + 4q .. n + 4q + 3: for each c the eight lanes
-//   read 128 contiguous bytes, so every warp load is four full 128-byte lines.
-// * The eight codes of a word are unpacked in registers straight into the
-//   A fragment of mma.m16n8k16 (weights as A: 16 columns x 16 k; X as B:
-//   16 k x 8 tokens).  The k order inside one MMA does not change the sum as
-//   long as X uses the same order, so the natural (k, k+4) pairs of the
-//   magic-number unpack are used as they come and X is permuted to match with
-//   two byte-permutes per register.  Weights are the exact FP16 dequantised
-//   values (one rounding), accumulation is FP32 on the tensor cores, which
-//   keeps the CUDA-core work per weight to a handful of ALU operations.
-// * Split-K: the eight warps of a CTA take consecutive K ranges of the same
-//   columns; `splits` CTAs of a thread-block cluster take consecutive K ranges
-//   of the same column block.  Partial sums are reduced in a fixed order
-//   through shared memory and then distributed shared memory, so results are
-//   bitwise reproducible and no global scratch is needed.
+// * A CTA owns 64 output columns and a range of K.  One producer thread
+//   streams, per stage (32 packed rows = 256 k), two TMA boxes of qweight
+//   (32 columns x 32 rows each, stored with the 128-byte swizzle), one box of
+//   the scale rows the stage needs and the X rows (bulk copies, 576-byte
+//   pitch) into an S-stage ring in shared memory, so tens of KB per SM are in
+//   flight without holding registers.
+// * Eight consumer warps: two column slices of 32 x four stage phases.  A
+//   lane (q = lane/4, c = lane%4) reads the 16-byte vector of packed row 4j+c
+//   at column chunk chunk_of(q) of its slice (a permutation of the chunks
+//   that makes the eight lanes of every quarter-warp hit distinct banks
+//   through the swizzle) and feeds mma.m16n8k16 with the weights
+//   as A (16 columns x 16 k) and X as B (16 k x 8 tokens).  Which k sits in
+//   which MMA slot does not change the sum as long as X uses the same order,
+//   so the (k, k+4) pairs of the magic-number unpack are used as they come and
+//   X is permuted to match with byte permutes.
+// * Each weight is dequantised exactly as defined, fp16((q - 8) * s): 1024 + q
+//   by a LOP3 into the FP16 mantissa of 1024, minus 1032 (exact), times the
+//   group scale (one rounding).  Keeping the definition's per-weight rounding
+//   matters: on inputs with large activation outliers, skipping it (scaling
+//   FP32 partial sums per group instead) moves Y by up to ~1e-2 relative.  The
+//   scale vector of a lane is loaded and broadcast once per run of rows that
+//   share a group.
+// * Split-K: the four stage phases of a CTA and the `splits` CTAs of a
+//   thread-block cluster (consecutive K ranges of the same columns) are
+//   reduced in a fixed order through shared memory and distributed shared
+//   memory: bitwise reproducible, no global scratch.
+// * Programmatic dependent launch: before waiting for the previous kernel in
+//   the stream, the producer only prefetches its first weight rows into L2 (a
+//   prefetch cannot observe stale data); every copy into shared memory and
+//   every store of Y happens after the wait.
+// * Every mbarrier wait is bounded in time; on expiry the kernel records
+//   GPTQ_ERR_TIMEOUT in the device error word and winds down.
 //
 // Bytes per call: K*N/2 (qweight) + n_groups*N*2 (scales) + M*K*2 + M*N*2.
 #include <cuda_runtime.h>
 
-#include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc05.cuh"
+#include "tmap.h"
 
 namespace gptq {
 
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
+constexpr int WC = 64;                 // output columns per CTA
+constexpr int RB = 32;                 // packed rows (32 x 8 = 256 k) per stage
+constexpr int RQ_STAGE = RB / 4;       // row quads per stage
+constexpr int QW_SLICE = 32 * RB * 4;  // one 32-column slice of a stage: 4 KB, 128-B swizzled
+constexpr int X_PITCH = RB * 16 + 64;  // 576 B: 36 x 16 B, = 4 mod 8 units
+constexpr int S_PITCH = WC * 2;        // 128 B per scale row
+constexpr int kConsumerWarps = 8;      // 2 slices x 4 phases
+constexpr int kPhases = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kMaxStages = 8;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
-template <int TT, int WCV>
-struct DecodeFrag {
-  uint4 w[WCV];   // qweight words, columns col[v] .. col[v] + 3
-  uint2 s[WCV];   // their scales (four halves)
-  uint4 xv[TT];   // X[token q + 8 tt][8 i .. 8 i + 7]
+struct DecodeShape {
+  int stage_bytes;   // qweight + scales + X of one stage (1024-aligned)
+  int qw_off, s_off, x_off;
+  int scale_rows;    // scale rows per stage (the scale box height)
+  int stages;        // ring depth
+  int smem_bytes;    // whole dynamic allocation
 };
 
-// TT: token tiles of 8 (1: M <= 8, 2: M <= 16); WCV: 16-byte column vectors per
-// lane (columns per CTA = 32 * WCV).
-template <int TT, int WCV>
-__global__ void __launch_bounds__(kThreads, 2)
-    decode_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ qweight,
-                  const uint16_t* __restrict__ scales, uint16_t* __restrict__ y, int M, int K,
-                  int N, int group_shift) {
-  constexpr int WC = 32 * WCV;
-  constexpr int TOK = 8 * TT;
-  constexpr int RED_STRIDE = WC + 4;
-  __shared__ float red[kWarps][TOK][RED_STRIDE];
-  __shared__ float part[TOK * WC];
+__host__ __device__ inline int align128(int v) { return (v + 127) & ~127; }
+__host__ __device__ inline int align1024(int v) { return (v + 1023) & ~1023; }
+
+// Scale rows one 256-k stage touches.
+__host__ __device__ inline int scale_rows_per_stage(int group_shift) {
+  return group_shift >= 8 ? 1 : (256 >> group_shift);
+}
+
+inline DecodeShape decode_shape(int M, int group_shift) {
+  DecodeShape d;
+  d.qw_off = 0;
+  d.scale_rows = scale_rows_per_stage(group_shift);
+  d.s_off = 2 * QW_SLICE;
+  d.x_off = d.s_off + align128(d.scale_rows * S_PITCH);
+  d.stage_bytes = align1024(d.x_off + M * X_PITCH);
+  // ring: as deep as fits in ~72 KB (three CTAs per SM for M <= 8, two
+  // otherwise), at least 4 stages
+  int s = ((M <= 8 ? 72 : 96) * 1024) / d.stage_bytes;
+  d.stages = s < 4 ? 4 : (s > kMaxStages ? kMaxStages : s);
+  const int barriers = 256;
+  d.smem_bytes = 1024 + d.stages * d.stage_bytes + barriers;
+  return d;
+}
+
+struct DecodeBars {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  int abort_flag;
+};
+
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+
+// Column chunk (of four) a lane reads: conflict-free against the 128-byte
+// swizzle for the eight lanes of each quarter-warp.
+__device__ __forceinline__ int chunk_of(int q) { return (q >> 1) + 4 * (q & 1); }
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(addr));
+  return r;
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 r;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
+  return r;
+}
+
+__device__ __forceinline__ void record_timeout(int* err, volatile int* abort_flag) {
+  atomicExch(err, kDeviceErrTimeout);
+  *abort_flag = 1;
+}
+
+// TT: token tiles of 8 (1: M <= 8, 2: M <= 16).  STAGE_SCALE: the whole
+// 256-k stage lies in one group (groups >= 256 or -1), so a warp loads its
+// scales once per stage; otherwise once per row quad (with group 16 each
+// lane's own row picks its group).
+template <int TT, bool STAGE_SCALE>
+__global__ void __launch_bounds__(kThreads, TT == 1 ? 3 : 2)
+    decode_kernel(const __grid_constant__ CUtensorMap qw_map,
+                  const __grid_constant__ CUtensorMap s_map, const uint16_t* __restrict__ x,
+                  uint16_t* __restrict__ y, int M, int K, int N, int group_shift, int stages,
+                  int stage_bytes, int s_off, int x_off, int scale_rows, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  DecodeBars* bar = reinterpret_cast<DecodeBars*>(smem + stages * stage_bytes);
+  volatile int* abort_flag = &bar->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q = lane >> 2, c = lane & 3;
   const int n_blk = blockIdx.x * WC;
+  const int ncols = min(WC, N - n_blk);          // multiple of 8
+  const int P = K >> 3;
+  const int NS = (P + RB - 1) / RB;              // stages over all of K
   const int splits = gridDim.y;
-  const int P = K >> 3;                 // packed rows
-  const int RQ = (P + 3) >> 2;          // row quads (the last may be half full)
-  const int split = blockIdx.y * kWarps + warp;
-  const int S = splits * kWarps;
-  const int rq_begin = (int)((int64_t)split * RQ / S);
-  const int rq_end = (int)((int64_t)(split + 1) * RQ / S);
+  const int st_begin = (int)((int64_t)blockIdx.y * NS / splits);
+  const int st_end = (int)((int64_t)(blockIdx.y + 1) * NS / splits);
+  const int n_st = st_end - st_begin;
 
-  int col[WCV];
-  bool col_ok[WCV];
-#pragma unroll
-  for (int v = 0; v < WCV; ++v) {
-    col[v] = n_blk + 32 * v + 4 * q;
-    col_ok[v] = col[v] < N;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&bar->full[s], 1);
+      mbar_init(&bar->empty[s], kConsumerWarps);  // every consumer warp reads every stage
+    }
+    bar->abort_flag = 0;
+    fence_mbarrier_init();
   }
+  if (warp == kConsumerWarps && lane == 0) {
+    prefetch_tensormap(&qw_map);
+    prefetch_tensormap(&s_map);
+    // L2 prefetch of the first stages' weight boxes: safe before the wait
+    const int pf = min(n_st, 4);
+    for (int t = 0; t < pf; ++t) {
+      tma_prefetch_l2_2d(&qw_map, n_blk, (st_begin + t) * RB);
+      tma_prefetch_l2_2d(&qw_map, n_blk + 32, (st_begin + t) * RB);
+    }
+  }
+  __syncthreads();
+  grid_dependency_wait();
 
-  float acc[WCV][2][TT][4];
+  if (warp == kConsumerWarps) {
+    // ---------------- producer (one lane) ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int t = 0; t < n_st; ++t) {
+        const int s = t % stages;
+        const uint32_t ph = (uint32_t)(t / stages) & 1u;
+        if (!mbar_wait_bounded(&bar->empty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
+          record_timeout(err, abort_flag);
+          break;
+        }
+        uint8_t* st = smem + s * stage_bytes;
+        const int r0 = (st_begin + t) * RB;
+        const int nrows = min(RB, P - r0);
+        const int g0 = (int)(((int64_t)r0 * 8) >> group_shift);
+        const uint32_t bytes =
+            (uint32_t)(2 * QW_SLICE + scale_rows * S_PITCH + M * nrows * 16);
+        mbar_arrive_expect_tx(&bar->full[s], bytes);
+        tma_load_2d(st, &qw_map, n_blk, r0, &bar->full[s]);
+        tma_load_2d(st + QW_SLICE, &qw_map, n_blk + 32, r0, &bar->full[s]);
+        tma_load_2d(st + s_off, &s_map, n_blk, g0, &bar->full[s]);
+        for (int m = 0; m < M; ++m)
+          bulk_g2s(st + x_off + m * X_PITCH, x + (int64_t)m * K + (int64_t)r0 * 8,
+                   (uint32_t)nrows * 16, &bar->full[s]);
+        ++issued;
+      }
+      if (*abort_flag) {
+        // wind down: wait (bounded) for the copies still landing in the ring
+        int never = 0;
+        for (int t = issued - 1; t >= 0 && t >= issued - stages; --t)
+          mbar_wait_bounded(&bar->full[t % stages], (uint32_t)(t / stages) & 1u, &never,
+                            200000000ull);
+      }
+      // all of this CTA's copies are issued: the next kernel in the stream may
+      // start its prologue (it waits for this grid before touching its inputs)
+      allow_dependent_launch();
+    }
+  } else {
+    // ---------------- consumers ----------------
+    // warp w: column slice w & 1, row quads p and p + 4 of every stage
+    // (p = w >> 1), so all eight warps share each stage and at most a stage or
+    // two of the ring is held while the rest keeps loading
+    const int slice = warp & 1;
+    const int phase = warp >> 1;
+    const int q = lane >> 2, c = lane & 3;
+    const int chunk = chunk_of(q);
+    // byte offsets, inside a 128-byte swizzled row, of this lane's chunk in
+    // rows with (row & 7) = c (even row quads) and c + 4 (odd row quads)
+    const uint32_t off_even = (uint32_t)((chunk ^ c) << 4);
+    const uint32_t off_odd = (uint32_t)((chunk ^ (c + 4)) << 4);
+    bool x_ok[TT];
 #pragma unroll
-  for (int v = 0; v < WCV; ++v)
+    for (int tt = 0; tt < TT; ++tt) x_ok[tt] = q + 8 * tt < M;
+
+    float acc[2][TT][4];
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
       for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[v][mt][tt][e] = 0.f;
+        for (int e = 0; e < 4; ++e) acc[mt][tt][e] = 0.f;
 
-  auto fetch = [&](int r, DecodeFrag<TT, WCV>& f) {
-    const int i = 4 * r + c;
-    const bool row_ok = i < P;
-    const int64_t g = ((int64_t)i * 8) >> group_shift;
-#pragma unroll
-    for (int v = 0; v < WCV; ++v) {
-      if (row_ok && col_ok[v]) {
-        f.w[v] = ld_stream_v4(qweight + (int64_t)i * N + col[v]);
-        f.s[v] = ld_nc_v2(scales + g * N + col[v]);
-      } else {
-        f.w[v] = make_uint4(0, 0, 0, 0);
-        f.s[v] = make_uint2(0, 0);
+    bool ok = true;
+    for (int t = 0; t < n_st; ++t) {
+      const int s = t % stages;
+      const uint32_t ph = (uint32_t)(t / stages) & 1u;
+      ok = mbar_wait_bounded(&bar->full[s], ph, abort_flag, kWaitLimitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) record_timeout(err, abort_flag);
+        break;
       }
-    }
+      const uint32_t st = smem_u32(smem + s * stage_bytes);
+      const int nrows = min(RB, P - (st_begin + t) * RB);
+      const uint32_t qw_lane = st + slice * QW_SLICE + c * 128;  // row 4j + c: + 512 j
+      const uint32_t s_lane = st + s_off + slice * 64 + chunk * 8;
+      uint32_t x_lane[TT];
 #pragma unroll
-    for (int tt = 0; tt < TT; ++tt) {
-      const int tok = q + 8 * tt;
-      if (row_ok && tok < M)
-        f.xv[tt] = ld_nc_v4(x + (int64_t)tok * K + (int64_t)i * 8);
-      else
-        f.xv[tt] = make_uint4(0, 0, 0, 0);
-    }
-  };
+      for (int tt = 0; tt < TT; ++tt) x_lane[tt] = st + x_off + (q + 8 * tt) * X_PITCH + c * 16;
+      uint32_t s2[4] = {0u, 0u, 0u, 0u};
 
-  auto compute = [&](const DecodeFrag<TT, WCV>& f) {
-    uint32_t bx[TT][4];
+      // One row quad: 32 k x this lane's four columns, eight tokens per tile.
+      auto row_quad = [&](int j, bool full, bool first) {
+        const int row = 4 * j + c;
+        const bool row_ok = full || row < nrows;
+        if (!STAGE_SCALE || first) {
+          // the stage starts on a 256-k boundary, so the scale row of this
+          // lane's row is (8 row) >> log2(group) within the stage's box; rows
+          // past the end read a valid scale row and meet x = 0
+          const int gl = row_ok ? ((row << 3) >> group_shift) : 0;
+          const uint2 sv = lds64(s_lane + gl * S_PITCH);
+          s2[0] = prmt(sv.x, sv.x, 0x1010);
+          s2[1] = prmt(sv.x, sv.x, 0x3232);
+          s2[2] = prmt(sv.y, sv.y, 0x1010);
+          s2[3] = prmt(sv.y, sv.y, 0x3232);
+        }
+        const uint4 w4 = lds128(qw_lane + 512 * j + ((j & 1) ? off_odd : off_even));
+        uint32_t bx[TT][4];
 #pragma unroll
-    for (int tt = 0; tt < TT; ++tt) {
-      bx[tt][0] = prmt(f.xv[tt].x, f.xv[tt].z, 0x5410);  // (x0, x4)
-      bx[tt][1] = prmt(f.xv[tt].x, f.xv[tt].z, 0x7632);  // (x1, x5)
-      bx[tt][2] = prmt(f.xv[tt].y, f.xv[tt].w, 0x5410);  // (x2, x6)
-      bx[tt][3] = prmt(f.xv[tt].y, f.xv[tt].w, 0x7632);  // (x3, x7)
-    }
+        for (int tt = 0; tt < TT; ++tt) {
+          const uint4 xv = (row_ok && x_ok[tt]) ? lds128(x_lane[tt] + 64 * j)
+                                                : make_uint4(0, 0, 0, 0);
+          bx[tt][0] = prmt(xv.x, xv.z, 0x5410);  // (x0, x4)
+          bx[tt][1] = prmt(xv.x, xv.z, 0x7632);  // (x1, x5)
+          bx[tt][2] = prmt(xv.y, xv.w, 0x5410);  // (x2, x6)
+          bx[tt][3] = prmt(xv.y, xv.w, 0x7632);  // (x3, x7)
+        }
+        const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-    for (int v = 0; v < WCV; ++v) {
-      const uint32_t words[4] = {f.w[v].x, f.w[v].y, f.w[v].z, f.w[v].w};
-      const uint32_t s01 = f.s[v].x, s23 = f.s[v].y;
-      const uint32_t s2[4] = {prmt(s01, s01, 0x1010), prmt(s01, s01, 0x3232),
-                              prmt(s23, s23, 0x1010), prmt(s23, s23, 0x3232)};
-      uint32_t p[4][4];
+        for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) dequant_word_paired(words[j], s2[j], p[j]);
+          for (int kk = 0; kk < 2; ++kk) {
+            // column slots q (word 2mt) and q + 8 (word 2mt+1); MMA kk takes
+            // the codes of bytes 0/2 (kk = 0) or 1/3 (kk = 1) of each word
+            const uint32_t wa = kk ? (wd[2 * mt] >> 8) : wd[2 * mt];
+            const uint32_t wb = kk ? (wd[2 * mt + 1] >> 8) : wd[2 * mt + 1];
+            uint32_t a[4];
+            a[0] = hmul2_rn(hsub2_rn(lop3_and_or(wa, 0x000F000Fu, kMagic1024), kMinus1032),
+                            s2[2 * mt]);
+            a[1] = hmul2_rn(hsub2_rn(lop3_and_or(wb, 0x000F000Fu, kMagic1024), kMinus1032),
+                            s2[2 * mt + 1]);
+            a[2] = hmul2_rn(
+                hfma2_rn(lop3_and_or(wa, 0x00F000F0u, kMagic1024), kOneSixteenth, kMinus72),
+                s2[2 * mt]);
+            a[3] = hmul2_rn(
+                hfma2_rn(lop3_and_or(wb, 0x00F000F0u, kMagic1024), kOneSixteenth, kMinus72),
+                s2[2 * mt + 1]);
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        const int a = 2 * mt, b = 2 * mt + 1;  // column slots q and q + 8
+            for (int tt = 0; tt < TT; ++tt)
+              mma_m16n8k16(acc[mt][tt], a, bx[tt][2 * kk], bx[tt][2 * kk + 1]);
+          }
+        }
+      };
+
+      if (nrows == RB) {
 #pragma unroll
-        for (int st = 0; st < 2; ++st) {
-          const uint32_t afrag[4] = {p[a][2 * st], p[b][2 * st], p[a][2 * st + 1],
-                                     p[b][2 * st + 1]};
-#pragma unroll
-          for (int tt = 0; tt < TT; ++tt)
-            mma_m16n8k16(acc[v][mt][tt], afrag, bx[tt][2 * st], bx[tt][2 * st + 1]);
+        for (int i = 0; i < RQ_STAGE / kPhases; ++i) row_quad(phase + kPhases * i, true, i == 0);
+      } else {
+#pragma unroll 1
+        for (int i = 0; i < RQ_STAGE / kPhases; ++i) {
+          const int j = phase + kPhases * i;
+          if (4 * j < nrows) row_quad(j, false, i == 0);
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->empty[s]);
     }
-  };
 
-  if (rq_begin < rq_end) {
-    DecodeFrag<TT, WCV> cur, nxt;
-    fetch(rq_begin, cur);
-    for (int r = rq_begin; r < rq_end; ++r) {
-      if (r + 1 < rq_end) fetch(r + 1, nxt);
-      compute(cur);
-      cur = nxt;
-    }
-  }
-
-  // Accumulator (v, mt, tt, e) holds column slot q (+8 for e >= 2) and token
-  // 2c + (e & 1) of its tile; slot q maps to column 4q + 2mt, slot q + 8 to
-  // column 4q + 2mt + 1 within vector v.
-#pragma unroll
-  for (int v = 0; v < WCV; ++v)
+    // stash this warp's partial tile (reusing the ring: every stage consumed)
+    __syncthreads();
+    float* red = reinterpret_cast<float*>(smem);  // [phase][slice][tok][32 + 4]
+    constexpr int TOK = 8 * TT, RS = 36;
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
       for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int nl = 32 * v + 4 * q + 2 * mt + (e >> 1);
+          const int nl = 4 * chunk_of(q) + 2 * mt + (e >> 1);
           const int tok = 8 * tt + 2 * c + (e & 1);
-          red[warp][tok][nl] = acc[v][mt][tt][e];
+          red[((phase * 2 + slice) * TOK + tok) * RS + nl] = acc[mt][tt][e];
         }
+  }
+  if (warp == kConsumerWarps) __syncthreads();  // matches the consumers' stash barrier
   __syncthreads();
 
+  // fixed-order reduction: phases, then the cluster's CTAs
+  constexpr int TOK = 8 * TT, RS = 36;
+  const float* red = reinterpret_cast<const float*>(smem);
+  float* part = reinterpret_cast<float*>(smem) + kPhases * 2 * TOK * RS;
   for (int idx = threadIdx.x; idx < TOK * WC; idx += kThreads) {
     const int tok = idx / WC, nl = idx - tok * WC;
+    const int slice = nl >> 5, col = nl & 31;
     float s = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) s += red[w][tok][nl];  // fixed order
+    for (int ph = 0; ph < kPhases; ++ph) s += red[((ph * 2 + slice) * TOK + tok) * RS + col];
     if (splits == 1) {
-      if (tok < M && n_blk + nl < N) y[(int64_t)tok * N + n_blk + nl] = __half_as_ushort(__float2half_rn(s));
+      if (tok < M && nl < ncols)
+        y[(int64_t)tok * N + n_blk + nl] = __half_as_ushort(__float2half_rn(s));
     } else {
       part[idx] = s;
     }
   }
   if (splits > 1) {
-    cluster_sync_all();  // every CTA's partial is visible cluster-wide
+    cluster_sync_all();
     const int rank = (int)cluster_ctarank();
     const int E = TOK * WC;
     const int begin = rank * E / splits, end = (rank + 1) * E / splits;
     const uint32_t base = smem_u32(part);
-    for (int idx = begin + threadIdx.x; idx < end; idx += kThreads) {
+    for (int idx = begin + (int)threadIdx.x; idx < end; idx += kThreads) {
       const int tok = idx / WC, nl = idx - tok * WC;
-      if (tok >= M || n_blk + nl >= N) continue;
+      if (tok >= M || nl >= ncols) continue;
       float s = 0.f;
       for (int r = 0; r < splits; ++r) s += ld_dsmem_f32(map_to_rank(base + 4u * idx, r));
       y[(int64_t)tok * N + n_blk + nl] = __half_as_ushort(__float2half_rn(s));
     }
-    cluster_sync_all();  // keep every CTA's shared memory alive until read
+    cluster_sync_all();
   }
 }
 
-template <int TT, int WCV>
-cudaError_t launch_decode_t(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
-                            uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
-                            int splits, cudaStream_t stream) {
-  constexpr int WC = 32 * WCV;
+template <int TT, bool STAGE_SCALE>
+cudaError_t launch_t(const CUtensorMap& qw_map, const CUtensorMap& s_map, const uint16_t* x,
+                     uint16_t* y, int M, int K, int N, int group_shift, int splits,
+                     const DecodeShape& d, cudaStream_t stream, const DeviceInfo& dev) {
+  static std::once_flag once[64];
+  static cudaError_t attr_err[64];
+  const int di = dev.device & 63;
+  std::call_once(once[di], [&] {
+    attr_err[di] = cudaFuncSetAttribute(decode_kernel<TT, STAGE_SCALE>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  });
+  if (attr_err[di] != cudaSuccess) return attr_err[di];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((N + WC - 1) / WC), (unsigned)splits, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = (size_t)d.smem_bytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = (unsigned)splits;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (splits > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 1;
+    attr[n].val.clusterDim.y = (unsigned)splits;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<TT, WCV>, x, qweight, scales, y, (int)M, (int)K,
-                            (int)N, group_shift);
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<TT, STAGE_SCALE>, qw_map, s_map, x, y, M, K, N, group_shift,
+                            d.stages, d.stage_bytes, d.s_off, d.x_off, d.scale_rows,
+                            dev.error_word);
 }
 
 }  // namespace
 
 int decode_pick_splits(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev) {
-  // Fill the machine with CTAs of 8 warps; each warp should keep at least
-  // three row quads (96 k) of work so the loads can be pipelined.
-  (void)M;
-  const int64_t WC = 64;
+  // CTAs that all fit at once (three per SM for M <= 8, two otherwise), each
+  // with at least four stages (1024 k) of work so that the ring stays full.
   const int64_t nblk = (N + WC - 1) / WC;
-  const int64_t rq = ((K >> 3) + 3) >> 2;
-  const int64_t slots = (int64_t)dev.num_sms * 2;
+  const int64_t ns = ((K >> 3) + RB - 1) / RB;
+  const int64_t slots = (int64_t)dev.num_sms * (M <= 8 ? 3 : 2);
   int best = 1;
-  double best_eff = -1.0;
-  for (int s = 1; s <= 8; ++s) {
-    if (s > 1 && rq < (int64_t)s * kWarps * 3) break;
-    const int64_t ctas = nblk * s;
-    const int64_t waves = (ctas + slots - 1) / slots;
-    const double eff = (double)ctas / (double)(waves * slots);
-    if (eff > best_eff + 0.02) {
-      best_eff = eff;
-      best = s;
-    }
+  for (int s = 2; s <= 8; ++s) {
+    if (ns < (int64_t)s * 4) break;
+    if (nblk * s > slots) break;
+    best = s;
   }
   return best;
 }
@@ -250,9 +454,26 @@ cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint1
                           uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
                           int splits, cudaStream_t stream, const DeviceInfo& dev) {
   if (splits <= 0) splits = decode_pick_splits(M, K, N, dev);
-  if (M <= 8)
-    return launch_decode_t<1, 2>(x, qweight, scales, y, M, K, N, group_shift, splits, stream);
-  return launch_decode_t<2, 2>(x, qweight, scales, y, M, K, N, group_shift, splits, stream);
+  const DecodeShape d = decode_shape((int)M, group_shift);
+  // the reduction reuses the ring: it must fit
+  const int red_bytes = (kPhases * 2 * 16 * 36 + 16 * WC) * 4;
+  if (d.stages * d.stage_bytes < red_bytes) return cudaErrorInvalidValue;
+  const int iM = (int)M, iK = (int)K, iN = (int)N;
+  const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
+                               ? 1 : (K + (int64_t(1) << group_shift) - 1) >> group_shift;
+  CUtensorMap qw_map, s_map;
+  if (!tensor_map_2d(&qw_map, qweight, CU_TENSOR_MAP_DATA_TYPE_INT32, (uint64_t)N,
+                     (uint64_t)(K / 8), (uint64_t)N * 4, 32, RB, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tensor_map_2d(&s_map, scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, (uint64_t)N,
+                     (uint64_t)n_groups, (uint64_t)N * 2, WC, (uint32_t)d.scale_rows,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  const bool stage_scale = group_shift >= 8;
+#define GPTQ_DECODE_LAUNCH(TT_, SS_) \
+  launch_t<TT_, SS_>(qw_map, s_map, x, y, iM, iK, iN, group_shift, splits, d, stream, dev)
+  if (M <= 8) return stage_scale ? GPTQ_DECODE_LAUNCH(1, true) : GPTQ_DECODE_LAUNCH(1, false);
+  return stage_scale ? GPTQ_DECODE_LAUNCH(2, true) : GPTQ_DECODE_LAUNCH(2, false);
+#undef GPTQ_DECODE_LAUNCH
 }
 
 }  // namespace gptq

@@ -58,7 +58,7 @@ def call(lib, x=X, qw=QW, s=S, M=4, K=512, N=256, g=128, y=Y, kernel=None):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(M=-1), 2), (dict(K=0), 2), (dict(K=-16), 2), (dict(N=0), 2),
-    (dict(K=520), 2), (dict(N=252), 2), (dict(K=16 * (1 << 20) + 16), 2),
+    (dict(K=520), 2), (dict(N=252), 2), (dict(K=65536 + 16), 2),
     (dict(N=(1 << 20) + 8), 2), (dict(M=(1 << 23) + 1), 2),
     (dict(g=0), 3), (dict(g=8), 3), (dict(g=100), 3), (dict(g=2048), 3), (dict(g=-2), 3),
     (dict(qw=0), 1), (dict(s=0), 1), (dict(x=0), 1), (dict(y=0), 1),

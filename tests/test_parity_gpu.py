@@ -207,7 +207,7 @@ def test_empty_m():
 
 
 def test_maximum_k_and_n():
-    p = W.make_problem(2, 1 << 20, 8, 1024, seed=11)
+    p = W.make_problem(2, 1 << 16, 8, 1024, seed=11)
     y = run(p, B.KERNEL_DECODE)
     check_rows(p, y, [0, 1], "max K decode")
     y = run(p, B.KERNEL_PREFILL)
