@@ -118,9 +118,11 @@ __device__ __forceinline__ uint16_t ld_nc_u16(const void* p) {
 
 // ---- warp-level MMA (m16n8k16, FP16 inputs, FP32 accumulate) ------------------
 
+// Not volatile: the MMA is a pure function of its operands, so the compiler
+// may interleave it with independent work.
 __device__ __forceinline__ void mma_m16n8k16(float d[4], const uint32_t a[4], uint32_t b0,
                                              uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])

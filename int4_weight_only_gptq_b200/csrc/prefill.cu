@@ -127,6 +127,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                             kDrainLimitNs);
       }
     }
+    __syncwarp();  // the whole warp reaches the CTA barrier below together
   } else if (warp == 1) {
     // ---------------- MMA issuer (one lane) ----------------
     if (lane == 0) {
@@ -157,6 +158,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_wait_bounded(&bar->dfull, 0, &never, kDrainLimitNs);
       }
     }
+    __syncwarp();  // the whole warp reaches the CTA barrier below together
   } else {
     // ---------------- dequantisation, then epilogue ----------------
     const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31

@@ -120,6 +120,10 @@ def test_tiny(M, kernel):
 EDGE = [  # (M, K, N, G)
     (1, 16, 8, -1), (3, 48, 40, 16), (5, 528, 24, 128), (7, 96, 72, 32), (8, 160, 264, 64),
     (9, 64, 8, 16), (13, 1040, 136, 1024), (16, 272, 520, 16), (2, 5120, 8, 512),
+    # K-stages that straddle group boundaries (stages of 768 k for M <= 8,
+    # 512 k for M <= 16), ragged last stages
+    (4, 3072, 64, 1024), (3, 2304, 16, 512), (8, 6144, 24, 256), (1, 1600, 72, 512),
+    (12, 2560, 40, 1024), (16, 1536, 200, 512),
 ]
 
 
