@@ -45,19 +45,48 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode_up")
+    ap.add_argument("--workload", default="decode_up", choices=sorted(WORKLOADS))
     ap.add_argument("--no-sweep", action="store_true")
     return ap.parse_args()
 
 
+# name -> (problem, description, roofline).  The default is the headline.
 WORKLOADS = {
-    "decode_up": (lambda: W.decode_up(), "decode GEMV, FFN up-projection: M=1, K=5120, N=17408, group=128"),
+    "decode_up": (lambda: W.decode_up(),
+                  "decode GEMV, FFN up-projection: M=1, K=5120, N=17408, group=128", "hbm"),
+    "decode_down_m1": (lambda: W.decode_down(1),
+                       "decode, FFN down-projection: M=1, K=17408, N=5120, group=32, outliers", "hbm"),
+    "decode_down_m16": (lambda: W.decode_down(16),
+                        "decode, FFN down-projection: M=16, K=17408, N=5120, group=32, outliers", "hbm"),
+    "prefill_m2048": (lambda: W.prefill(2048),
+                      "prefill GEMM: M=2048, K=5120, N=17408, group=128", "tensor"),
+    "prefill_m8192": (lambda: W.prefill(8192),
+                      "prefill GEMM: M=8192, K=5120, N=17408, group=128", "tensor"),
 }
 
 
 def dist_env():
     return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
             int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The largest `value` over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(bytes_per_step: int, steps: int, elapsed_ms_max: float, world: int):
+    """(ms per step, whole-job GB/s, per-GPU GB/s) for weak scaling: every
+    rank moved bytes_per_step per step; the slowest rank's time counts."""
+    ms = elapsed_ms_max / steps
+    per_gpu = bytes_per_step / (ms * 1e-3) / 1e9
+    return ms, per_gpu * world, per_gpu
 
 
 def peaks():
@@ -215,10 +244,12 @@ def run_ours(args):
     lib = binding.load()
     props = torch.cuda.get_device_properties(local_rank)
     l2 = props.L2_cache_size
-    make, desc = WORKLOADS[args.workload]
+    make, desc, bound = WORKLOADS[args.workload]
     p = make()
     bytes_per_step = p.algorithmic_bytes
-    copies = copies_for(p, l2)
+    # HBM-bound workloads rotate over copies whose total exceeds twice the L2;
+    # the tensor-bound ones move more than the L2 per call anyway
+    copies = copies_for(p, l2) if bound == "hbm" else 1
     sets = to_device(p, torch, copies)
     stream = torch.cuda.current_stream()
     sh = ctypes.c_void_p(stream.cuda_stream)
@@ -243,16 +274,13 @@ def run_ours(args):
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    elapsed_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(e0.elapsed_time(e1), "cuda")
     if binding.device_error() != 0:
         raise RuntimeError("a kernel reported a bounded-wait timeout")
-    ms = elapsed_ms / args.steps
-    value = bytes_per_step * world / (ms * 1e-3) / 1e9
-    per_gpu = bytes_per_step / (ms * 1e-3) / 1e9
+    ms, value, per_gpu = aggregate(bytes_per_step, args.steps, elapsed_ms, world)
+    if bound == "tensor":  # the same aggregation in TFLOP/s
+        value = value * p.flops / bytes_per_step / 1e3
+        per_gpu = per_gpu * p.flops / bytes_per_step / 1e3
 
     # end to end through the public API with host buffers: pinned X in, Y out
     xh = torch.from_numpy(p.x.view(np.int16)).view(torch.float16).pin_memory()
@@ -262,7 +290,7 @@ def run_ours(args):
     for rep in range(2):
         torch.cuda.synchronize()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_e2e = max(10, min(args.steps, 500))
+        n_e2e = max(3, min(args.steps, 500 if bound == "hbm" else 20))
         a0.record(stream)
         for i in range(n_e2e):
             xs, qws, ss, ys = sets[i % copies]
@@ -272,11 +300,7 @@ def run_ours(args):
         a1.record(stream)
         torch.cuda.synchronize()
         e2.append(a0.elapsed_time(a1) / n_e2e)
-    e2e_ms = min(e2)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(min(e2), "cuda")
 
     hbm, tf, src = peaks()
     out = None
@@ -284,9 +308,21 @@ def run_ours(args):
         clocks = clk.summary()
         kernel_id, split = binding.select(p.M, p.K, p.N, p.group)
         traffic = traffic_record("decode.cu", f"{args.workload}")
+        if bound == "hbm":
+            metric = "W4A16 GEMM decode GB/s (algorithmic bytes: packed weights + scales + X + Y)"
+            unit, peak, punit = "GB/s", hbm, "GB/s"
+            peak_src = ("measured (MEASURED_PEAKS.json hbm_gbs)" if src == "measured"
+                        else "fallback 6.65 TB/s")
+            e2e_val = bytes_per_step * world / (e2e_ms * 1e-3) / 1e9
+        else:
+            metric = "W4A16 GEMM prefill TFLOP/s (2*M*K*N)"
+            unit, peak, punit = "TFLOP/s", tf, "TFLOP/s"
+            peak_src = ("measured (MEASURED_PEAKS.json bf16_tflops burst; FP16 dense has the "
+                        "same nominal rate)" if src == "measured" else "fallback 1.59 PFLOP/s")
+            e2e_val = p.flops * world / (e2e_ms * 1e-3) / 1e12
         out = {
-            "metric": "W4A16 GEMM decode GB/s (algorithmic bytes: packed weights + scales + X + Y)",
-            "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "metric": metric,
+            "value": round(value, 1), "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": round(ms, 6),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp16 x int4 -> fp32 acc -> fp16", "data": "synthetic (seeded, PCG64 seed 0)",
@@ -296,12 +332,11 @@ def run_ours(args):
                        "parallelism": f"replicas x{world} (no exchange)",
                        "kernel": {1: "decode", 2: "prefill"}.get(kernel_id, kernel_id),
                        "split_k_ctas": split},
-            "roofline": {"bound": "hbm", "achieved": round(per_gpu, 1), "peak": hbm,
-                         "unit": "GB/s", "frac": round(per_gpu / hbm, 4),
-                         "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6.65 TB/s",
-                         "traffic": traffic},
-            "e2e": {"value": round(bytes_per_step * world / (e2e_ms * 1e-3) / 1e9, 1),
-                    "unit": "GB/s", "ms_per_step": round(e2e_ms, 6),
+            "roofline": {"bound": bound, "achieved": round(per_gpu, 1), "peak": peak,
+                         "unit": punit, "frac": round(per_gpu / peak, 4),
+                         "peak_source": peak_src, "traffic": traffic},
+            "e2e": {"value": round(e2e_val, 1),
+                    "unit": unit, "ms_per_step": round(e2e_ms, 6),
                     "h2d_bytes_per_step": int(p.M * p.K * 2),
                     "d2h_bytes_per_step": int(p.M * p.N * 2),
                     "note": "pinned host X -> device, gptq_w4a16_gemm, device Y -> pinned host; weights resident"},
@@ -313,7 +348,7 @@ def run_ours(args):
         if rank == 0:
             out["sweep"] = sweep
     if rank == 0:
-        out["cpu_baseline"] = cpu_baseline(p, bytes_per_step)
+        out["cpu_baseline"] = cpu_baseline(p, bytes_per_step, bound)
         print(json.dumps(out), flush=True)
     if world > 1:
         dist.barrier()
@@ -355,23 +390,31 @@ def run_sweep(lib, torch, l2, hbm, tf):
 
 # ---- CPU oracle ----------------------------------------------------------
 
-def cpu_baseline(p, bytes_per_step, budget_s: float = 10.0):
-    """The oracle as it stands, single-threaded, on whole calls of the same
-    workload (M=1 computes every output), repeated for about budget_s."""
+def cpu_baseline(p, bytes_per_step, bound="hbm", budget_s: float = 10.0):
+    """The oracle as it stands (OpenMP over output columns) on a bounded
+    sample of the same workload, repeated for about budget_s: every row when
+    M <= 16, else four rows (first, last, two inside), scaled to the metric's
+    unit by the share of the work they are."""
     import oracle
     oracle.build()
     threads = oracle.get_threads()
+    rows = list(range(p.M)) if p.M <= 16 else sorted({0, p.M // 3, 2 * p.M // 3, p.M - 1})
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle.gemm_rows(p.x, p.qweight, p.scales, p.group, list(range(p.M)))
+        oracle.gemm_rows(p.x, p.qweight, p.scales, p.group, rows)
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s or n >= 1000:
             break
     per = el / n
-    return {"value": round(bytes_per_step / per / 1e9, 4), "unit": "GB/s", "cores": threads,
-            "kind": "oracle",
-            "sample": f"{n} whole call(s) of the workload ({el:.1f} s, {threads} OpenMP threads over output columns)",
+    share = len(rows) / p.M
+    if bound == "hbm":
+        value, unit = bytes_per_step * share / per / 1e9, "GB/s"
+    else:
+        value, unit = p.flops * share / per / 1e12, "TFLOP/s"
+    what = "whole call(s) of the workload" if share == 1 else f"calls on {len(rows)} of {p.M} rows"
+    return {"value": round(value, 6), "unit": unit, "cores": threads, "kind": "oracle",
+            "sample": f"{n} {what} ({el:.1f} s, {threads} OpenMP threads over output columns)",
             "s_per_call": round(per, 4)}
 
 
@@ -382,7 +425,7 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    make, desc = WORKLOADS[args.workload]
+    make, desc, bound = WORKLOADS[args.workload]
     p = make()
     import oracle
     oracle.build()
