@@ -12,9 +12,11 @@
 //   warps unpack each int32 word (eight consecutive k of one column) into four
 //   32-bit TMEM cells of that column's lane, so dequantised weights never
 //   touch shared memory.
-// * X is the B operand: a TMA producer warp streams [256 tokens x 64 k] FP16
-//   tiles into shared memory with the 128-byte swizzle the MMA descriptor
-//   expects; out-of-range tokens and k read as zero.
+// * One TMA producer thread streams, per 64-k stage, the X tile [256 tokens x
+//   64 k] (FP16, 128-byte swizzle: the B operand), the qweight tile [8 packed
+//   rows x 128 columns] and the scale rows of the stage; out-of-range rows and
+//   columns read as zero.  The dequantisation warps read their column's words
+//   and scales from shared memory at fixed offsets.
 // * One thread issues tcgen05.mma (kind::f16, FP32 accumulate) into a
 //   128 x 256 FP32 accumulator in TMEM; tcgen05.commit releases each stage.
 // * The dequantisation warps then read the accumulator back (tcgen05.ld),
@@ -23,7 +25,7 @@
 //   GPTQ_ERR_TIMEOUT in the device error word, drains its own copies and MMAs,
 //   frees TMEM and exits.  Nothing traps.
 //
-// Bytes per CTA tile: 128 x K / 2 (qweight) + scales + 256 x K x 2 (X, from L2).
+// Bytes per CTA tile: 128 x K / 2 (qweight) + scales + 256 x K x 2 (X, mostly from L2).
 // FLOPs per call: 2 M K N.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -33,6 +35,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tc05.cuh"
+#include "tmap.h"
 
 namespace gptq {
 
@@ -45,13 +48,19 @@ constexpr int STAGES = 4;
 constexpr int DQ_WARPS = 8;  // dequantisation + epilogue warps
 constexpr int THREADS = (2 + DQ_WARPS) * 32;
 constexpr int X_STAGE_BYTES = BT * BK * 2;
+constexpr int QW_STAGE_BYTES = BW * (BK / 8) * 4;  // 128 columns x 8 packed rows: 4 KB
+constexpr int S_ROW_BYTES = BW * 2;                // one scale row of the tile: 256 B
+constexpr int S_STAGE_MAX_ROWS = BK / 16;          // group 16: four rows per stage
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t D_COL = 0;                 // accumulator: columns [0, 256)
 constexpr uint32_t A_COL = 256;               // A stages: [256, 256 + 4 * 32)
 constexpr uint32_t A_STAGE_COLS = BK / 2;     // two FP16 per 32-bit column
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint64_t kDrainLimitNs = 200000000ull;
-constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * X_STAGE_BYTES + 256;
+constexpr int QW_OFF = STAGES * X_STAGE_BYTES;
+constexpr int S_OFF = QW_OFF + STAGES * QW_STAGE_BYTES;
+constexpr int BAR_OFF = S_OFF + STAGES * S_STAGE_MAX_ROWS * S_ROW_BYTES;
+constexpr size_t kSmemBytes = 1024 + (size_t)BAR_OFF + 256;
 
 struct Barriers {
   uint64_t xfull[STAGES];   // X tile landed (TMA transaction count)
@@ -67,22 +76,24 @@ __device__ __forceinline__ void record_timeout(int* err, Barriers* b) {
   *reinterpret_cast<volatile int*>(&b->abort_flag) = 1;
 }
 
+// scale_rows: scale rows one 64-k stage touches (1, or 64/group for groups
+// below 64); stages start on 64-k boundaries, so they align with groups.
 __global__ void __launch_bounds__(THREADS, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap x_map, const int32_t* __restrict__ qweight,
-                   const uint16_t* __restrict__ scales, uint16_t* __restrict__ y, int M, int K,
-                   int N, int group_shift, int* err) {
+    prefill_kernel(const __grid_constant__ CUtensorMap x_map,
+                   const __grid_constant__ CUtensorMap qw_map,
+                   const __grid_constant__ CUtensorMap s_map, uint16_t* __restrict__ y, int M,
+                   int K, int N, int group_shift, int scale_rows, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* xs = smem;
-  Barriers* bar = reinterpret_cast<Barriers*>(smem + STAGES * X_STAGE_BYTES);
+  Barriers* bar = reinterpret_cast<Barriers*>(smem + BAR_OFF);
   volatile int* abort_flag = &bar->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BW;
   const int t0 = blockIdx.y * BT;
   const int KB = (K + BK - 1) / BK;
-  const int P = K >> 3;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -94,7 +105,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     bar->abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == 0 && lane == 0) prefetch_tensormap(&x_map);
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&x_map);
+    prefetch_tensormap(&qw_map);
+    prefetch_tensormap(&s_map);
+  }
   if (warp == 1) {
     tmem_alloc(&bar->tmem_base, TMEM_COLS);
     tmem_relinquish();
@@ -115,8 +130,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           record_timeout(err, bar);
           break;
         }
-        mbar_arrive_expect_tx(&bar->xfull[s], X_STAGE_BYTES);
+        mbar_arrive_expect_tx(&bar->xfull[s],
+                              X_STAGE_BYTES + QW_STAGE_BYTES + scale_rows * S_ROW_BYTES);
         tma_load_2d(xs + s * X_STAGE_BYTES, &x_map, kb * BK, t0, &bar->xfull[s]);
+        tma_load_2d(smem + QW_OFF + s * QW_STAGE_BYTES, &qw_map, n0, kb * (BK / 8),
+                    &bar->xfull[s]);
+        tma_load_2d(smem + S_OFF + s * S_STAGE_MAX_ROWS * S_ROW_BYTES, &s_map, n0,
+                    (int)(((int64_t)kb * BK) >> group_shift), &bar->xfull[s]);
         ++issued;
       }
       if (*abort_flag) {
@@ -167,35 +187,40 @@ __global__ void __launch_bounds__(THREADS, 1)
     const bool col_ok = n < N;
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
 
-    uint32_t cw[4], cs[4], nw[4], ns[4];
-    auto load = [&](int kb, uint32_t (&w)[4], uint32_t (&sc)[4]) {
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int row = kb * (BK / 8) + 4 * half + r;
-        if (col_ok && row < P) {
-          w[r] = ld_nc_u32(qweight + (int64_t)row * N + n);
-          sc[r] = ld_nc_u16(scales + ((int64_t(row) * 8) >> group_shift) * N + n);
-        } else {
-          w[r] = 0x88888888u;  // every code 8: weight (8 - 8) * 0 = 0
-          sc[r] = 0;
-        }
-      }
-    };
+    // this thread's column in the stage's qweight and scale tiles; packed
+    // rows 4*half .. 4*half+3 of every stage
+    const int col = 32 * quarter + lane;
+    const uint8_t* qw_tile = smem + QW_OFF + (4 * half) * (BW * 4) + col * 4;
+    const uint8_t* s_tile = smem + S_OFF + col * 2;
 
     bool ok = true;
-    load(0, cw, cs);
     for (int kb = 0; kb < KB; ++kb) {
       const int s = kb % STAGES;
       const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-      if (kb + 1 < KB) load(kb + 1, nw, ns);
+      // qweight and scale tiles of the stage have landed (with X)
+      ok = mbar_wait_bounded(&bar->xfull[s], ph, abort_flag, kWaitLimitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) record_timeout(err, bar);
+        break;
+      }
+      const uint8_t* qw = qw_tile + s * QW_STAGE_BYTES;
+      const uint8_t* sc = s_tile + s * S_STAGE_MAX_ROWS * S_ROW_BYTES;
       uint32_t cells[16];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
+        // scale row of packed row 4*half + r inside the stage (0 unless the
+        // group is smaller than the 64-k stage)
+        const int gl = ((4 * half + r) * 8) >> group_shift;
+        const uint16_t sv = *reinterpret_cast<const uint16_t*>(sc + gl * S_ROW_BYTES);
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(qw + r * (BW * 4));
         uint32_t nat[4];
-        dequant_word_natural(cw[r], half2_broadcast((uint16_t)cs[r]), nat);
+        dequant_word_natural(w, half2_broadcast(sv), nat);
 #pragma unroll
         for (int j = 0; j < 4; ++j) cells[4 * r + j] = nat[j];
       }
+      // the A columns of this stage are free once the MMAs of its previous
+      // use have completed
       ok = mbar_wait_bounded(&bar->empty[s], ph ^ 1u, abort_flag, kWaitLimitNs);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
@@ -207,11 +232,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar->afull[s]);
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        cw[r] = nw[r];
-        cs[r] = ns[r];
-      }
     }
 
     if (ok) {
@@ -247,41 +267,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
 }  // namespace
 
 cudaError_t launch_prefill(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                            uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
                            cudaStream_t stream, const DeviceInfo& dev) {
-  EncodeTiledFn encode = get_encode_fn();
-  if (!encode) return cudaErrorNotSupported;
-  CUtensorMap map;
-  const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
-  const cuuint64_t gstride[1] = {(cuuint64_t)K * 2};
-  const cuuint32_t box[2] = {BK, BT};
-  const cuuint32_t estride[2] = {1, 1};
-  if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(x), gdim, gstride,
-             box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+  const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
+                               ? 1 : (K + (int64_t(1) << group_shift) - 1) >> group_shift;
+  const int scale_rows = group_shift >= 6 ? 1 : (BK >> group_shift);
+  CUtensorMap x_map, qw_map, s_map;
+  if (!tensor_map_2d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M,
+                     (uint64_t)K * 2, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tensor_map_2d(&qw_map, qweight, CU_TENSOR_MAP_DATA_TYPE_INT32, (uint64_t)N,
+                     (uint64_t)(K / 8), (uint64_t)N * 4, BW, BK / 8, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !tensor_map_2d(&s_map, scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, (uint64_t)N,
+                     (uint64_t)n_groups, (uint64_t)N * 2, BW, (uint32_t)scale_rows,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   static std::once_flag attr_once[64];
   static cudaError_t attr_err[64];
@@ -292,8 +293,9 @@ cudaError_t launch_prefill(const uint16_t* x, const int32_t* qweight, const uint
   });
   if (attr_err[d] != cudaSuccess) return attr_err[d];
   const dim3 grid((unsigned)((N + BW - 1) / BW), (unsigned)((M + BT - 1) / BT), 1);
-  prefill_kernel<<<grid, THREADS, kSmemBytes, stream>>>(map, qweight, scales, y, (int)M, (int)K,
-                                                       (int)N, group_shift, dev.error_word);
+  prefill_kernel<<<grid, THREADS, kSmemBytes, stream>>>(x_map, qw_map, s_map, y, (int)M, (int)K,
+                                                       (int)N, group_shift, scale_rows,
+                                                       dev.error_word);
   return cudaGetLastError();
 }
 
