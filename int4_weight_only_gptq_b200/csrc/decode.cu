@@ -173,8 +173,9 @@ __global__ void __launch_bounds__(Geo<NW>::THREADS) __maxnreg__(TT == 1 ? 72 : 9
   constexpr int RB = Geo<NW>::RB, QW_BOX = Geo<NW>::QW_BOX, X_PITCH = Geo<NW>::X_PITCH;
   constexpr int kConsumerWarps = NW, kThreads = Geo<NW>::THREADS;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base, derived from the shared array itself so that the
+  // compiler keeps the shared address space (plain LDS, no generic loads)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   DecodeBars* bar = reinterpret_cast<DecodeBars*>(smem + stages * stage_bytes);
   volatile int* abort_flag = &bar->abort_flag;
 

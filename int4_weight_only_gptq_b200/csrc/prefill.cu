@@ -84,8 +84,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                    const __grid_constant__ CUtensorMap s_map, uint16_t* __restrict__ y, int M,
                    int K, int N, int group_shift, int scale_rows, int* err) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base, derived from the shared array itself so that the
+  // compiler keeps the shared address space (plain LDS, no generic loads)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* xs = smem;
   Barriers* bar = reinterpret_cast<Barriers*>(smem + BAR_OFF);
   volatile int* abort_flag = &bar->abort_flag;
