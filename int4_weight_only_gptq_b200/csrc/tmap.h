@@ -1,4 +1,4 @@
-// Cached construction of TMA tensor maps (2-D, row-major) on the host.
+// Cached construction of TMA tensor maps (2-D and 3-D) on the host.
 #pragma once
 
 #include <cuda.h>
@@ -12,6 +12,12 @@ namespace gptq {
 // entry point is unavailable or rejects the arguments.
 bool tensor_map_2d(CUtensorMap* out, const void* ptr, CUtensorMapDataType dtype, uint64_t dim0,
                    uint64_t dim1, uint64_t row_bytes, uint32_t box0, uint32_t box1,
+                   CUtensorMapSwizzle swizzle);
+
+// Same for a 3-D view: dims[0] contiguous, dims[1] and dims[2] `strides[0]`
+// and `strides[1]` bytes apart (any order of strides), boxes of box[0..2].
+bool tensor_map_3d(CUtensorMap* out, const void* ptr, CUtensorMapDataType dtype,
+                   const uint64_t dims[3], const uint64_t strides[2], const uint32_t box[3],
                    CUtensorMapSwizzle swizzle);
 
 }  // namespace gptq
