@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int s = kb % STAGES;
       const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
       // qweight and scale tiles of the stage have landed (with X)
-      ok = mbar_wait_bounded(&bar->xfull[s], ph, abort_flag, kWaitLimitNs);
+      ok = mbar_wait_bounded<true>(&bar->xfull[s], ph, abort_flag, kWaitLimitNs);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         if (lane == 0) record_timeout(err, bar);
@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       // the A columns of this stage are free once the MMAs of its previous
       // use have completed
-      ok = mbar_wait_bounded(&bar->empty[s], ph ^ 1u, abort_flag, kWaitLimitNs);
+      ok = mbar_wait_bounded<true>(&bar->empty[s], ph ^ 1u, abort_flag, kWaitLimitNs);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         if (lane == 0) record_timeout(err, bar);
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 
     if (ok) {
-      ok = mbar_wait_bounded(&bar->dfull, 0, abort_flag, kWaitLimitNs);
+      ok = mbar_wait_bounded<true>(&bar->dfull, 0, abort_flag, kWaitLimitNs);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok && lane == 0) record_timeout(err, bar);
     }

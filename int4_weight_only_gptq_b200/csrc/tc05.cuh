@@ -22,13 +22,17 @@ constexpr uint32_t kWaitSleepNs = 1000;
 
 // Waits for the phase with the given parity to complete.  Gives up (returns
 // false) after `limit_ns` or as soon as *abort is set by another thread.
+// SLEEP: polls may suspend the thread (for waits that are long and not on
+// the critical path); otherwise the thread spins on the barrier.
+template <bool SLEEP = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort, uint64_t limit_ns) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait_sleep(addr, parity, kWaitSleepNs)) return true;
+    if (SLEEP ? mbar_try_wait_sleep(addr, parity, kWaitSleepNs) : mbar_try_wait(addr, parity))
+      return true;
     if ((n & 63u) == 0) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) return false;
