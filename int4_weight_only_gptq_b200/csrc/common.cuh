@@ -98,37 +98,6 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   return r;
 }
 
-__device__ __forceinline__ uint2 ld_nc_v2(const void* p) {
-  uint2 r;
-  asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t ld_nc_u32(const void* p) {
-  uint32_t r;
-  asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(r) : "l"(p));
-  return r;
-}
-
-__device__ __forceinline__ uint16_t ld_nc_u16(const void* p) {
-  uint16_t r;
-  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));
-  return r;
-}
-
-// ---- warp-level MMA (m16n8k16, FP16 inputs, FP32 accumulate) ------------------
-
-// Not volatile: the MMA is a pure function of its operands, so the compiler
-// may interleave it with independent work.
-__device__ __forceinline__ void mma_m16n8k16(float d[4], const uint32_t a[4], uint32_t b0,
-                                             uint32_t b1) {
-  asm(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 // ---- shared memory / cluster ------------------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
