@@ -340,9 +340,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     const bool x_writer = (dw % GROUP_WARPS) * 32 < x_chunks;
 
     bool ok = true;
-    for (int t = grp; t < n_st && ok; t += GROUPS) {
-      const int s = t % stages;
-      const uint32_t ph = (uint32_t)(t / stages) & 1u;
+    // ring slot and phase of stage t, advanced incrementally (GROUPS <= stages)
+    int s = grp % stages;
+    uint32_t ph = (uint32_t)(grp / stages) & 1u;
+    for (int t = grp; t < n_st && ok; t += GROUPS, s += GROUPS) {
+      if (s >= stages) {
+        s -= stages;
+        ph ^= 1u;
+      }
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar->full[s], ph, abort_flag, kWaitLimitNs));
       if (!ok) break;
       uint8_t* st = smem + s * stage_bytes;
