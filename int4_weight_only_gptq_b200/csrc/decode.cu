@@ -237,6 +237,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           record_timeout(err, bar);
           break;
         }
+        // the first two stages go out alone, so that they land before the
+        // rest of the ring is requested (every CTA starts at once)
+        if (t == 2 && !mbar_wait_bounded(&bar->full[0], 0u, abort_flag, kWaitLimitNs)) {
+          record_timeout(err, bar);
+          break;
+        }
         uint8_t* st = smem + s * stage_bytes;
         const int k0 = (st_begin + t) * BKS;
         mbar_arrive_expect_tx(&bar->full[s],
@@ -418,15 +424,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int j = 0; j < BT; ++j) r[j] = 0u;  // an empty K range contributes zero
       if (ok && n_st > 0) {
         tc_fence_after();
-        // accumulators summed in a fixed order
+        // all accumulators requested at once, then summed in a fixed order
+        uint32_t v[NACC][BT];
 #pragma unroll
-        for (int c = 0; c < NACC; ++c) {
-          uint32_t v[BT];
-          tmem_ld_32x32b_x16(tmem + lane_addr + D_COL + c * BT, v);
-          tmem_wait_ld();
+        for (int c = 0; c < NACC; ++c) tmem_ld_32x32b_x16(tmem + lane_addr + D_COL + c * BT, v[c]);
+        tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < BT; ++j)
-            r[j] = c == 0 ? v[j] : __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(v[j]));
+        for (int j = 0; j < BT; ++j) {
+          float acc = __uint_as_float(v[0][j]);
+#pragma unroll
+          for (int c = 1; c < NACC; ++c) acc += __uint_as_float(v[c][j]);
+          r[j] = __float_as_uint(acc);
         }
       }
       if (splits == 1) {
