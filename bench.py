@@ -385,8 +385,11 @@ def run_sweep(lib, torch, l2, hbm, tf):
         tfl = p.flops / (ms * 1e-3) / 1e12
         res[name] = {"ms": round(ms, 4), "TFLOP/s": round(tfl, 1), "frac_tensor": round(tfl / tf, 3)}
 
-    for M in (1, 2, 4, 8, 16):
+    for M in (1, 2, 4, 8, 16, 32):
         hbm_case(f"decode_down_M{M}", W.decode_down(M))
+    # between the kernels: decode up to M = 32, prefill (64-token tile) above
+    for M in (24, 32, 48, 64):
+        hbm_case(f"midm_up_M{M}", W.make_problem(M, 5120, 17408, 128, seed=0), steps=100)
     for M in (512, 2048, 8192):
         tc_case(f"prefill_M{M}", W.prefill(M))
     for g in W.GROUP_SIZES:

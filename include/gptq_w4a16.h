@@ -61,14 +61,14 @@ typedef enum {
 /* Kernel identifiers reported by gptq_w4a16_select and accepted by
  * gptq_w4a16_gemm_kernel. */
 #define GPTQ_KERNEL_AUTO 0
-#define GPTQ_KERNEL_DECODE 1   /* M <= 16: streams qweight, split-K, warp MMA      */
+#define GPTQ_KERNEL_DECODE 1   /* M <= 32: streams qweight, split-K, tcgen05 MMA   */
 #define GPTQ_KERNEL_PREFILL 2  /* any M: TMA + tcgen05 MMA with TMEM accumulators  */
 
 /* Size limits (inclusive). */
 #define GPTQ_MAX_K 65536
 #define GPTQ_MAX_N 1048576
 #define GPTQ_MAX_M 8388608
-#define GPTQ_DECODE_MAX_M 16
+#define GPTQ_DECODE_MAX_M 32
 
 /*
  * Y = X . dequant(qweight, scales).

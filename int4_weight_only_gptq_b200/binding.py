@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libgptq_w4a16.so")
 
 KERNEL_AUTO, KERNEL_DECODE, KERNEL_PREFILL = 0, 1, 2
-DECODE_MAX_M = 16
+DECODE_MAX_M = 32
 GROUP_SIZES = (-1, 16, 32, 64, 128, 256, 512, 1024)
 
 STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_NULL", 2: "GPTQ_ERR_SHAPE", 3: "GPTQ_ERR_GROUP",

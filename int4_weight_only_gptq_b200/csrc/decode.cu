@@ -1,4 +1,4 @@
-// Decode kernel: Y[M, N] = X[M, K] . dequant(qweight, scales) for M <= 16,
+// Decode kernel: Y[M, N] = X[M, K] . dequant(qweight, scales) for M <= 32,
 // on the 5th-generation tensor cores (tcgen05) with TMEM accumulators.
 //
 // Operation: GPTQ-Pro README, "Runtime contract" and "Ampere kernel
@@ -10,7 +10,7 @@
 //
 // * The product is computed transposed, Y^T = W^T . X^T: a CTA owns 128 weight
 //   columns (the MMA's M, one TMEM lane each) and a range of K; the tokens are
-//   the MMA's N = 16 (rows at or beyond M read as zero).
+//   the MMA's N = BT, 16 or 32 (rows at or beyond M read as zero).
 // * One TMA producer thread streams, per 256-k stage, the qweight tile [32
 //   packed rows x 128 columns], the scale rows of the stage and the X tile
 //   [16 tokens x 256 k] (FP16, 128-byte swizzle: the B operand) into a ring of
@@ -59,7 +59,6 @@ namespace gptq {
 namespace {
 
 constexpr int BW = 128;                  // weight columns per CTA (MMA M)
-constexpr int BT = 16;                   // token slots (MMA N)
 constexpr int BKA = 256;                 // k per A slot fill (16 MMAs of k16)
 constexpr int HALVES = 2;                // A slot fills per ring stage
 constexpr int BKS = BKA * HALVES;        // k per ring stage
@@ -72,27 +71,37 @@ constexpr int CHUNKS = PRA / (SLICES * WPT);  // TMEM stores per thread per fill
 constexpr int GROUP_WARPS = 4 * SLICES;  // four TMEM lane quarters per slice
 constexpr int DQ_WARPS = GROUPS * GROUP_WARPS;
 constexpr int THREADS = (2 + DQ_WARPS) * 32;
-constexpr int X_ATOM_BYTES = BT * 128;   // 64 k x 16 tokens, 128-byte swizzle
 constexpr int X_ATOMS = BKS / 64;
-constexpr int X_STAGE_BYTES = X_ATOMS * X_ATOM_BYTES;
 constexpr int QW_STAGE_BYTES = PRS * BW * 4;
 constexpr int S_ROW_BYTES = BW * 2;
-constexpr int QW_OFF = X_STAGE_BYTES;
-constexpr int S_OFF = QW_OFF + QW_STAGE_BYTES;
 constexpr int kMaxStages = 8;
 constexpr int kRingBudget = 224 * 1024;
 constexpr int A_SLOTS = 3;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int NACC = 4;                  // independent accumulators (MMA k16 steps round-robin)
-constexpr uint32_t D_COL = 0;            // accumulators: NACC x 16 columns
+constexpr uint32_t D_COL = 0;            // accumulators: NACC x BT columns
 constexpr uint32_t A_COL0 = 128;         // A slots: [128, 512), 128 columns each
 constexpr uint32_t A_SLOT_COLS = BKA / 2;  // two FP16 per 32-bit column
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 
 static_assert(A_COL0 + A_SLOTS * A_SLOT_COLS <= TMEM_COLS, "TMEM budget");
-static_assert(D_COL + NACC * BT <= A_COL0, "accumulators below the A slots");
-static_assert(BT * BW * 4 <= X_STAGE_BYTES + QW_STAGE_BYTES, "reduction buffer fits a stage");
+
+// Geometry that depends on the token tile BT (the MMA's N): a stage holds X
+// as X_ATOMS atoms of [BT tokens x 64 k] (128-byte swizzle), then qweight,
+// then the scale rows.
+template <int BT_>
+struct TokGeo {
+  static constexpr int BT = BT_;
+  static constexpr int X_ATOM_BYTES = BT * 128;
+  static constexpr int X_STAGE_BYTES = X_ATOMS * X_ATOM_BYTES;
+  static constexpr int QW_OFF = X_STAGE_BYTES;
+  static constexpr int S_OFF = QW_OFF + QW_STAGE_BYTES;
+  // independent accumulators (the k16 steps go round-robin), NACC x BT <= 128
+  static constexpr int NACC = 128 / BT < 4 ? 128 / BT : 4;
+  static_assert(BT % 16 == 0 && BT >= 16 && BT <= 64, "token tile");
+  static_assert(D_COL + NACC * BT <= A_COL0, "accumulators below the A slots");
+  static_assert(BT * BW * 4 <= X_STAGE_BYTES + QW_STAGE_BYTES, "reduction buffer fits a stage");
+};
 static_assert(1024 + kRingBudget + 256 <= 227 * 1024, "shared memory per CTA");
 
 struct DecodeShape {
@@ -106,10 +115,11 @@ inline int align1024(int v) { return (v + 1023) & ~1023; }
 
 // Stages start on multiples of 512 k and groups are powers of two, so a
 // stage touches 512 / group scale rows (one for groups of 512 and more).
+template <int BT>
 inline DecodeShape decode_shape(int group_shift) {
   DecodeShape d;
   d.scale_rows = group_shift >= 9 ? 1 : (BKS >> group_shift);
-  d.stage_bytes = align1024(S_OFF + d.scale_rows * S_ROW_BYTES);
+  d.stage_bytes = align1024(TokGeo<BT>::S_OFF + d.scale_rows * S_ROW_BYTES);
   const int s = kRingBudget / d.stage_bytes;
   d.stages = s > kMaxStages ? kMaxStages : s;
   d.smem_bytes = 1024 + d.stages * d.stage_bytes + 256;
@@ -172,13 +182,18 @@ __device__ __forceinline__ void permute_x_chunk(uint8_t* p) {
 // group 16, 4 for group 32, 8 (the thread's whole slice) for 64 and more.
 // x3d: X arrives as one 3-D box per stage (K a multiple of 64) instead of
 // one 2-D box per 64-k atom.
-template <int WPS>
+template <int WPS, int BT>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap x_map,
                   const __grid_constant__ CUtensorMap qw_map,
                   const __grid_constant__ CUtensorMap s_map, uint16_t* __restrict__ y, int M,
                   int K, int N, int group_shift, int stages, int stage_bytes, int scale_rows,
                   int x3d, int* err) {
+  constexpr int X_ATOM_BYTES = TokGeo<BT>::X_ATOM_BYTES;
+  constexpr int X_STAGE_BYTES = TokGeo<BT>::X_STAGE_BYTES;
+  constexpr int QW_OFF = TokGeo<BT>::QW_OFF;
+  constexpr int S_OFF = TokGeo<BT>::S_OFF;
+  constexpr int NACC = TokGeo<BT>::NACC;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array itself so that the
   // compiler keeps the shared address space (plain LDS, no generic loads)
@@ -418,37 +433,41 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (h == 0) {
       // the four warps of slice 0 hold the four lane quarters: column `col`,
-      // tokens 0..15
-      uint32_t r[BT];
+      // tokens in blocks of 16; an empty K range contributes zero
+      float* part = reinterpret_cast<float*>(smem);  // [token][column], splits > 1
+      if (ok && n_st > 0) tc_fence_after();
+#pragma unroll 1
+      for (int tb = 0; tb < BT / 16; ++tb) {
+        float r[16];
 #pragma unroll
-      for (int j = 0; j < BT; ++j) r[j] = 0u;  // an empty K range contributes zero
-      if (ok && n_st > 0) {
-        tc_fence_after();
-        // all accumulators requested at once, then summed in a fixed order
-        uint32_t v[NACC][BT];
+        for (int j = 0; j < 16; ++j) r[j] = 0.f;
+        if (ok && n_st > 0) {
+          // the block's accumulators requested at once, then summed in a fixed order
+          uint32_t v[NACC][16];
 #pragma unroll
-        for (int c = 0; c < NACC; ++c) tmem_ld_32x32b_x16(tmem + lane_addr + D_COL + c * BT, v[c]);
-        tmem_wait_ld();
+          for (int c = 0; c < NACC; ++c)
+            tmem_ld_32x32b_x16(tmem + lane_addr + D_COL + c * BT + 16 * tb, v[c]);
+          tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < BT; ++j) {
-          float acc = __uint_as_float(v[0][j]);
+          for (int j = 0; j < 16; ++j) {
+            float acc = __uint_as_float(v[0][j]);
 #pragma unroll
-          for (int c = 1; c < NACC; ++c) acc += __uint_as_float(v[c][j]);
-          r[j] = __float_as_uint(acc);
+            for (int c = 1; c < NACC; ++c) acc += __uint_as_float(v[c][j]);
+            r[j] = acc;
+          }
         }
-      }
-      if (splits == 1) {
-        if (ok && n < N) {
+        if (splits == 1) {
+          if (ok && n < N) {
 #pragma unroll
-          for (int tok = 0; tok < BT; ++tok)
-            if (tok < M)
-              y[(int64_t)tok * N + n] = __half_as_ushort(__float2half_rn(__uint_as_float(r[tok])));
+            for (int j = 0; j < 16; ++j)
+              if (16 * tb + j < M)
+                y[(int64_t)(16 * tb + j) * N + n] = __half_as_ushort(__float2half_rn(r[j]));
+          }
+        } else {
+          // partial tile in the (fully consumed) ring
+#pragma unroll
+          for (int j = 0; j < 16; ++j) part[(16 * tb + j) * BW + col] = r[j];
         }
-      } else {
-        // partial tile [token][column] in the (fully consumed) ring
-        float* part = reinterpret_cast<float*>(smem);
-#pragma unroll
-        for (int tok = 0; tok < BT; ++tok) part[tok * BW + col] = __uint_as_float(r[tok]);
       }
     }
   }
@@ -478,7 +497,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int WPS>
+template <int WPS, int BT>
 cudaError_t launch_t(const CUtensorMap& x_map, const CUtensorMap& qw_map, const CUtensorMap& s_map,
                      uint16_t* y, int M, int K, int N, int group_shift, int splits, int x3d,
                      const DecodeShape& d, cudaStream_t stream, const DeviceInfo& dev) {
@@ -486,7 +505,7 @@ cudaError_t launch_t(const CUtensorMap& x_map, const CUtensorMap& qw_map, const 
   static cudaError_t attr_err[64];
   const int di = dev.device & 63;
   std::call_once(once[di], [&] {
-    attr_err[di] = cudaFuncSetAttribute(decode_kernel<WPS>,
+    attr_err[di] = cudaFuncSetAttribute(decode_kernel<WPS, BT>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         1024 + kRingBudget + 256);
   });
@@ -510,7 +529,7 @@ cudaError_t launch_t(const CUtensorMap& x_map, const CUtensorMap& qw_map, const 
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS>, x_map, qw_map, s_map, y, M, K, N,
+  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT>, x_map, qw_map, s_map, y, M, K, N,
                             group_shift, d.stages, d.stage_bytes, d.scale_rows, x3d,
                             dev.error_word);
 }
@@ -539,12 +558,15 @@ int decode_pick_splits(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev) {
   return best;
 }
 
-cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
-                          uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
-                          int splits, cudaStream_t stream, const DeviceInfo& dev) {
-  if (splits <= 0) splits = decode_pick_splits(M, K, N, dev);
-  const DecodeShape d = decode_shape(group_shift);
-  if (d.smem_bytes > 1024 + kRingBudget + 256) return cudaErrorInvalidValue;
+namespace {
+
+// Tensor maps and launch for a token tile of BT.
+template <int BT>
+cudaError_t launch_bt(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                      uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift, int splits,
+                      cudaStream_t stream, const DeviceInfo& dev) {
+  const DecodeShape d = decode_shape<BT>(group_shift);
+  if (d.stages < GROUPS || d.smem_bytes > 1024 + kRingBudget + 256) return cudaErrorInvalidValue;
   const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
                                ? 1 : (K + (int64_t(1) << group_shift) - 1) >> group_shift;
   CUtensorMap x_map, qw_map, s_map;
@@ -570,13 +592,25 @@ cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint1
     return cudaErrorInvalidValue;
   const int iM = (int)M, iK = (int)K, iN = (int)N;
   if (group_shift == 4)
-    return launch_t<2>(x_map, qw_map, s_map, y, iM, iK, iN, group_shift, splits, x3d, d, stream,
-                       dev);
+    return launch_t<2, BT>(x_map, qw_map, s_map, y, iM, iK, iN, group_shift, splits, x3d, d,
+                           stream, dev);
   if (group_shift == 5)
-    return launch_t<4>(x_map, qw_map, s_map, y, iM, iK, iN, group_shift, splits, x3d, d, stream,
-                       dev);
-  return launch_t<WPT>(x_map, qw_map, s_map, y, iM, iK, iN, group_shift, splits, x3d, d, stream,
-                       dev);
+    return launch_t<4, BT>(x_map, qw_map, s_map, y, iM, iK, iN, group_shift, splits, x3d, d,
+                           stream, dev);
+  return launch_t<WPT, BT>(x_map, qw_map, s_map, y, iM, iK, iN, group_shift, splits, x3d, d,
+                           stream, dev);
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                          uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
+                          int splits, cudaStream_t stream, const DeviceInfo& dev) {
+  if (splits <= 0) splits = decode_pick_splits(M, K, N, dev);
+  // token tile: 16 tokens up to M = 16, else 32
+  if (M <= 16)
+    return launch_bt<16>(x, qweight, scales, y, M, K, N, group_shift, splits, stream, dev);
+  return launch_bt<32>(x, qweight, scales, y, M, K, N, group_shift, splits, stream, dev);
 }
 
 }  // namespace gptq

@@ -31,7 +31,7 @@ cudaError_t launch_dequant(const int32_t* qweight, const uint16_t* scales, int64
                            int group_shift, uint16_t* w_out, cudaStream_t stream,
                            const DeviceInfo& dev);
 
-// Decode (M <= 16).  splits = number of CTAs that share one column block along
+// Decode (M <= 32).  splits = number of CTAs that share one column block along
 // K (the cluster size, 1..8); 0 picks it from the shape.
 int decode_pick_splits(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev);
 cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,

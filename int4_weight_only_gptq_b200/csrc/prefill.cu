@@ -42,25 +42,32 @@ namespace gptq {
 namespace {
 
 constexpr int BW = 128;  // weight columns per CTA (MMA M; one TMEM lane each)
-constexpr int BT = 256;  // tokens per CTA (MMA N)
+constexpr int BT_MAX = 256;  // tokens per CTA (MMA N): 64, 128 or 256, by M
 constexpr int BK = 64;   // k per pipeline stage (four k16 MMAs)
 constexpr int STAGES = 4;
 constexpr int DQ_WARPS = 8;  // dequantisation + epilogue warps
 constexpr int THREADS = (2 + DQ_WARPS) * 32;
-constexpr int X_STAGE_BYTES = BT * BK * 2;
 constexpr int QW_STAGE_BYTES = BW * (BK / 8) * 4;  // 128 columns x 8 packed rows: 4 KB
 constexpr int S_ROW_BYTES = BW * 2;                // one scale row of the tile: 256 B
 constexpr int S_STAGE_MAX_ROWS = BK / 16;          // group 16: four rows per stage
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t D_COL = 0;                 // accumulator: columns [0, 256)
+constexpr uint32_t D_COL = 0;                 // accumulator: columns [0, BT)
 constexpr uint32_t A_COL = 256;               // A stages: [256, 256 + 4 * 32)
 constexpr uint32_t A_STAGE_COLS = BK / 2;     // two FP16 per 32-bit column
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint64_t kDrainLimitNs = 200000000ull;
-constexpr int QW_OFF = STAGES * X_STAGE_BYTES;
-constexpr int S_OFF = QW_OFF + STAGES * QW_STAGE_BYTES;
-constexpr int BAR_OFF = S_OFF + STAGES * S_STAGE_MAX_ROWS * S_ROW_BYTES;
-constexpr size_t kSmemBytes = 1024 + (size_t)BAR_OFF + 256;
+
+// Shared-memory layout for a token tile of BT: the X ring, then the qweight
+// and scale rings, then the barriers.
+template <int BT>
+struct Layout {
+  static constexpr int X_STAGE_BYTES = BT * BK * 2;
+  static constexpr int QW_OFF = STAGES * X_STAGE_BYTES;
+  static constexpr int S_OFF = QW_OFF + STAGES * QW_STAGE_BYTES;
+  static constexpr int BAR_OFF = S_OFF + STAGES * S_STAGE_MAX_ROWS * S_ROW_BYTES;
+  static constexpr size_t kSmemBytes = 1024 + (size_t)BAR_OFF + 256;
+};
+static_assert(BT_MAX <= A_COL, "accumulator below the A stages");
 
 struct Barriers {
   uint64_t xfull[STAGES];   // X tile landed (TMA transaction count)
@@ -78,11 +85,17 @@ __device__ __forceinline__ void record_timeout(int* err, Barriers* b) {
 
 // scale_rows: scale rows one 64-k stage touches (1, or 64/group for groups
 // below 64); stages start on 64-k boundaries, so they align with groups.
+template <int BT>
 __global__ void __launch_bounds__(THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap x_map,
                    const __grid_constant__ CUtensorMap qw_map,
                    const __grid_constant__ CUtensorMap s_map, uint16_t* __restrict__ y, int M,
                    int K, int N, int group_shift, int scale_rows, int* err) {
+  static_assert(BT >= 64 && BT <= BT_MAX && BT % 64 == 0, "token tile");
+  constexpr int X_STAGE_BYTES = Layout<BT>::X_STAGE_BYTES;
+  constexpr int QW_OFF = Layout<BT>::QW_OFF;
+  constexpr int S_OFF = Layout<BT>::S_OFF;
+  constexpr int BAR_OFF = Layout<BT>::BAR_OFF;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array itself so that the
   // compiler keeps the shared address space (plain LDS, no generic loads)
@@ -268,14 +281,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-}  // namespace
-
-cudaError_t launch_prefill(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
-                           uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
-                           cudaStream_t stream, const DeviceInfo& dev) {
-  const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
-                               ? 1 : (K + (int64_t(1) << group_shift) - 1) >> group_shift;
-  const int scale_rows = group_shift >= 6 ? 1 : (BK >> group_shift);
+// Tensor maps and launch for a token tile of BT.
+template <int BT>
+cudaError_t launch_t(const uint16_t* x, const int32_t* qweight, const uint16_t* scales, uint16_t* y,
+                     int64_t M, int64_t K, int64_t N, int group_shift, int scale_rows,
+                     int64_t n_groups, cudaStream_t stream, const DeviceInfo& dev) {
   CUtensorMap x_map, qw_map, s_map;
   if (!tensor_map_2d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M,
                      (uint64_t)K * 2, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -285,19 +295,40 @@ cudaError_t launch_prefill(const uint16_t* x, const int32_t* qweight, const uint
                      (uint64_t)n_groups, (uint64_t)N * 2, BW, (uint32_t)scale_rows,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
+  constexpr size_t smem = Layout<BT>::kSmemBytes;
   static std::once_flag attr_once[64];
   static cudaError_t attr_err[64];
   const int d = dev.device & 63;
   std::call_once(attr_once[d], [&] {
-    attr_err[d] = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
+    attr_err[d] = cudaFuncSetAttribute(prefill_kernel<BT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   });
   if (attr_err[d] != cudaSuccess) return attr_err[d];
   const dim3 grid((unsigned)((N + BW - 1) / BW), (unsigned)((M + BT - 1) / BT), 1);
-  prefill_kernel<<<grid, THREADS, kSmemBytes, stream>>>(x_map, qw_map, s_map, y, (int)M, (int)K,
-                                                       (int)N, group_shift, scale_rows,
-                                                       dev.error_word);
+  prefill_kernel<BT><<<grid, THREADS, smem, stream>>>(x_map, qw_map, s_map, y, (int)M, (int)K,
+                                                      (int)N, group_shift, scale_rows,
+                                                      dev.error_word);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+// The token tile follows M (64, 128 or 256 tokens per CTA), so that small M
+// does not pay for MMAs over empty token columns.
+cudaError_t launch_prefill(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                           uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
+                           cudaStream_t stream, const DeviceInfo& dev) {
+  const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
+                               ? 1 : (K + (int64_t(1) << group_shift) - 1) >> group_shift;
+  const int scale_rows = group_shift >= 6 ? 1 : (BK >> group_shift);
+  if (M <= 64)
+    return launch_t<64>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups, stream,
+                        dev);
+  if (M <= 128)
+    return launch_t<128>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups, stream,
+                         dev);
+  return launch_t<256>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups, stream,
+                       dev);
 }
 
 }  // namespace gptq

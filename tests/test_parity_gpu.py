@@ -124,6 +124,8 @@ EDGE = [  # (M, K, N, G)
     # 512 k for M <= 16), ragged last stages
     (4, 3072, 64, 1024), (3, 2304, 16, 512), (8, 6144, 24, 256), (1, 1600, 72, 512),
     (12, 2560, 40, 1024), (16, 1536, 200, 512),
+    # the 32-token tile (17 <= M <= 32)
+    (17, 528, 136, 128), (24, 2048, 72, 16), (32, 1040, 264, -1), (29, 6144, 40, 32),
 ]
 
 
@@ -139,7 +141,10 @@ def test_edge_shapes_small_m(M, K, N, G, kernel):
 
 
 @pytest.mark.parametrize("M,K,N,G", [(17, 64, 8, 16), (129, 528, 136, 128), (300, 96, 264, 32),
-                                     (257, 1040, 128, -1), (513, 160, 392, 64)])
+                                     (257, 1040, 128, -1), (513, 160, 392, 64),
+                                     # token tiles of 64 (M <= 64) and 128 (M <= 128)
+                                     (33, 96, 72, 32), (64, 160, 136, 64), (100, 528, 264, 128),
+                                     (128, 1040, 128, -1), (65, 2048, 200, 16)])
 def test_edge_shapes_prefill(M, K, N, G):
     p = W.make_problem(M, K, N, G, seed=M + K + N)
     y = run(p)
@@ -167,6 +172,20 @@ def test_all_codes_eight_gives_exact_zero(kernel):
     assert np.all(y.astype(np.float64) == 0.0)
 
 
+def test_one_hot_x_32_token_tile_bitwise():
+    """Decode with 32 tokens: every row one-hot at a different k."""
+    p = W.make_problem(32, 2048, 136, 64, seed=14)
+    ks = [0, 1, 2, 3, 4, 5, 6, 7, 8, 63, 64, 65, 127, 128, 255, 256, 511, 512, 777, 1000,
+          1023, 1024, 1500, 1535, 1536, 1600, 1800, 2000, 2040, 2045, 2046, 2047]
+    p.x[:] = 0
+    for m, k in enumerate(ks):
+        p.x[m, k] = 1
+    y = run(p, B.KERNEL_DECODE)
+    w = oracle.dequant(p.qweight, p.scales, 64)
+    for m, k in enumerate(ks):
+        assert np.array_equal(y[m].view(np.uint16), w[k].view(np.uint16)), (m, k)
+
+
 @pytest.mark.parametrize("kernel", [B.KERNEL_DECODE, B.KERNEL_PREFILL])
 def test_one_hot_x_reproduces_dequantised_rows_bitwise(kernel):
     p = W.make_problem(16, 1024, 264, 32, seed=4)
@@ -181,7 +200,7 @@ def test_one_hot_x_reproduces_dequantised_rows_bitwise(kernel):
 
 
 @pytest.mark.parametrize("kernel", [B.KERNEL_DECODE, B.KERNEL_PREFILL])
-@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("M", [1, 5, 16, 27, 32])
 def test_integer_exact_inputs_match_bitwise(kernel, M):
     """x in {-4..4}, scales 2^-6: every product and partial sum is exact in
     FP32, so any summation order gives the oracle's value exactly."""
@@ -195,7 +214,7 @@ def test_integer_exact_inputs_match_bitwise(kernel, M):
 
 
 @pytest.mark.parametrize("kernel,M", [(B.KERNEL_DECODE, 1), (B.KERNEL_DECODE, 16),
-                                      (B.KERNEL_PREFILL, 300)])
+                                      (B.KERNEL_DECODE, 32), (B.KERNEL_PREFILL, 300)])
 def test_deterministic(kernel, M):
     p = W.make_problem(M, 5120, 1024, 128, seed=9)
     a, b = run(p, kernel), run(p, kernel)
@@ -230,7 +249,7 @@ def test_decode_up_projection_full():
     check_rows(p, run(p), [0], "decode up-projection M=1")
 
 
-@pytest.mark.parametrize("M", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 16, 32])
 def test_decode_down_projection_sweep(M):
     p = W.decode_down(M)
     assert B.select(M, 17408, 5120, 32)[0] == B.KERNEL_DECODE
