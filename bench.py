@@ -247,6 +247,40 @@ def time_gemm(lib, torch, p, steps, warmup, kernel=0, stream=None, l2_bytes=0):
     return e0.elapsed_time(e1) / steps, copies
 
 
+def time_grouped(lib, torch, ps, steps, warmup, l2_bytes):
+    """Device time per call (ms) of back-to-back grouped calls (linears sharing
+    X), rotating enough weight copies that they do not stay in L2."""
+    total = sum(p.algorithmic_bytes for p in ps)
+    copies = max(1, -(-2 * l2_bytes // total) + 1)
+    sh = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    keep, argv = [], []
+    M, K, count = ps[0].M, ps[0].K, len(ps)
+    x = torch.from_numpy(ps[0].x.view(np.int16)).view(torch.float16).cuda()
+    for c in range(copies):
+        qws = [torch.from_numpy(p.qweight).cuda() for p in ps]
+        ss = [torch.from_numpy(p.scales.view(np.int16)).view(torch.float16).cuda() for p in ps]
+        ys = [torch.empty((M, p.N), dtype=torch.float16, device="cuda") for p in ps]
+        keep += qws + ss + ys
+        qa = (ctypes.c_void_p * count)(*[ctypes.c_void_p(t.data_ptr()) for t in qws])
+        sa = (ctypes.c_void_p * count)(*[ctypes.c_void_p(t.data_ptr()) for t in ss])
+        na = (ctypes.c_int64 * count)(*[p.N for p in ps])
+        ya = (ctypes.c_void_p * count)(*[ctypes.c_void_p(t.data_ptr()) for t in ys])
+        argv.append((ctypes.c_void_p(x.data_ptr()), qa, sa, na, count, M, K, ps[0].group, ya, sh))
+    fn = lib.gptq_w4a16_gemm_grouped
+    for i in range(warmup):
+        st = fn(*argv[i % copies])
+        if st:
+            raise RuntimeError(f"grouped gemm status {st}")
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        fn(*argv[i % copies])
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -404,6 +438,14 @@ def run_sweep(lib, torch, l2, hbm, tf):
         key = "ms"
         total = sum(res[f"layer_{n}_M{M}"][key] * c for n, _, _, c in W.LAYER_LINEARS)
         res[f"layer_total_M{M}_ms"] = round(total, 4)
+    # shared-input linears in one call (q/k/v: 3 x 5120->5120; gate+up: 2 x 5120->17408)
+    for name, count, N in (("qkv", 3, 5120), ("gate_up", 2, 17408)):
+        for M in (1, 16):
+            ps = [W.make_problem(M, 5120, N, 128, seed=i) for i in range(count)]
+            ms = time_grouped(lib, torch, ps, 200, 20, l2)
+            gbs = sum(p.algorithmic_bytes for p in ps) / (ms * 1e-3) / 1e9
+            res[f"grouped_{name}_M{M}"] = {"ms": round(ms, 5), "GB/s": round(gbs, 1),
+                                           "frac_hbm": round(gbs / hbm, 3)}
     return res
 
 

@@ -69,6 +69,7 @@ typedef enum {
 #define GPTQ_MAX_N 1048576
 #define GPTQ_MAX_M 8388608
 #define GPTQ_DECODE_MAX_M 32
+#define GPTQ_MAX_GROUPED 8     /* linears per gptq_w4a16_gemm_grouped call */
 
 /*
  * Y = X . dequant(qweight, scales).
@@ -106,6 +107,33 @@ GPTQ_API int gptq_w4a16_gemm_decode_splits(const uint16_t* x, const int32_t* qwe
                                            const uint16_t* scales, int64_t M, int64_t K,
                                            int64_t N, int32_t group, uint16_t* y, void* stream,
                                            int32_t splits);
+
+/*
+ * Several linears that share one input X, for example the q, k and v
+ * projections or the gate and up projections of a layer:
+ *   Y_i = X . dequant(qweights[i], scales[i]),   i = 0 .. count-1.
+ * The GPTQModel wiki ("Installation and Quickstart") describes engines that
+ * merge such linears into one (gate_up_proj, qkv_proj); here each linear keeps
+ * its own native qweight and scales, and X is shared.
+ *   x          [M, K] FP16 bits, device (may be NULL only when M == 0)
+ *   qweights   HOST array of `count` device pointers, qweights[i] [K/8, Ns[i]]
+ *   scales     HOST array of `count` device pointers, scales[i] [n_groups, Ns[i]]
+ *              (one group size and one K for all linears)
+ *   Ns         HOST array of `count` output widths, each > 0 and % 8 == 0
+ *   ys         HOST array of `count` device pointers, ys[i] [M, Ns[i]], written;
+ *              pairwise disjoint and not overlapping x, any qweight or any scales
+ *   count      1 .. GPTQ_MAX_GROUPED
+ * For M <= GPTQ_DECODE_MAX_M all linears are computed by ONE decode launch
+ * (one X read, one fixed launch cost); for larger M each linear gets its own
+ * prefill launch.  The host arrays are read during the call only.  Results
+ * are within the same tolerance as separate calls, and deterministic.
+ * Errors as gptq_w4a16_gemm (any linear failing a check fails the call before
+ * anything is enqueued), plus GPTQ_ERR_SHAPE for count out of range.
+ */
+GPTQ_API int gptq_w4a16_gemm_grouped(const uint16_t* x, const int32_t* const* qweights,
+                                     const uint16_t* const* scales, const int64_t* Ns,
+                                     int32_t count, int64_t M, int64_t K, int32_t group,
+                                     uint16_t* const* ys, void* stream);
 
 /*
  * W[K, N] = dequant(qweight, scales) as FP16 bits, each value rounded once from

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libgptq_w4a16.so")
 
 KERNEL_AUTO, KERNEL_DECODE, KERNEL_PREFILL = 0, 1, 2
 DECODE_MAX_M = 32
+MAX_GROUPED = 8
 GROUP_SIZES = (-1, 16, 32, 64, 128, 256, 512, 1024)
 
 STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_NULL", 2: "GPTQ_ERR_SHAPE", 3: "GPTQ_ERR_GROUP",
@@ -27,7 +28,7 @@ STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_NULL", 2: "GPTQ_ERR_SHAPE", 3: "GPTQ_ERR_GR
 
 # Every entry point declared in include/gptq_w4a16.h.
 EXPORTS = ("gptq_w4a16_gemm", "gptq_w4a16_gemm_kernel", "gptq_w4a16_gemm_decode_splits",
-           "gptq_dequant", "gptq_w4a16_select", "gptq_status_string", "gptq_device_error",
+           "gptq_w4a16_gemm_grouped", "gptq_dequant", "gptq_w4a16_select", "gptq_status_string", "gptq_device_error",
            "gptq_version")
 
 
@@ -59,6 +60,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.gptq_w4a16_gemm.argtypes = gemm_args
             lib.gptq_w4a16_gemm_kernel.argtypes = gemm_args + [_i32]
             lib.gptq_w4a16_gemm_decode_splits.argtypes = gemm_args + [_i32]
+            lib.gptq_w4a16_gemm_grouped.argtypes = [_p, _p, _p, _p, _i32, _i64, _i64, _i32,
+                                                    _p, _p]
             lib.gptq_dequant.argtypes = [_p, _p, _i64, _i64, _i32, _p, _p]
             lib.gptq_w4a16_select.argtypes = [_i64, _i64, _i64, _i32,
                                               ctypes.POINTER(_i32), ctypes.POINTER(_i32)]
@@ -67,7 +70,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.gptq_device_error.argtypes = []
             lib.gptq_version.restype = ctypes.c_char_p
             for name in ("gptq_w4a16_gemm", "gptq_w4a16_gemm_kernel",
-                         "gptq_w4a16_gemm_decode_splits", "gptq_dequant",
+                         "gptq_w4a16_gemm_decode_splits", "gptq_w4a16_gemm_grouped",
+                         "gptq_dequant",
                          "gptq_w4a16_select", "gptq_device_error"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
@@ -146,6 +150,44 @@ def gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, group: in
     else:
         _check(lib.gptq_w4a16_gemm_kernel(*args, kernel))
     return out
+
+
+def gemm_grouped(x: torch.Tensor, qweights, scales, group: int, outs=None,
+                 stream=None) -> list:
+    """Y_i = x . dequant(qweights[i], scales[i]) for linears sharing x (one
+    decode launch for M <= DECODE_MAX_M)."""
+    lib = load()
+    if not 1 <= len(qweights) <= MAX_GROUPED or len(scales) != len(qweights):
+        raise ValueError(f"need 1..{MAX_GROUPED} linears with one scales tensor each")
+    dev = qweights[0].device
+    _require(x, "x", lambda d: d == torch.float16, dev)
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D")
+    M, K = x.shape
+    Ns = []
+    for i, (qw, sc) in enumerate(zip(qweights, scales)):
+        _require(qw, f"qweights[{i}]", lambda d: d == torch.int32, dev)
+        _require(sc, f"scales[{i}]", lambda d: d == torch.float16, dev)
+        if qw.dim() != 2 or qw.shape[0] * 8 != K:
+            raise ValueError(f"qweights[{i}] does not match K={K}")
+        Ns.append(qw.shape[1])
+    if outs is None:
+        outs = [torch.empty((M, n), dtype=torch.float16, device=dev) for n in Ns]
+    else:
+        if len(outs) != len(Ns):
+            raise ValueError("one output per linear")
+        for i, (o, n) in enumerate(zip(outs, Ns)):
+            _require(o, f"outs[{i}]", lambda d: d == torch.float16, dev)
+            if tuple(o.shape) != (M, n):
+                raise ValueError(f"outs[{i}] has shape {tuple(o.shape)}, expected {(M, n)}")
+    count = len(Ns)
+    qa = (ctypes.c_void_p * count)(*[_ptr(q) for q in qweights])
+    sa = (ctypes.c_void_p * count)(*[_ptr(t) for t in scales])
+    na = (ctypes.c_int64 * count)(*Ns)
+    ya = (ctypes.c_void_p * count)(*[_ptr(o) for o in outs])
+    _check(lib.gptq_w4a16_gemm_grouped(_ptr(x), qa, sa, na, count, M, K, group, ya,
+                                       _stream_handle(stream, dev)))
+    return outs
 
 
 def dequant(qweight: torch.Tensor, scales: torch.Tensor, group: int,

@@ -160,6 +160,56 @@ int gptq_w4a16_gemm_decode_splits(const uint16_t* x, const int32_t* qweight,
   return gemm_impl(x, qweight, scales, M, K, N, group, y, stream, GPTQ_KERNEL_DECODE, splits);
 }
 
+int gptq_w4a16_gemm_grouped(const uint16_t* x, const int32_t* const* qweights,
+                            const uint16_t* const* scales, const int64_t* Ns, int32_t count,
+                            int64_t M, int64_t K, int32_t group, uint16_t* const* ys,
+                            void* stream) {
+  if (count < 1 || count > GPTQ_MAX_GROUPED) return GPTQ_ERR_SHAPE;
+  if (!qweights || !scales || !Ns || !ys) return GPTQ_ERR_NULL;
+  for (int i = 0; i < count; ++i) {
+    const int st = check_shape(M, K, Ns[i], group);
+    if (st != GPTQ_OK) return st;
+  }
+  for (int i = 0; i < count; ++i)
+    if (!qweights[i] || !scales[i]) return GPTQ_ERR_NULL;
+  if (M == 0) return GPTQ_OK;
+  if (!x) return GPTQ_ERR_NULL;
+  for (int i = 0; i < count; ++i)
+    if (!ys[i]) return GPTQ_ERR_NULL;
+  if (!aligned16(x)) return GPTQ_ERR_ALIGN;
+  for (int i = 0; i < count; ++i)
+    if (!aligned16(qweights[i]) || !aligned16(scales[i]) || !aligned16(ys[i]))
+      return GPTQ_ERR_ALIGN;
+  const int64_t ng = num_groups(K, group);
+  for (int i = 0; i < count; ++i) {
+    const int64_t ybytes = M * Ns[i] * 2;
+    if (overlaps(ys[i], ybytes, x, M * K * 2)) return GPTQ_ERR_ALIAS;
+    for (int j = 0; j < count; ++j) {
+      if (overlaps(ys[i], ybytes, qweights[j], K / 8 * Ns[j] * 4) ||
+          overlaps(ys[i], ybytes, scales[j], ng * Ns[j] * 2) ||
+          (j != i && overlaps(ys[i], ybytes, ys[j], M * Ns[j] * 2)))
+        return GPTQ_ERR_ALIAS;
+    }
+  }
+  const DeviceInfo* dev = nullptr;
+  const int st = query_device(&dev);
+  if (st != GPTQ_OK) return st;
+  const int gs = group_shift_of(group);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (M <= GPTQ_DECODE_MAX_M) {
+    e = launch_decode_grouped(x, qweights, scales, Ns, ys, count, M, K, gs, s, *dev);
+  } else {
+    for (int i = 0; i < count && e == cudaSuccess; ++i)
+      e = launch_prefill(x, qweights[i], scales[i], ys[i], M, K, Ns[i], gs, s, *dev);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  return GPTQ_OK;
+}
+
 int gptq_dequant(const int32_t* qweight, const uint16_t* scales, int64_t K, int64_t N,
                  int32_t group, uint16_t* w_out, void* stream) {
   int st = check_shape(0, K, N, group);

@@ -50,6 +50,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "gptq_w4a16.h"
 #include "kernels.h"
 #include "tc05.cuh"
 #include "tmap.h"
@@ -136,6 +137,20 @@ struct DecodeBars {
   int abort_flag;
 };
 
+constexpr int kMaxLinears = GPTQ_MAX_GROUPED;
+
+// The linears of one launch: one for a plain call, several that share X for
+// a grouped call.  Per linear its tensor maps, output and width, and the first
+// column block of the grid that it owns (blk0[count] = total blocks).
+struct LinearSet {
+  CUtensorMap qw[kMaxLinears];
+  CUtensorMap sc[kMaxLinears];
+  uint16_t* y[kMaxLinears];
+  int n[kMaxLinears];
+  int blk0[kMaxLinears + 1];
+  int count;
+};
+
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
@@ -184,10 +199,8 @@ __device__ __forceinline__ void permute_x_chunk(uint8_t* p) {
 // one 2-D box per 64-k atom.
 template <int WPS, int BT>
 __global__ void __launch_bounds__(THREADS, 1)
-    decode_kernel(const __grid_constant__ CUtensorMap x_map,
-                  const __grid_constant__ CUtensorMap qw_map,
-                  const __grid_constant__ CUtensorMap s_map, uint16_t* __restrict__ y, int M,
-                  int K, int N, int group_shift, int stages, int stage_bytes, int scale_rows,
+    decode_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ LinearSet ls,
+                  int M, int K, int group_shift, int stages, int stage_bytes, int scale_rows,
                   int x3d, int* err) {
   constexpr int X_ATOM_BYTES = TokGeo<BT>::X_ATOM_BYTES;
   constexpr int X_STAGE_BYTES = TokGeo<BT>::X_STAGE_BYTES;
@@ -202,7 +215,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   volatile int* abort_flag = &bar->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BW;
+  // this CTA's linear and column block
+  int li = 0;
+  while (li + 1 < ls.count && (int)blockIdx.x >= ls.blk0[li + 1]) ++li;
+  const CUtensorMap* qw_map = &ls.qw[li];
+  const CUtensorMap* s_map = &ls.sc[li];
+  uint16_t* __restrict__ y = ls.y[li];
+  const int N = ls.n[li];
+  const int n0 = ((int)blockIdx.x - ls.blk0[li]) * BW;
   const int NS = ((K >> 3) + PRS - 1) / PRS;  // stages over all of K
   const int splits = gridDim.y;
   const int st_begin = (int)((int64_t)blockIdx.y * NS / splits);
@@ -225,11 +245,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&x_map);
-    prefetch_tensormap(&qw_map);
-    prefetch_tensormap(&s_map);
+    prefetch_tensormap(qw_map);
+    prefetch_tensormap(s_map);
     // L2 prefetch of the first stages' weight tiles: safe before the wait
     const int pf = min(n_st, 2);
-    for (int t = 0; t < pf; ++t) tma_prefetch_l2_2d(&qw_map, n0, (st_begin + t) * PRS);
+    for (int t = 0; t < pf; ++t) tma_prefetch_l2_2d(qw_map, n0, (st_begin + t) * PRS);
   }
   if (warp == 1) {
     tmem_alloc(&bar->tmem_base, TMEM_COLS);
@@ -262,8 +282,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int k0 = (st_begin + t) * BKS;
         mbar_arrive_expect_tx(&bar->full[s],
                               X_STAGE_BYTES + QW_STAGE_BYTES + scale_rows * S_ROW_BYTES);
-        tma_load_2d(st + QW_OFF, &qw_map, n0, k0 >> 3, &bar->full[s]);
-        tma_load_2d(st + S_OFF, &s_map, n0, k0 >> gs, &bar->full[s]);
+        tma_load_2d(st + QW_OFF, qw_map, n0, k0 >> 3, &bar->full[s]);
+        tma_load_2d(st + S_OFF, s_map, n0, k0 >> gs, &bar->full[s]);
         if (x3d) {
           tma_load_3d(st, &x_map, 0, 0, k0 >> 6, &bar->full[s]);
         } else {
@@ -498,9 +518,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 template <int WPS, int BT>
-cudaError_t launch_t(const CUtensorMap& x_map, const CUtensorMap& qw_map, const CUtensorMap& s_map,
-                     uint16_t* y, int M, int K, int N, int group_shift, int splits, int x3d,
-                     const DecodeShape& d, cudaStream_t stream, const DeviceInfo& dev) {
+cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, int M, int K, int group_shift,
+                     int splits, int x3d, const DecodeShape& d, cudaStream_t stream,
+                     const DeviceInfo& dev) {
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
   const int di = dev.device & 63;
@@ -511,7 +531,7 @@ cudaError_t launch_t(const CUtensorMap& x_map, const CUtensorMap& qw_map, const 
   });
   if (attr_err[di] != cudaSuccess) return attr_err[di];
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((N + BW - 1) / BW), (unsigned)splits, 1);
+  cfg.gridDim = dim3((unsigned)ls.blk0[ls.count], (unsigned)splits, 1);
   cfg.blockDim = dim3(THREADS, 1, 1);
   cfg.dynamicSmemBytes = (size_t)d.smem_bytes;
   cfg.stream = stream;
@@ -529,19 +549,87 @@ cudaError_t launch_t(const CUtensorMap& x_map, const CUtensorMap& qw_map, const 
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT>, x_map, qw_map, s_map, y, M, K, N,
-                            group_shift, d.stages, d.stage_bytes, d.scale_rows, x3d,
-                            dev.error_word);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT>, x_map, ls, M, K, group_shift, d.stages,
+                            d.stage_bytes, d.scale_rows, x3d, dev.error_word);
+}
+
+// One linear of a launch, as the host sees it.
+struct LinearArgs {
+  const int32_t* qweight;
+  const uint16_t* scales;
+  uint16_t* y;
+  int64_t n;
+};
+
+// Tensor maps and launch for a token tile of BT over `count` linears that
+// share X (count = 1 for a plain call).
+template <int BT>
+cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count, int64_t M, int64_t K,
+                      int group_shift, int splits, cudaStream_t stream, const DeviceInfo& dev) {
+  const DecodeShape d = decode_shape<BT>(group_shift);
+  if (d.stages < GROUPS || d.smem_bytes > 1024 + kRingBudget + 256) return cudaErrorInvalidValue;
+  if (count < 1 || count > kMaxLinears) return cudaErrorInvalidValue;
+  const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
+                               ? 1 : (K + (int64_t(1) << group_shift) - 1) >> group_shift;
+  LinearSet ls;
+  ls.count = count;
+  ls.blk0[0] = 0;
+  for (int i = 0; i < count; ++i) {
+    const uint64_t N = (uint64_t)lin[i].n;
+    if (!tensor_map_2d(&ls.qw[i], lin[i].qweight, CU_TENSOR_MAP_DATA_TYPE_INT32, N,
+                       (uint64_t)(K / 8), N * 4, BW, PRS, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !tensor_map_2d(&ls.sc[i], lin[i].scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, N,
+                       (uint64_t)n_groups, N * 2, BW, (uint32_t)d.scale_rows,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    ls.y[i] = lin[i].y;
+    ls.n[i] = (int)N;
+    ls.blk0[i + 1] = ls.blk0[i] + (int)((N + BW - 1) / BW);
+  }
+  for (int i = count; i < kMaxLinears; ++i) {
+    ls.qw[i] = ls.qw[0];
+    ls.sc[i] = ls.sc[0];
+    ls.y[i] = nullptr;
+    ls.n[i] = 0;
+    ls.blk0[i + 1] = ls.blk0[count];
+  }
+  // X as [K/64 atoms][M tokens][64 k] (one box per stage) when K is a
+  // multiple of 64, else as [M][K] in one box per 64-k atom; rows at or beyond
+  // M and k at or beyond K read as zero either way
+  CUtensorMap x_map;
+  int x3d = 0;
+  if (K % 64 == 0) {
+    const uint64_t dims[3] = {64, (uint64_t)M, (uint64_t)(K / 64)};
+    const uint64_t strides[2] = {(uint64_t)K * 2, 128};
+    const uint32_t box[3] = {64, BT, X_ATOMS};
+    x3d = tensor_map_3d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, dims, strides, box,
+                        CU_TENSOR_MAP_SWIZZLE_128B) ? 1 : 0;
+  }
+  if (!x3d && !tensor_map_2d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K,
+                             (uint64_t)M, (uint64_t)K * 2, 64, BT, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (splits <= 0) splits = decode_pick_splits_blocks(ls.blk0[count], K, dev);
+  const int iM = (int)M, iK = (int)K;
+  if (group_shift == 4)
+    return launch_t<2, BT>(x_map, ls, iM, iK, group_shift, splits, x3d, d, stream, dev);
+  if (group_shift == 5)
+    return launch_t<4, BT>(x_map, ls, iM, iK, group_shift, splits, x3d, d, stream, dev);
+  return launch_t<WPT, BT>(x_map, ls, iM, iK, group_shift, splits, x3d, d, stream, dev);
+}
+
+cudaError_t launch_set(const uint16_t* x, const LinearArgs* lin, int count, int64_t M, int64_t K,
+                       int group_shift, int splits, cudaStream_t stream, const DeviceInfo& dev) {
+  // token tile: 16 tokens up to M = 16, else 32
+  if (M <= 16) return launch_bt<16>(x, lin, count, M, K, group_shift, splits, stream, dev);
+  return launch_bt<32>(x, lin, count, M, K, group_shift, splits, stream, dev);
 }
 
 }  // namespace
 
-int decode_pick_splits(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev) {
+int decode_pick_splits_blocks(int64_t nblk, int64_t K, const DeviceInfo& dev) {
   // One CTA per SM.  Pick the split that minimises (waves of CTAs) x (stages
   // per CTA) plus one stage for the cluster reduction, among splits whose
   // CTAs are all resident at once.  Ties go to the smaller split.
-  (void)M;
-  const int64_t nblk = (N + BW - 1) / BW;
   const int64_t ns = ((K >> 3) + PRS - 1) / PRS;
   const int64_t sms = dev.num_sms;
   int best = 1;
@@ -558,59 +646,26 @@ int decode_pick_splits(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev) {
   return best;
 }
 
-namespace {
-
-// Tensor maps and launch for a token tile of BT.
-template <int BT>
-cudaError_t launch_bt(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
-                      uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift, int splits,
-                      cudaStream_t stream, const DeviceInfo& dev) {
-  const DecodeShape d = decode_shape<BT>(group_shift);
-  if (d.stages < GROUPS || d.smem_bytes > 1024 + kRingBudget + 256) return cudaErrorInvalidValue;
-  const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
-                               ? 1 : (K + (int64_t(1) << group_shift) - 1) >> group_shift;
-  CUtensorMap x_map, qw_map, s_map;
-  if (!tensor_map_2d(&qw_map, qweight, CU_TENSOR_MAP_DATA_TYPE_INT32, (uint64_t)N,
-                     (uint64_t)(K / 8), (uint64_t)N * 4, BW, PRS, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !tensor_map_2d(&s_map, scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, (uint64_t)N,
-                     (uint64_t)n_groups, (uint64_t)N * 2, BW, (uint32_t)d.scale_rows,
-                     CU_TENSOR_MAP_SWIZZLE_NONE))
-    return cudaErrorInvalidValue;
-  // X as [K/64 atoms][M tokens][64 k] (one box per stage) when K is a
-  // multiple of 64, else as [M][K] in one box per 64-k atom; rows at or beyond
-  // M and k at or beyond K read as zero either way
-  int x3d = 0;
-  if (K % 64 == 0) {
-    const uint64_t dims[3] = {64, (uint64_t)M, (uint64_t)(K / 64)};
-    const uint64_t strides[2] = {(uint64_t)K * 2, 128};
-    const uint32_t box[3] = {64, BT, X_ATOMS};
-    x3d = tensor_map_3d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, dims, strides, box,
-                        CU_TENSOR_MAP_SWIZZLE_128B) ? 1 : 0;
-  }
-  if (!x3d && !tensor_map_2d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K,
-                             (uint64_t)M, (uint64_t)K * 2, 64, BT, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  const int iM = (int)M, iK = (int)K, iN = (int)N;
-  if (group_shift == 4)
-    return launch_t<2, BT>(x_map, qw_map, s_map, y, iM, iK, iN, group_shift, splits, x3d, d,
-                           stream, dev);
-  if (group_shift == 5)
-    return launch_t<4, BT>(x_map, qw_map, s_map, y, iM, iK, iN, group_shift, splits, x3d, d,
-                           stream, dev);
-  return launch_t<WPT, BT>(x_map, qw_map, s_map, y, iM, iK, iN, group_shift, splits, x3d, d,
-                           stream, dev);
+int decode_pick_splits(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev) {
+  (void)M;
+  return decode_pick_splits_blocks((N + BW - 1) / BW, K, dev);
 }
-
-}  // namespace
 
 cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                           uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
                           int splits, cudaStream_t stream, const DeviceInfo& dev) {
-  if (splits <= 0) splits = decode_pick_splits(M, K, N, dev);
-  // token tile: 16 tokens up to M = 16, else 32
-  if (M <= 16)
-    return launch_bt<16>(x, qweight, scales, y, M, K, N, group_shift, splits, stream, dev);
-  return launch_bt<32>(x, qweight, scales, y, M, K, N, group_shift, splits, stream, dev);
+  const LinearArgs one{qweight, scales, y, N};
+  return launch_set(x, &one, 1, M, K, group_shift, splits, stream, dev);
+}
+
+cudaError_t launch_decode_grouped(const uint16_t* x, const int32_t* const* qweights,
+                                  const uint16_t* const* scales, const int64_t* ns,
+                                  uint16_t* const* ys, int count, int64_t M, int64_t K,
+                                  int group_shift, cudaStream_t stream, const DeviceInfo& dev) {
+  if (count < 1 || count > kMaxLinears) return cudaErrorInvalidValue;
+  LinearArgs lin[kMaxLinears];
+  for (int i = 0; i < count; ++i) lin[i] = LinearArgs{qweights[i], scales[i], ys[i], ns[i]};
+  return launch_set(x, lin, count, M, K, group_shift, 0, stream, dev);
 }
 
 }  // namespace gptq

@@ -34,9 +34,16 @@ cudaError_t launch_dequant(const int32_t* qweight, const uint16_t* scales, int64
 // Decode (M <= 32).  splits = number of CTAs that share one column block along
 // K (the cluster size, 1..8); 0 picks it from the shape.
 int decode_pick_splits(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev);
+int decode_pick_splits_blocks(int64_t column_blocks, int64_t K, const DeviceInfo& dev);
 cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                           uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
                           int splits, cudaStream_t stream, const DeviceInfo& dev);
+// Decode of `count` linears that share X (1..GPTQ_MAX_GROUPED), one launch;
+// the split is picked from the total number of column blocks.
+cudaError_t launch_decode_grouped(const uint16_t* x, const int32_t* const* qweights,
+                                  const uint16_t* const* scales, const int64_t* ns,
+                                  uint16_t* const* ys, int count, int64_t M, int64_t K,
+                                  int group_shift, cudaStream_t stream, const DeviceInfo& dev);
 
 // Prefill (any M >= 1): TMA + tcgen05 with TMEM accumulators.
 cudaError_t launch_prefill(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,

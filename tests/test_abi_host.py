@@ -119,3 +119,41 @@ def test_missing_library_fails_loudly(tmp_path):
             binding.load(str(tmp_path / "nope.so"))
         finally:
             binding._lib = saved
+
+
+# ---- gptq_w4a16_gemm_grouped: host-side checks ------------------------------
+
+Y2, QW2, S2 = 0xC00000, 0x1000000, 0x1400000
+
+
+def call_grouped(lib, count=2, x=X, qws=(QW, QW2), ss=(S, S2), ns=(256, 136), ys=(Y, Y2),
+                 M=4, K=512, g=128, arrays=True):
+    n = max(count, 1)
+    qa = (ctypes.c_void_p * n)(*[ctypes.c_void_p(v) for v in (list(qws) + [QW] * n)[:n]])
+    sa = (ctypes.c_void_p * n)(*[ctypes.c_void_p(v) for v in (list(ss) + [S] * n)[:n]])
+    na = (ctypes.c_int64 * n)(*(list(ns) + [256] * n)[:n])
+    ya = (ctypes.c_void_p * n)(*[ctypes.c_void_p(v) for v in (list(ys) + [Y] * n)[:n]])
+    if not arrays:
+        qa = sa = na = ya = None
+    return lib.gptq_w4a16_gemm_grouped(ctypes.c_void_p(x), qa, sa, na, count, M, K, g, ya, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(count=0), 2), (dict(count=9), 2), (dict(arrays=False), 1),
+    (dict(ns=(256, 252)), 2), (dict(ns=(256, 0)), 2), (dict(K=520), 2), (dict(g=100), 3),
+    (dict(qws=(QW, 0)), 1), (dict(ss=(0, S2)), 1), (dict(x=0), 1), (dict(ys=(Y, 0)), 1),
+    (dict(ys=(Y, Y2 + 2)), 4), (dict(qws=(QW + 4, QW2)), 4), (dict(x=X + 2), 4),
+    (dict(ys=(Y, Y + 16)), 8),            # two outputs overlap
+    (dict(ys=(Y, QW + 64)), 8),           # an output overlaps another linear's qweight
+    (dict(ys=(S2, Y2)), 8),               # an output overlaps another linear's scales
+    (dict(ys=(X, Y2)), 8),                # an output overlaps x
+])
+def test_grouped_argument_checks(lib, kw, status):
+    assert call_grouped(lib, **kw) == status
+
+
+def test_grouped_empty_m_and_no_device(lib):
+    import torch
+    assert call_grouped(lib, M=0, x=0, ys=(0, 0)) == 0
+    if not torch.cuda.is_available():
+        assert call_grouped(lib) == 5

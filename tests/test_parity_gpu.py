@@ -275,3 +275,63 @@ def test_group_sweep(G, M):
 def test_layer_linears(which, M):
     p = W.layer_linear(which, M)
     check_rows(p, run(p), sample_rows(M, 2), f"layer {which} M={M}")
+
+
+# ---- several linears sharing X in one call ------------------------------------
+
+def grouped_problem(M, K, Ns, G, seed):
+    ps = [W.make_problem(M, K, n, G, seed=seed + i) for i, n in enumerate(Ns)]
+    for q in ps[1:]:
+        q.x[:] = ps[0].x  # one shared X
+    return ps
+
+
+def run_grouped(ps):
+    x = torch.from_numpy(ps[0].x.view(np.int16)).view(torch.float16).cuda()
+    qws = [torch.from_numpy(p.qweight).cuda() for p in ps]
+    ss = [torch.from_numpy(p.scales.view(np.int16)).view(torch.float16).cuda() for p in ps]
+    ys = B.gemm_grouped(x, qws, ss, ps[0].group)
+    torch.cuda.synchronize()
+    return [y.cpu().numpy() for y in ys]
+
+
+@pytest.mark.parametrize("M,K,Ns,G", [
+    (1, 2048, (264, 136, 8), 128), (5, 1040, (72, 200), 32), (16, 2560, (128, 128, 40, 8), 16),
+    (32, 1536, (136, 264), -1), (33, 528, (64, 24), 128),   # M = 33: one prefill launch each
+    (3, 512, (8, 8, 8, 8, 8, 8, 8, 8), 64),                  # the most linears per call
+])
+def test_grouped_parity(M, K, Ns, G):
+    ps = grouped_problem(M, K, Ns, G, seed=M + K)
+    ys = run_grouped(ps)
+    for i, (p, y) in enumerate(zip(ps, ys)):
+        ref = oracle.gemm(p.x, p.qweight, p.scales, G)
+        err = rel_err(y, ref)
+        print(f"[parity] grouped M={M} K={K} linear {i} N={p.N} G={G}: {err:.3e}")
+        assert err <= TOL
+
+
+def test_grouped_one_hot_bitwise():
+    ps = grouped_problem(16, 1024, (264, 136), 32, seed=21)
+    ks = [0, 1, 7, 8, 100, 511, 512, 777, 1000, 1023, 64, 65, 3, 300, 900, 31]
+    for p in ps:
+        p.x[:] = 0
+        for m, k in enumerate(ks):
+            p.x[m, k] = 1
+    ys = run_grouped(ps)
+    for p, y in zip(ps, ys):
+        w = oracle.dequant(p.qweight, p.scales, 32)
+        for m, k in enumerate(ks):
+            assert np.array_equal(y[m].view(np.uint16), w[k].view(np.uint16)), (m, k)
+
+
+def test_grouped_single_linear_equals_plain_call_bitwise():
+    p = W.make_problem(7, 4096, 392, 128, seed=22)
+    (y,) = run_grouped([p])
+    assert np.array_equal(y.view(np.uint16), run(p).view(np.uint16))
+
+
+def test_grouped_qkv_full_size():
+    ps = grouped_problem(1, 5120, (5120, 5120, 5120), 128, seed=23)
+    ys = run_grouped(ps)
+    for i, (p, y) in enumerate(zip(ps, ys)):
+        check_rows(p, y, [0], f"grouped q/k/v linear {i}")
