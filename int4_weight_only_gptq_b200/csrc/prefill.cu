@@ -44,47 +44,69 @@ namespace {
 constexpr int BW = 128;  // weight columns per CTA (MMA M; one TMEM lane each)
 constexpr int BT_MAX = 256;  // tokens per CTA (MMA N): 64, 128 or 256, by M
 constexpr int BK = 64;   // k per pipeline stage (four k16 MMAs)
-constexpr int STAGES = 4;
+constexpr int XS = 4;        // X ring stages (BT x 64 k each)
+constexpr int WS = 8;        // weight-tile ring stages (qweight + scales of 64 k)
+constexpr int AS = 8;        // A slots in TMEM (64 k each)
 constexpr int DQ_WARPS = 8;  // dequantisation + epilogue warps
-constexpr int THREADS = (2 + DQ_WARPS) * 32;
+constexpr int DQ_WARP0 = 3;  // warps 0, 1, 2: X producer, MMA issuer, weight producer
+constexpr int THREADS = (DQ_WARP0 + DQ_WARPS) * 32;
 constexpr int QW_STAGE_BYTES = BW * (BK / 8) * 4;  // 128 columns x 8 packed rows: 4 KB
 constexpr int S_ROW_BYTES = BW * 2;                // one scale row of the tile: 256 B
 constexpr int S_STAGE_MAX_ROWS = BK / 16;          // group 16: four rows per stage
+constexpr int W_STAGE_BYTES = QW_STAGE_BYTES + S_STAGE_MAX_ROWS * S_ROW_BYTES;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t D_COL = 0;                 // accumulator: columns [0, BT)
-constexpr uint32_t A_COL = 256;               // A stages: [256, 256 + 4 * 32)
+constexpr uint32_t A_COL = 256;               // A slots: [256, 256 + 8 * 32)
 constexpr uint32_t A_STAGE_COLS = BK / 2;     // two FP16 per 32-bit column
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint64_t kDrainLimitNs = 200000000ull;
+static_assert(BT_MAX <= A_COL, "accumulator below the A slots");
+static_assert(A_COL + AS * A_STAGE_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(AS == WS, "a weight stage and its A slot share an index");
 
-// Shared-memory layout for a token tile of BT: the X ring, then the qweight
-// and scale rings, then the barriers.
+// Shared-memory layout for a token tile of BT: the X ring, then the weight
+// ring (qweight then scale rows per stage), then the barriers.
 template <int BT>
 struct Layout {
   static constexpr int X_STAGE_BYTES = BT * BK * 2;
-  static constexpr int QW_OFF = STAGES * X_STAGE_BYTES;
-  static constexpr int S_OFF = QW_OFF + STAGES * QW_STAGE_BYTES;
-  static constexpr int BAR_OFF = S_OFF + STAGES * S_STAGE_MAX_ROWS * S_ROW_BYTES;
-  static constexpr size_t kSmemBytes = 1024 + (size_t)BAR_OFF + 256;
+  static constexpr int W_OFF = XS * X_STAGE_BYTES;
+  static constexpr int BAR_OFF = W_OFF + WS * W_STAGE_BYTES;
+  static constexpr size_t kSmemBytes = 1024 + (size_t)BAR_OFF + 512;
 };
-static_assert(BT_MAX <= A_COL, "accumulator below the A stages");
 
 struct Barriers {
-  uint64_t xfull[STAGES];   // X tile landed (TMA transaction count)
-  uint64_t afull[STAGES];   // A stage written by all dequantisation threads
-  uint64_t empty[STAGES];   // MMAs of the stage done: X slot and A columns free
-  uint64_t dfull;           // all MMAs of the tile done
+  uint64_t xfull[XS];    // X tile landed (TMA transaction count)
+  uint64_t xempty[XS];   // MMAs reading the X tile done
+  uint64_t wfull[WS];    // qweight and scale tiles landed
+  uint64_t wempty[WS];   // weight tiles read by every dequantisation warp
+  uint64_t afull[AS];    // A slot written by every dequantisation thread
+  uint64_t aempty[AS];   // MMAs reading the A slot done
+  uint64_t dfull;        // all MMAs of the tile done
   uint32_t tmem_base;
   int abort_flag;
 };
+static_assert(sizeof(Barriers) <= 512, "barrier area");
 
 __device__ __forceinline__ void record_timeout(int* err, Barriers* b) {
   atomicExch(err, kDeviceErrTimeout);
   *reinterpret_cast<volatile int*>(&b->abort_flag) = 1;
 }
 
+// One lane of a converged warp (the lowest active one) returns true.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(p));
+  return p != 0;
+}
+
 // scale_rows: scale rows one 64-k stage touches (1, or 64/group for groups
 // below 64); stages start on 64-k boundaries, so they align with groups.
+//
+// The X tiles and the weight tiles travel in separate rings: the weight ring
+// and the A slots are twice as deep as the X ring, so the dequantisation runs
+// up to eight stages ahead of the MMAs while the large X tiles only need four.
 template <int BT>
 __global__ void __launch_bounds__(THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap x_map,
@@ -93,8 +115,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                    int K, int N, int group_shift, int scale_rows, int* err) {
   static_assert(BT >= 64 && BT <= BT_MAX && BT % 64 == 0, "token tile");
   constexpr int X_STAGE_BYTES = Layout<BT>::X_STAGE_BYTES;
-  constexpr int QW_OFF = Layout<BT>::QW_OFF;
-  constexpr int S_OFF = Layout<BT>::S_OFF;
+  constexpr int W_OFF = Layout<BT>::W_OFF;
   constexpr int BAR_OFF = Layout<BT>::BAR_OFF;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array itself so that the
@@ -110,10 +131,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int KB = (K + BK - 1) / BK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < XS; ++s) {
       mbar_init(&bar->xfull[s], 1);
-      mbar_init(&bar->afull[s], DQ_WARPS * 32);
-      mbar_init(&bar->empty[s], 1);
+      mbar_init(&bar->xempty[s], 1);
+    }
+    for (int j = 0; j < WS; ++j) {
+      mbar_init(&bar->wfull[j], 1);
+      mbar_init(&bar->wempty[j], DQ_WARPS);
+      mbar_init(&bar->afull[j], DQ_WARPS * 32);
+      mbar_init(&bar->aempty[j], 1);
     }
     mbar_init(&bar->dfull, 1);
     bar->abort_flag = 0;
@@ -133,70 +159,80 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
 
-  if (warp == 0) {
-    // ---------------- TMA producer (one lane) ----------------
+  if (warp == 0 || warp == 2) {
+    // ---------------- TMA producers: X (warp 0), weights (warp 2) ----------------
     if (lane == 0) {
+      const bool xp = warp == 0;
+      const int depth = xp ? XS : WS;
       int issued = 0;
       for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-        if (!mbar_wait_bounded(&bar->empty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
+        const int s = kb % depth;
+        const uint32_t ph = (uint32_t)(kb / depth) & 1u;
+        uint64_t* emp = xp ? &bar->xempty[s] : &bar->wempty[s];
+        if (!mbar_wait_bounded(emp, ph ^ 1u, abort_flag, kWaitLimitNs)) {
           record_timeout(err, bar);
           break;
         }
-        mbar_arrive_expect_tx(&bar->xfull[s],
-                              X_STAGE_BYTES + QW_STAGE_BYTES + scale_rows * S_ROW_BYTES);
-        tma_load_2d(xs + s * X_STAGE_BYTES, &x_map, kb * BK, t0, &bar->xfull[s]);
-        tma_load_2d(smem + QW_OFF + s * QW_STAGE_BYTES, &qw_map, n0, kb * (BK / 8),
-                    &bar->xfull[s]);
-        tma_load_2d(smem + S_OFF + s * S_STAGE_MAX_ROWS * S_ROW_BYTES, &s_map, n0,
-                    (int)(((int64_t)kb * BK) >> group_shift), &bar->xfull[s]);
+        if (xp) {
+          mbar_arrive_expect_tx(&bar->xfull[s], X_STAGE_BYTES);
+          tma_load_2d(xs + s * X_STAGE_BYTES, &x_map, kb * BK, t0, &bar->xfull[s]);
+        } else {
+          uint8_t* wst = smem + W_OFF + s * W_STAGE_BYTES;
+          mbar_arrive_expect_tx(&bar->wfull[s], QW_STAGE_BYTES + scale_rows * S_ROW_BYTES);
+          tma_load_2d(wst, &qw_map, n0, kb * (BK / 8), &bar->wfull[s]);
+          tma_load_2d(wst + QW_STAGE_BYTES, &s_map, n0, (int)(((int64_t)kb * BK) >> group_shift),
+                      &bar->wfull[s]);
+        }
         ++issued;
       }
       if (*abort_flag) {
         // drain: wait for the last load issued into each slot
         int never = 0;
-        for (int j = issued - 1; j >= 0 && j >= issued - STAGES; --j)
-          mbar_wait_bounded(&bar->xfull[j % STAGES], (uint32_t)(j / STAGES) & 1u, &never,
-                            kDrainLimitNs);
+        for (int j = issued - 1; j >= 0 && j >= issued - depth; --j)
+          mbar_wait_bounded(xp ? &bar->xfull[j % depth] : &bar->wfull[j % depth],
+                            (uint32_t)(j / depth) & 1u, &never, kDrainLimitNs);
       }
     }
     __syncwarp();  // the whole warp reaches the CTA barrier below together
   } else if (warp == 1) {
-    // ---------------- MMA issuer (one lane) ----------------
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f16_f32(BW, BT);
-      bool aborted = false;
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-        if (!mbar_wait_bounded(&bar->xfull[s], ph, abort_flag, kWaitLimitNs) ||
-            !mbar_wait_bounded(&bar->afull[s], ph, abort_flag, kWaitLimitNs)) {
-          record_timeout(err, bar);
-          aborted = true;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t xa = smem_u32(xs + s * X_STAGE_BYTES);
+    // ---------------- MMA issuer ----------------
+    // The whole warp runs the loop converged (so the descriptors stay
+    // warp-uniform) and one elected lane issues the MMAs and commits.
+    const uint32_t idesc = idesc_f16_f32(BW, BT);
+    bool ok = true;
+    for (int kb = 0; kb < KB && ok; ++kb) {
+      const int s = kb % XS, a = kb % AS;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_bounded(&bar->xfull[s], (uint32_t)(kb / XS) & 1u, abort_flag,
+                                        kWaitLimitNs) &&
+                          mbar_wait_bounded(&bar->afull[a], (uint32_t)(kb / AS) & 1u, abort_flag,
+                                            kWaitLimitNs));
+      if (!ok) break;
+      tc_fence_after();
+      const uint64_t b_desc0 = smem_desc_sw128(smem_u32(xs + s * X_STAGE_BYTES));
+      const uint32_t a_base = tmem + A_COL + a * A_STAGE_COLS;
+      if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint32_t a_tmem = tmem + A_COL + s * A_STAGE_COLS + kk * 8;
-          const uint64_t b_desc = smem_desc_sw128(xa + kk * 32);
-          mma_f16_ts(tmem + D_COL, a_tmem, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
-        }
-        mma_commit(&bar->empty[s]);
+        for (int kk = 0; kk < BK / 16; ++kk)
+          mma_f16_ts(tmem + D_COL, a_base + kk * 8, b_desc0 + (uint64_t)((kk * 32) >> 4), idesc,
+                     (kb | kk) != 0 ? 1u : 0u);
+        mma_commit(&bar->xempty[s]);
+        mma_commit(&bar->aempty[a]);
       }
-      mma_commit(&bar->dfull);
-      if (aborted) {
-        int never = 0;
-        mbar_wait_bounded(&bar->dfull, 0, &never, kDrainLimitNs);
-      }
+      __syncwarp();
+    }
+    if (!ok && lane == 0) record_timeout(err, bar);
+    if (elect_one()) mma_commit(&bar->dfull);
+    __syncwarp();
+    if (!ok) {
+      int never = 0;
+      mbar_wait_bounded(&bar->dfull, 0, &never, kDrainLimitNs);
     }
     __syncwarp();  // the whole warp reaches the CTA barrier below together
   } else {
     // ---------------- dequantisation, then epilogue ----------------
-    const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
-    const int half = (warp - 2) >> 2;      // packed rows 4*half .. +3 of a stage
+    const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
+    const int half = (warp - DQ_WARP0) >> 2;      // packed rows 4*half .. +3 of a stage
     const int n = n0 + 32 * quarter + lane;
     const bool col_ok = n < N;
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
@@ -204,22 +240,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     // this thread's column in the stage's qweight and scale tiles; packed
     // rows 4*half .. 4*half+3 of every stage
     const int col = 32 * quarter + lane;
-    const uint8_t* qw_tile = smem + QW_OFF + (4 * half) * (BW * 4) + col * 4;
-    const uint8_t* s_tile = smem + S_OFF + col * 2;
+    const uint8_t* qw_tile = smem + W_OFF + (4 * half) * (BW * 4) + col * 4;
+    const uint8_t* s_tile = smem + W_OFF + QW_STAGE_BYTES + col * 2;
 
     bool ok = true;
     for (int kb = 0; kb < KB; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-      // qweight and scale tiles of the stage have landed (with X)
-      ok = mbar_wait_bounded<true>(&bar->xfull[s], ph, abort_flag, kWaitLimitNs);
-      ok = __all_sync(0xffffffffu, ok);
+      const int j = kb % WS;
+      const uint32_t ph = (uint32_t)(kb / WS) & 1u;
+      // qweight and scale tiles of the stage have landed
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_bounded<true>(&bar->wfull[j], ph, abort_flag, kWaitLimitNs));
       if (!ok) {
         if (lane == 0) record_timeout(err, bar);
         break;
       }
-      const uint8_t* qw = qw_tile + s * QW_STAGE_BYTES;
-      const uint8_t* sc = s_tile + s * S_STAGE_MAX_ROWS * S_ROW_BYTES;
+      const uint8_t* qw = qw_tile + j * W_STAGE_BYTES;
+      const uint8_t* sc = s_tile + j * W_STAGE_BYTES;
       uint32_t cells[16];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
@@ -231,21 +267,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t nat[4];
         dequant_word_natural(w, half2_broadcast(sv), nat);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) cells[4 * r + j] = nat[j];
+        for (int q = 0; q < 4; ++q) cells[4 * r + q] = nat[q];
       }
-      // the A columns of this stage are free once the MMAs of its previous
-      // use have completed
-      ok = mbar_wait_bounded<true>(&bar->empty[s], ph ^ 1u, abort_flag, kWaitLimitNs);
-      ok = __all_sync(0xffffffffu, ok);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->wempty[j]);  // weight tiles of the stage read
+      // the A slot is free once the MMAs of its previous use have completed
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded<true>(&bar->aempty[j], ph ^ 1u, abort_flag,
+                                                           kWaitLimitNs));
       if (!ok) {
         if (lane == 0) record_timeout(err, bar);
         break;
       }
       tc_fence_after();
-      tmem_st_32x32b_x16(tmem + lane_addr + A_COL + s * A_STAGE_COLS + 16 * half, cells);
+      tmem_st_32x32b_x16(tmem + lane_addr + A_COL + j * A_STAGE_COLS + 16 * half, cells);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar->afull[s]);
+      mbar_arrive(&bar->afull[j]);
     }
 
     if (ok) {
@@ -263,10 +300,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_wait_ld();
         if (col_ok) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int t = t0 + tok0 + j;
+          for (int q = 0; q < 32; ++q) {
+            const int t = t0 + tok0 + q;
             if (t < M)
-              y[(int64_t)t * N + n] = __half_as_ushort(__float2half_rn(__uint_as_float(r[j])));
+              y[(int64_t)t * N + n] = __half_as_ushort(__float2half_rn(__uint_as_float(r[q])));
           }
         }
       }
