@@ -47,7 +47,8 @@ constexpr int BK = 64;   // k per pipeline stage (four k16 MMAs)
 constexpr int XS = 4;        // X ring stages (BT x 64 k each)
 constexpr int WS = 8;        // weight-tile ring stages (qweight + scales of 64 k)
 constexpr int AS = 8;        // A slots in TMEM (64 k each)
-constexpr int DQ_WARPS = 8;  // dequantisation + epilogue warps
+constexpr int DQ_GROUPS = 4;                // dequantisation groups, taking stages kb = g mod 4
+constexpr int DQ_WARPS = 4 * DQ_GROUPS;     // one warp per TMEM lane quarter in each group
 constexpr int DQ_WARP0 = 3;  // warps 0, 1, 2: X producer, MMA issuer, weight producer
 constexpr int THREADS = (DQ_WARP0 + DQ_WARPS) * 32;
 constexpr int QW_STAGE_BYTES = BW * (BK / 8) * 4;  // 128 columns x 8 packed rows: 4 KB
@@ -107,6 +108,9 @@ __device__ __forceinline__ bool elect_one() {
 // The X tiles and the weight tiles travel in separate rings: the weight ring
 // and the A slots are twice as deep as the X ring, so the dequantisation runs
 // up to eight stages ahead of the MMAs while the large X tiles only need four.
+// A stage gives each dequantisation thread little work, so four groups of
+// four warps take stages in turn (kb = g mod 4) and keep four stages in
+// flight.
 template <int BT>
 __global__ void __launch_bounds__(THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap x_map,
@@ -137,8 +141,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int j = 0; j < WS; ++j) {
       mbar_init(&bar->wfull[j], 1);
-      mbar_init(&bar->wempty[j], DQ_WARPS);
-      mbar_init(&bar->afull[j], DQ_WARPS * 32);
+      mbar_init(&bar->wempty[j], 4);        // the four warps of the stage's group
+      mbar_init(&bar->afull[j], 4 * 32);    // every thread of that group
       mbar_init(&bar->aempty[j], 1);
     }
     mbar_init(&bar->dfull, 1);
@@ -232,19 +236,19 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // ---------------- dequantisation, then epilogue ----------------
     const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
-    const int half = (warp - DQ_WARP0) >> 2;      // packed rows 4*half .. +3 of a stage
+    const int grp = (warp - DQ_WARP0) >> 2;       // stages kb = grp mod DQ_GROUPS
     const int n = n0 + 32 * quarter + lane;
     const bool col_ok = n < N;
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
 
-    // this thread's column in the stage's qweight and scale tiles; packed
-    // rows 4*half .. 4*half+3 of every stage
+    // this thread's column in the stage's qweight and scale tiles: all eight
+    // packed rows of its group's stages
     const int col = 32 * quarter + lane;
-    const uint8_t* qw_tile = smem + W_OFF + (4 * half) * (BW * 4) + col * 4;
+    const uint8_t* qw_tile = smem + W_OFF + col * 4;
     const uint8_t* s_tile = smem + W_OFF + QW_STAGE_BYTES + col * 2;
 
     bool ok = true;
-    for (int kb = 0; kb < KB; ++kb) {
+    for (int kb = grp; kb < KB; kb += DQ_GROUPS) {
       const int j = kb % WS;
       const uint32_t ph = (uint32_t)(kb / WS) & 1u;
       // qweight and scale tiles of the stage have landed
@@ -256,12 +260,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       const uint8_t* qw = qw_tile + j * W_STAGE_BYTES;
       const uint8_t* sc = s_tile + j * W_STAGE_BYTES;
-      uint32_t cells[16];
+      uint32_t cells[32];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        // scale row of packed row 4*half + r inside the stage (0 unless the
-        // group is smaller than the 64-k stage)
-        const int gl = ((4 * half + r) * 8) >> group_shift;
+      for (int r = 0; r < BK / 8; ++r) {
+        // scale row of packed row r inside the stage (0 unless the group is
+        // smaller than the 64-k stage)
+        const int gl = (r * 8) >> group_shift;
         const uint16_t sv = *reinterpret_cast<const uint16_t*>(sc + gl * S_ROW_BYTES);
         const uint32_t w = *reinterpret_cast<const uint32_t*>(qw + r * (BW * 4));
         uint32_t nat[4];
@@ -279,7 +283,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       tc_fence_after();
-      tmem_st_32x32b_x16(tmem + lane_addr + A_COL + j * A_STAGE_COLS + 16 * half, cells);
+      tmem_st_32x32b_x32(tmem + lane_addr + A_COL + j * A_STAGE_COLS, cells);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar->afull[j]);
@@ -291,16 +295,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!ok && lane == 0) record_timeout(err, bar);
     }
     if (ok) {
+      // group g writes tokens [g*BT/4, (g+1)*BT/4) of the tile, 16 at a time
       tc_fence_after();
+      constexpr int TPG = BT / DQ_GROUPS;
 #pragma unroll 1
-      for (int chunk = 0; chunk < (BT / 2) / 32; ++chunk) {
-        const int tok0 = (BT / 2) * half + 32 * chunk;
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + lane_addr + D_COL + tok0, r);
+      for (int chunk = 0; chunk < TPG / 16; ++chunk) {
+        const int tok0 = TPG * grp + 16 * chunk;
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tmem + lane_addr + D_COL + tok0, r);
         tmem_wait_ld();
         if (col_ok) {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
+          for (int q = 0; q < 16; ++q) {
             const int t = t0 + tok0 + q;
             if (t < M)
               y[(int64_t)t * N + n] = __half_as_ushort(__float2half_rn(__uint_as_float(r[q])));
