@@ -143,6 +143,16 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
                : "memory");
 }
 
+// Arrive on an mbarrier of any CTA of the cluster (shared::cluster address).
+// CTA-scope release: it hands over TMEM contents, whose order is set by the
+// tcgen05 wait and fences around the arrive; a cluster-scope release would
+// also wait for this thread's memory writes to reach cluster scope, which
+// costs thousands of cycles under load and orders nothing the reader needs.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
                    smem_u32(bar)),

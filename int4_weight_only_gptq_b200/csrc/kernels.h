@@ -49,5 +49,11 @@ cudaError_t launch_decode_grouped(const uint16_t* x, const int32_t* const* qweig
 cudaError_t launch_prefill(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                            uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
                            cudaStream_t stream, const DeviceInfo& dev);
+// The same on CTA pairs (tcgen05 cta_group::2; 256 weight columns x 128 or
+// 256 tokens per pair, half of the X tile loaded by each CTA).
+cudaError_t launch_prefill_pair(const uint16_t* x, const int32_t* qweight,
+                                const uint16_t* scales, uint16_t* y, int64_t M, int64_t K,
+                                int64_t N, int group_shift, cudaStream_t stream,
+                                const DeviceInfo& dev);
 
 }  // namespace gptq

@@ -356,8 +356,8 @@ cudaError_t launch_t(const uint16_t* x, const int32_t* qweight, const uint16_t* 
 
 }  // namespace
 
-// The token tile follows M (64, 128 or 256 tokens per CTA), so that small M
-// does not pay for MMAs over empty token columns.
+// The token tile follows M (64 or 128 tokens per CTA, then 256 per CTA pair),
+// so that small M does not pay for MMAs over empty token columns.
 cudaError_t launch_prefill(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                            uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
                            cudaStream_t stream, const DeviceInfo& dev) {
@@ -370,8 +370,8 @@ cudaError_t launch_prefill(const uint16_t* x, const int32_t* qweight, const uint
   if (M <= 128)
     return launch_t<128>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups, stream,
                          dev);
-  return launch_t<256>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups, stream,
-                       dev);
+  // above 128 tokens the CTA-pair kernel takes over: half the X traffic per SM
+  return launch_prefill_pair(x, qweight, scales, y, M, K, N, group_shift, stream, dev);
 }
 
 }  // namespace gptq

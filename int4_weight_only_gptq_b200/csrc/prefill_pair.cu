@@ -1,0 +1,396 @@
+// Prefill kernel on CTA pairs: Y[M, N] = X[M, K] . dequant(qweight, scales)
+// with tcgen05.mma.cta_group::2, for token tiles of 128 or 256.
+//
+// Operation: GPTQ-Pro README, "Runtime contract" and "Ampere kernel
+// architecture" (tensor-core prefill with FP32 accumulation that reads the
+// native int32 qweight; predicated tails; FP16 output).  The Ampere design is
+// prior art only.
+//
+// Same transposed product as the single-CTA prefill kernel (Y^T = W^T . X^T:
+// weights are the MMA's A operand from TMEM, tokens its N dimension), but the
+// two CTAs of a cluster share one 256-column x BT-token tile:
+//
+// * each CTA dequantises its own 128 weight columns into its own TMEM (A rows
+//   0..127 live in the even CTA, rows 128..255 in the odd one);
+// * each CTA loads only HALF of the X tile (BT/2 token rows x 64 k per
+//   stage); the pair MMA reads B rows 0..BT/2-1 from the even CTA and the
+//   rest from the odd CTA, so every X byte crosses from L2 once per pair
+//   instead of once per CTA;
+// * one thread of the even CTA issues the M = 256 MMAs; their completion is
+//   signalled to the barriers of both CTAs at once (tcgen05.commit with a
+//   CTA mask).  Both CTAs' X loads count their bytes on the even CTA's
+//   barrier, and both CTAs' dequantisation warps arrive on the even CTA's
+//   A-slot barrier.
+//
+// Halving the X traffic per SM matters because moving X from L2 into shared
+// memory is where most of the power of this kernel goes: with half of it the
+// SMs hold a higher clock under the board's power limit.
+//
+// Every wait is bounded in time; on expiry the CTA records GPTQ_ERR_TIMEOUT
+// in the device error word and winds down.  Both CTAs always reach the final
+// cluster barrier, so neither leaves while the other may still signal it.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc05.cuh"
+#include "tmap.h"
+
+namespace gptq {
+
+namespace {
+
+constexpr int BW = 128;   // weight columns per CTA (TMEM lanes); 256 per pair (MMA M)
+constexpr int BK = 64;    // k per pipeline stage (four k16 MMAs)
+constexpr int XS = 8;     // X ring stages (half tile per CTA)
+constexpr int WS = 8;     // weight-tile ring stages (qweight + scales of 64 k)
+constexpr int AS = 8;     // A slots in TMEM (64 k each)
+constexpr int DQ_GROUPS = 4;             // dequantisation groups, taking stages kb = g mod 4
+constexpr int DQ_WARPS = 4 * DQ_GROUPS;  // one warp per TMEM lane quarter in each group
+constexpr int DQ_WARP0 = 3;  // warps 0, 1, 2: X producer, MMA issuer, weight producer
+constexpr int THREADS = (DQ_WARP0 + DQ_WARPS) * 32;
+constexpr int QW_STAGE_BYTES = BW * (BK / 8) * 4;  // 128 columns x 8 packed rows: 4 KB
+constexpr int S_ROW_BYTES = BW * 2;                // one scale row of the tile: 256 B
+constexpr int S_STAGE_MAX_ROWS = BK / 16;          // group 16: four rows per stage
+constexpr int W_STAGE_BYTES = QW_STAGE_BYTES + S_STAGE_MAX_ROWS * S_ROW_BYTES;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t D_COL = 0;              // accumulator: columns [0, BT)
+constexpr uint32_t A_COL = 256;            // A slots: [256, 256 + 8 * 32)
+constexpr uint32_t A_STAGE_COLS = BK / 2;  // two FP16 per 32-bit column
+constexpr uint16_t kPairMask = 0x3;        // both CTAs of the cluster
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+constexpr uint64_t kDrainLimitNs = 200000000ull;
+static_assert(A_COL + AS * A_STAGE_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(AS == WS, "a weight stage and its A slot share an index");
+
+// Shared-memory layout for a pair token tile of BT (BT/2 X rows per CTA).
+template <int BT>
+struct PairLayout {
+  static constexpr int HT = BT / 2;
+  static constexpr int X_STAGE_BYTES = HT * BK * 2;
+  static constexpr int W_OFF = XS * X_STAGE_BYTES;
+  static constexpr int BAR_OFF = W_OFF + WS * W_STAGE_BYTES;
+  static constexpr size_t kSmemBytes = 1024 + (size_t)BAR_OFF + 512;
+  static_assert(X_STAGE_BYTES % 1024 == 0, "128-byte swizzle atoms stay aligned");
+};
+
+// Both CTAs hold the full set; xfull and afull are only used in the even CTA.
+struct PairBarriers {
+  uint64_t xfull[XS];   // both halves of the X tile landed (even CTA)
+  uint64_t xempty[XS];  // pair MMAs reading the X stage done
+  uint64_t wfull[WS];   // this CTA's qweight and scale tiles landed
+  uint64_t wempty[WS];  // weight tiles read by this CTA's group warps
+  uint64_t afull[AS];   // A slot written by the group warps of both CTAs (even CTA)
+  uint64_t aempty[AS];  // pair MMAs reading the A slot done
+  uint64_t dfull;       // all MMAs of the tile done
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(PairBarriers) <= 512, "barrier area");
+
+__device__ __forceinline__ void record_timeout(int* err, PairBarriers* b) {
+  atomicExch(err, kDeviceErrTimeout);
+  *reinterpret_cast<volatile int*>(&b->abort_flag) = 1;
+}
+
+// One lane of a converged warp (the lowest active one) returns true.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(p));
+  return p != 0;
+}
+
+// scale_rows: scale rows one 64-k stage touches (1, or 64/group for groups
+// below 64); stages start on 64-k boundaries, so they align with groups.
+template <int BT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    prefill_pair_kernel(const __grid_constant__ CUtensorMap x_map,
+                        const __grid_constant__ CUtensorMap qw_map,
+                        const __grid_constant__ CUtensorMap s_map, uint16_t* __restrict__ y,
+                        int M, int K, int N, int group_shift, int scale_rows, int* err) {
+  static_assert(BT == 128 || BT == 256, "pair token tile");
+  using L = PairLayout<BT>;
+  constexpr int HT = L::HT;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned base; the same offset in both CTAs, so that one MMA
+  // descriptor and one barrier offset name the matching buffers of the pair
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* xs = smem;
+  PairBarriers* bar = reinterpret_cast<PairBarriers*>(smem + L::BAR_OFF);
+  volatile int* abort_flag = &bar->abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: even CTA (issues the MMAs), 1: odd CTA
+  const bool even = rank == 0;
+  const int n0 = blockIdx.x * BW;
+  const int t0 = blockIdx.y * BT;
+  const int KB = (K + BK - 1) / BK;
+  // Does the odd CTA's half of the token tile hold any row below M?  If not,
+  // it loads nothing (no copy box lies wholly outside X) and the even CTA
+  // expects only its own bytes; the MMA then reads stale shared memory for
+  // token columns that are never stored.
+  const bool odd_rows = t0 + HT < M;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < XS; ++s) {
+      mbar_init(&bar->xfull[s], 1);   // the even CTA's expect_tx; bytes from both CTAs
+      mbar_init(&bar->xempty[s], 1);  // one pair commit
+    }
+    for (int j = 0; j < WS; ++j) {
+      mbar_init(&bar->wfull[j], 1);
+      mbar_init(&bar->wempty[j], 4);      // the four warps of the stage's group
+      mbar_init(&bar->afull[j], 2 * 4);   // those warps in both CTAs
+      mbar_init(&bar->aempty[j], 1);      // one pair commit
+    }
+    mbar_init(&bar->dfull, 1);
+    bar->abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&x_map);
+    prefetch_tensormap(&qw_map);
+    prefetch_tensormap(&s_map);
+  }
+  __syncwarp();
+  if (warp == 1) {
+    tmem_alloc_pair(&bar->tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  // both CTAs' barriers are initialised and TMEM is allocated before any
+  // thread signals the other CTA
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+  // the even CTA's barriers that both CTAs signal
+  const uint32_t xfull_even = map_to_rank(smem_u32(&bar->xfull[0]), 0);
+  const uint32_t afull_even = map_to_rank(smem_u32(&bar->afull[0]), 0);
+
+  if (warp == 0 || warp == 2) {
+    // ---------------- TMA producers: X half (warp 0), weights (warp 2) ----------------
+    if (lane == 0) {
+      const bool xp = warp == 0;
+      const int depth = xp ? XS : WS;
+      int issued = 0;
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % depth;
+        const uint32_t ph = (uint32_t)(kb / depth) & 1u;
+        uint64_t* emp = xp ? &bar->xempty[s] : &bar->wempty[s];
+        if (!mbar_wait_bounded(emp, ph ^ 1u, abort_flag, kWaitLimitNs)) {
+          record_timeout(err, bar);
+          break;
+        }
+        if (xp) {
+          if (even) mbar_arrive_expect_tx(&bar->xfull[s], (odd_rows ? 2 : 1) * L::X_STAGE_BYTES);
+          if (even || odd_rows)
+            tma_load_2d_pair(xs + s * L::X_STAGE_BYTES, &x_map, kb * BK, t0 + (int)rank * HT,
+                             xfull_even + 8u * (uint32_t)s);
+        } else if (n0 < N) {
+          uint8_t* wst = smem + L::W_OFF + s * W_STAGE_BYTES;
+          mbar_arrive_expect_tx(&bar->wfull[s], QW_STAGE_BYTES + scale_rows * S_ROW_BYTES);
+          tma_load_2d(wst, &qw_map, n0, kb * (BK / 8), &bar->wfull[s]);
+          tma_load_2d(wst + QW_STAGE_BYTES, &s_map, n0, (int)(((int64_t)kb * BK) >> group_shift),
+                      &bar->wfull[s]);
+        } else {
+          mbar_arrive(&bar->wfull[s]);  // padding CTA: no columns, nothing to load
+        }
+        ++issued;
+      }
+      if (*abort_flag && (!xp || even)) {
+        // drain: wait for the last loads issued into each slot (the odd
+        // CTA's X loads complete on the even CTA's barriers, which the even
+        // CTA drains)
+        int never = 0;
+        for (int j = issued - 1; j >= 0 && j >= issued - depth; --j)
+          mbar_wait_bounded(xp ? &bar->xfull[j % depth] : &bar->wfull[j % depth],
+                            (uint32_t)(j / depth) & 1u, &never, kDrainLimitNs);
+      }
+    }
+    __syncwarp();  // the whole warp reaches the cluster barrier below together
+  } else if (warp == 1) {
+    // ---------------- pair MMA issuer (even CTA) ----------------
+    if (even) {
+      const uint32_t idesc = idesc_f16_f32(2 * BW, BT);
+      bool ok = true;
+      for (int kb = 0; kb < KB && ok; ++kb) {
+        const int s = kb % XS, a = kb % AS;
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait_bounded(&bar->xfull[s], (uint32_t)(kb / XS) & 1u, abort_flag,
+                                          kWaitLimitNs) &&
+                            mbar_wait_bounded(&bar->afull[a], (uint32_t)(kb / AS) & 1u,
+                                              abort_flag, kWaitLimitNs));
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t b_desc0 = smem_desc_sw128(smem_u32(xs + s * L::X_STAGE_BYTES));
+        const uint32_t a_base = tmem + A_COL + a * A_STAGE_COLS;
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_f16_ts_pair(tmem + D_COL, a_base + kk * 8,
+                            b_desc0 + (uint64_t)((kk * 32) >> 4), idesc,
+                            (kb | kk) != 0 ? 1u : 0u);
+          mma_commit_pair(&bar->xempty[s], kPairMask);
+          mma_commit_pair(&bar->aempty[a], kPairMask);
+        }
+        __syncwarp();
+      }
+      if (!ok && lane == 0) record_timeout(err, bar);
+      if (elect_one()) mma_commit_pair(&bar->dfull, kPairMask);
+      __syncwarp();
+      if (!ok) {
+        int never = 0;
+        mbar_wait_bounded(&bar->dfull, 0, &never, kDrainLimitNs);
+      }
+    }
+    __syncwarp();  // the whole warp reaches the cluster barrier below together
+  } else {
+    // ---------------- dequantisation, then epilogue ----------------
+    const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+    const int grp = (warp - DQ_WARP0) >> 2;  // stages kb = grp mod DQ_GROUPS
+    const int n = n0 + 32 * quarter + lane;
+    const bool col_ok = n < N;
+    const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
+
+    // this thread's column in the stage's qweight and scale tiles
+    const int col = 32 * quarter + lane;
+    const uint8_t* qw_tile = smem + L::W_OFF + col * 4;
+    const uint8_t* s_tile = smem + L::W_OFF + QW_STAGE_BYTES + col * 2;
+
+    bool ok = true;
+    for (int kb = grp; kb < KB; kb += DQ_GROUPS) {
+      const int j = kb % WS;
+      const uint32_t ph = (uint32_t)(kb / WS) & 1u;
+      // qweight and scale tiles of the stage have landed
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_bounded<true>(&bar->wfull[j], ph, abort_flag, kWaitLimitNs));
+      if (!ok) {
+        if (lane == 0) record_timeout(err, bar);
+        break;
+      }
+      const uint8_t* qw = qw_tile + j * W_STAGE_BYTES;
+      const uint8_t* sc = s_tile + j * W_STAGE_BYTES;
+      uint32_t cells[32];
+#pragma unroll
+      for (int r = 0; r < BK / 8; ++r) {
+        // scale row of packed row r inside the stage (0 unless the group is
+        // smaller than the 64-k stage)
+        const int gl = group_shift >= 6 ? 0 : (r * 8) >> group_shift;
+        const uint16_t sv = *reinterpret_cast<const uint16_t*>(sc + gl * S_ROW_BYTES);
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(qw + r * (BW * 4));
+        uint32_t nat[4];
+        dequant_word_natural(w, half2_broadcast(sv), nat);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) cells[4 * r + q] = nat[q];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->wempty[j]);  // weight tiles of the stage read
+      // the A slot is free once the pair MMAs of its previous use completed
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded<true>(&bar->aempty[j], ph ^ 1u, abort_flag,
+                                                           kWaitLimitNs));
+      if (!ok) {
+        if (lane == 0) record_timeout(err, bar);
+        break;
+      }
+      tc_fence_after();
+      tmem_st_32x32b_x32(tmem + lane_addr + A_COL + j * A_STAGE_COLS, cells);
+      tmem_wait_st();  // the whole warp's cells are in TMEM
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(afull_even + 8u * (uint32_t)j);
+    }
+
+    if (ok) {
+      ok = mbar_wait_bounded<true>(&bar->dfull, 0, abort_flag, kWaitLimitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok && lane == 0) record_timeout(err, bar);
+    }
+    if (ok) {
+      // group g writes tokens [g*BT/4, (g+1)*BT/4) of the tile, 16 at a time
+      tc_fence_after();
+      constexpr int TPG = BT / DQ_GROUPS;
+#pragma unroll 1
+      for (int chunk = 0; chunk < TPG / 16; ++chunk) {
+        const int tok0 = TPG * grp + 16 * chunk;
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tmem + lane_addr + D_COL + tok0, r);
+        tmem_wait_ld();
+        if (col_ok) {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const int t = t0 + tok0 + q;
+            if (t < M)
+              y[(int64_t)t * N + n] = __half_as_ushort(__float2half_rn(__uint_as_float(r[q])));
+          }
+        }
+      }
+    }
+  }
+
+  // neither CTA leaves (or frees TMEM) while the pair's MMAs, loads or
+  // signals may still touch it
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+template <int BT>
+cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                          uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
+                          int scale_rows, int64_t n_groups, cudaStream_t stream,
+                          const DeviceInfo& dev) {
+  using L = PairLayout<BT>;
+  CUtensorMap x_map, qw_map, s_map;
+  if (!tensor_map_2d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M,
+                     (uint64_t)K * 2, BK, L::HT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tensor_map_2d(&qw_map, qweight, CU_TENSOR_MAP_DATA_TYPE_INT32, (uint64_t)N,
+                     (uint64_t)(K / 8), (uint64_t)N * 4, BW, BK / 8, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !tensor_map_2d(&s_map, scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, (uint64_t)N,
+                     (uint64_t)n_groups, (uint64_t)N * 2, BW, (uint32_t)scale_rows,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  constexpr size_t smem = L::kSmemBytes;
+  static std::once_flag attr_once[64];
+  static cudaError_t attr_err[64];
+  const int d = dev.device & 63;
+  std::call_once(attr_once[d], [&] {
+    attr_err[d] = cudaFuncSetAttribute(prefill_pair_kernel<BT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  });
+  if (attr_err[d] != cudaSuccess) return attr_err[d];
+  // an even number of 128-column CTAs: with an odd count the last pair's odd
+  // CTA has no columns, loads no weights and stores nothing
+  const unsigned ctas_n = (unsigned)(((N + BW - 1) / BW + 1) & ~int64_t(1));
+  const dim3 grid(ctas_n, (unsigned)((M + BT - 1) / BT), 1);
+  prefill_pair_kernel<BT><<<grid, THREADS, smem, stream>>>(x_map, qw_map, s_map, y, (int)M,
+                                                           (int)K, (int)N, group_shift,
+                                                           scale_rows, dev.error_word);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_pair(const uint16_t* x, const int32_t* qweight,
+                                const uint16_t* scales, uint16_t* y, int64_t M, int64_t K,
+                                int64_t N, int group_shift, cudaStream_t stream,
+                                const DeviceInfo& dev) {
+  const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
+                               ? 1 : (K + (int64_t(1) << group_shift) - 1) >> group_shift;
+  const int scale_rows = group_shift >= 6 ? 1 : (BK >> group_shift);
+  if (M <= 128)
+    return launch_pair_t<128>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups,
+                              stream, dev);
+  return launch_pair_t<256>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups,
+                            stream, dev);
+}
+
+}  // namespace gptq

@@ -176,6 +176,55 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// ---- CTA pair (cta_group::2) ------------------------------------------------
+//
+// Every tcgen05 instruction of a kernel uses one CTA-group size, so a kernel
+// that issues pair MMAs allocates, relinquishes and frees TMEM with these
+// forms too: warps with the same index in both CTAs of the pair execute them,
+// with the same shared-memory holder offset, and get the same TMEM base.
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* holder_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(holder_smem)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// D (+)= A . B^T over the pair, issued by one thread of the even CTA.  M =
+// 256: rows 0..127 of A and D are the TMEM lanes of the even CTA, rows
+// 128..255 those of the odd CTA (same TMEM addresses).  B (N rows) is split
+// along N: rows 0..N/2-1 in the even CTA's shared memory, the rest in the odd
+// CTA's, at the same descriptor address.
+__device__ __forceinline__ void mma_f16_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Once all pair MMAs this thread issued before it have completed, arrive once
+// on the mbarrier at this shared-memory offset in every CTA of `cta_mask`
+// (a signal sent by the tensor core, not a memory load).
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+
 // ---- TMA -------------------------------------------------------------------
 
 __device__ __forceinline__ void tma_load_2d(void* dst_smem, const CUtensorMap* map, int32_t c0,
@@ -193,6 +242,18 @@ __device__ __forceinline__ void tma_load_3d(void* dst_smem, const CUtensorMap* m
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst_smem)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// 2-D tile load into this CTA's shared memory whose bytes are counted on an
+// mbarrier of either CTA of the pair (`bar_cluster`: a shared::cluster
+// address, e.g. from mapa).  No multicast: one destination CTA.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst_smem, const CUtensorMap* map,
+                                                 int32_t c0, int32_t c1, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst_smem)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
       : "memory");
 }
 

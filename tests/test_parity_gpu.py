@@ -144,7 +144,12 @@ def test_edge_shapes_small_m(M, K, N, G, kernel):
                                      (257, 1040, 128, -1), (513, 160, 392, 64),
                                      # token tiles of 64 (M <= 64) and 128 (M <= 128)
                                      (33, 96, 72, 32), (64, 160, 136, 64), (100, 528, 264, 128),
-                                     (128, 1040, 128, -1), (65, 2048, 200, 16)])
+                                     (128, 1040, 128, -1), (65, 2048, 200, 16),
+                                     # CTA-pair tiles (M > 128): the odd CTA's half partly
+                                     # filled, empty, or with one row; padding CTAs (odd
+                                     # number of 128-column tiles); a single k stage
+                                     (200, 2048, 392, 128), (256, 528, 200, 16),
+                                     (385, 96, 136, 32), (160, 64, 8, -1), (255, 1024, 24, 64)])
 def test_edge_shapes_prefill(M, K, N, G):
     p = W.make_problem(M, K, N, G, seed=M + K + N)
     y = run(p)
@@ -197,6 +202,33 @@ def test_one_hot_x_reproduces_dequantised_rows_bitwise(kernel):
     w = oracle.dequant(p.qweight, p.scales, 32)
     for m, k in enumerate(ks):
         assert np.array_equal(y[m].view(np.uint16), w[k].view(np.uint16)), (m, k)
+
+
+def test_one_hot_x_pair_tile_bitwise():
+    """256 tokens = both halves of a CTA-pair tile (rows 0..127 loaded by
+    the even CTA, 128..255 by the odd one), 264 columns = two pairs, the
+    second with a padding CTA: each output row is one dequantised weight
+    row, bit for bit, so a token or column landing in the wrong place fails."""
+    p = W.make_problem(256, 1024, 264, 32, seed=5)
+    rng = np.random.default_rng(5)
+    ks = rng.integers(0, 1024, size=256)
+    p.x[:] = 0
+    p.x[np.arange(256), ks] = 1
+    y = run(p, B.KERNEL_PREFILL)
+    w = oracle.dequant(p.qweight, p.scales, 32)
+    for m in range(256):
+        assert np.array_equal(y[m].view(np.uint16), w[ks[m]].view(np.uint16)), (m, ks[m])
+
+
+@pytest.mark.parametrize("M", [129, 200, 256, 300])
+def test_integer_exact_inputs_pair_tile_bitwise(M):
+    rng = np.random.default_rng(M)
+    p = W.make_problem(M, 2048, 392, 64, seed=M)
+    p.x[:] = rng.integers(-4, 5, size=p.x.shape).astype(np.float16)
+    p.scales[:] = np.float16(2.0 ** -6)
+    y = run(p, B.KERNEL_PREFILL)
+    ref = oracle.round_to_half(oracle.gemm(p.x, p.qweight, p.scales, 64))
+    assert np.array_equal(y.view(np.uint16), ref.view(np.uint16))
 
 
 @pytest.mark.parametrize("kernel", [B.KERNEL_DECODE, B.KERNEL_PREFILL])
