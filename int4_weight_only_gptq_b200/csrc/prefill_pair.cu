@@ -45,37 +45,41 @@ namespace gptq {
 namespace {
 
 constexpr int BW = 128;   // weight columns per CTA (TMEM lanes); 256 per pair (MMA M)
-constexpr int BK = 64;    // k per pipeline stage (four k16 MMAs)
-constexpr int XS = 8;     // X ring stages (half tile per CTA)
-constexpr int WS = 8;     // weight-tile ring stages (qweight + scales of 64 k)
-constexpr int AS = 8;     // A slots in TMEM (64 k each)
-constexpr int DQ_GROUPS = 4;             // dequantisation groups, taking stages kb = g mod 4
+constexpr int BK = 128;   // k per pipeline stage (eight k16 MMAs)
+constexpr int XS = 4;     // X ring stages (half tile per CTA)
+constexpr int WS = 4;     // weight-tile ring stages (qweight + scales of 128 k)
+constexpr int AS = 4;     // A slots in TMEM (128 k each)
+constexpr int DQ_GROUPS = 4;             // dequantisation groups: group g takes stages kb = g mod 4
 constexpr int DQ_WARPS = 4 * DQ_GROUPS;  // one warp per TMEM lane quarter in each group
 constexpr int DQ_WARP0 = 3;  // warps 0, 1, 2: X producer, MMA issuer, weight producer
 constexpr int THREADS = (DQ_WARP0 + DQ_WARPS) * 32;
-constexpr int QW_STAGE_BYTES = BW * (BK / 8) * 4;  // 128 columns x 8 packed rows: 4 KB
+constexpr int QW_STAGE_BYTES = BW * (BK / 8) * 4;  // 128 columns x 16 packed rows: 8 KB
 constexpr int S_ROW_BYTES = BW * 2;                // one scale row of the tile: 256 B
-constexpr int S_STAGE_MAX_ROWS = BK / 16;          // group 16: four rows per stage
+constexpr int S_STAGE_MAX_ROWS = BK / 16;          // group 16: eight rows per stage
 constexpr int W_STAGE_BYTES = QW_STAGE_BYTES + S_STAGE_MAX_ROWS * S_ROW_BYTES;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t D_COL = 0;              // accumulator: columns [0, BT)
-constexpr uint32_t A_COL = 256;            // A slots: [256, 256 + 8 * 32)
+constexpr uint32_t A_COL = 256;            // A slots: [256, 256 + 4 * 64)
 constexpr uint32_t A_STAGE_COLS = BK / 2;  // two FP16 per 32-bit column
 constexpr uint16_t kPairMask = 0x3;        // both CTAs of the cluster
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 static_assert(A_COL + AS * A_STAGE_COLS <= TMEM_COLS, "TMEM budget");
-static_assert(AS == WS, "a weight stage and its A slot share an index");
+static_assert(AS == WS && XS == WS && WS == DQ_GROUPS,
+              "stage kb uses X, weight and A slot kb mod 4, dequantised by group kb mod 4");
 
 // Shared-memory layout for a pair token tile of BT (BT/2 X rows per CTA).
+// An X stage is two 64-k halves, each BT/2 rows of 128 bytes (128-byte
+// swizzle), the second right after the first.
 template <int BT>
 struct PairLayout {
   static constexpr int HT = BT / 2;
-  static constexpr int X_STAGE_BYTES = HT * BK * 2;
+  static constexpr int X_HALF_BYTES = HT * 64 * 2;
+  static constexpr int X_STAGE_BYTES = 2 * X_HALF_BYTES;
   static constexpr int W_OFF = XS * X_STAGE_BYTES;
   static constexpr int BAR_OFF = W_OFF + WS * W_STAGE_BYTES;
   static constexpr size_t kSmemBytes = 1024 + (size_t)BAR_OFF + 512;
-  static_assert(X_STAGE_BYTES % 1024 == 0, "128-byte swizzle atoms stay aligned");
+  static_assert(X_HALF_BYTES % 1024 == 0, "128-byte swizzle atoms stay aligned");
 };
 
 // Both CTAs hold the full set; xfull and afull are only used in the even CTA.
@@ -106,14 +110,17 @@ __device__ __forceinline__ bool elect_one() {
   return p != 0;
 }
 
-// scale_rows: scale rows one 64-k stage touches (1, or 64/group for groups
-// below 64); stages start on 64-k boundaries, so they align with groups.
+// scale_rows: scale rows one 128-k stage touches (1, or 128/group for groups
+// below 128); stages start on 128-k boundaries, so they align with groups.
+// x3d: X is read through a [K/64][M][64] view, one copy per stage (K a
+// multiple of 64); otherwise through [M][K], one copy per 64-k half.
 template <int BT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap x_map,
                         const __grid_constant__ CUtensorMap qw_map,
                         const __grid_constant__ CUtensorMap s_map, uint16_t* __restrict__ y,
-                        int M, int K, int N, int group_shift, int scale_rows, int* err) {
+                        int M, int K, int N, int group_shift, int scale_rows, int x3d,
+                        int* err) {
   static_assert(BT == 128 || BT == 256, "pair token tile");
   using L = PairLayout<BT>;
   constexpr int HT = L::HT;
@@ -144,7 +151,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
     for (int j = 0; j < WS; ++j) {
       mbar_init(&bar->wfull[j], 1);
-      mbar_init(&bar->wempty[j], 4);      // the four warps of the stage's group
+      mbar_init(&bar->wempty[j], 4);      // the four warps of the slot's group
       mbar_init(&bar->afull[j], 2 * 4);   // those warps in both CTAs
       mbar_init(&bar->aempty[j], 1);      // one pair commit
     }
@@ -187,10 +194,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           break;
         }
         if (xp) {
-          if (even) mbar_arrive_expect_tx(&bar->xfull[s], (odd_rows ? 2 : 1) * L::X_STAGE_BYTES);
-          if (even || odd_rows)
-            tma_load_2d_pair(xs + s * L::X_STAGE_BYTES, &x_map, kb * BK, t0 + (int)rank * HT,
-                             xfull_even + 8u * (uint32_t)s);
+          // the second 64-k half holds k below K (else it is neither loaded
+          // nor multiplied)
+          const int k0 = kb * BK;
+          const bool hi = k0 + 64 < K;
+          const uint32_t bytes = (x3d || hi) ? L::X_STAGE_BYTES : L::X_HALF_BYTES;
+          if (even) mbar_arrive_expect_tx(&bar->xfull[s], (odd_rows ? 2u : 1u) * bytes);
+          if (even || odd_rows) {
+            uint8_t* dst = xs + s * L::X_STAGE_BYTES;
+            const int row = t0 + (int)rank * HT;
+            const uint32_t bar_c = xfull_even + 8u * (uint32_t)s;
+            if (x3d) {
+              tma_load_3d_pair(dst, &x_map, 0, row, k0 / 64, bar_c);
+            } else {
+              tma_load_2d_pair(dst, &x_map, k0, row, bar_c);
+              if (hi) tma_load_2d_pair(dst + L::X_HALF_BYTES, &x_map, k0 + 64, row, bar_c);
+            }
+          }
         } else if (n0 < N) {
           uint8_t* wst = smem + L::W_OFF + s * W_STAGE_BYTES;
           mbar_arrive_expect_tx(&bar->wfull[s], QW_STAGE_BYTES + scale_rows * S_ROW_BYTES);
@@ -229,12 +249,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const uint64_t b_desc0 = smem_desc_sw128(smem_u32(xs + s * L::X_STAGE_BYTES));
         const uint32_t a_base = tmem + A_COL + a * A_STAGE_COLS;
+        const int nk = kb * BK + 64 < K ? BK / 16 : 4;  // k16 steps holding k below K
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            mma_f16_ts_pair(tmem + D_COL, a_base + kk * 8,
-                            b_desc0 + (uint64_t)((kk * 32) >> 4), idesc,
-                            (kb | kk) != 0 ? 1u : 0u);
+            if (kk < nk)
+              mma_f16_ts_pair(tmem + D_COL, a_base + kk * 8,
+                              b_desc0 + (uint64_t)(((kk >> 2) * L::X_HALF_BYTES +
+                                                    (kk & 3) * 32) >> 4),
+                              idesc, (kb | kk) != 0 ? 1u : 0u);
           mma_commit_pair(&bar->xempty[s], kPairMask);
           mma_commit_pair(&bar->aempty[a], kPairMask);
         }
@@ -263,9 +286,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint8_t* s_tile = smem + L::W_OFF + QW_STAGE_BYTES + col * 2;
 
     bool ok = true;
+    const int j = grp;  // this group's weight slot and A slot
+    const uint8_t* qw = qw_tile + j * W_STAGE_BYTES;
+    const uint8_t* sc = s_tile + j * W_STAGE_BYTES;
     for (int kb = grp; kb < KB; kb += DQ_GROUPS) {
-      const int j = kb % WS;
-      const uint32_t ph = (uint32_t)(kb / WS) & 1u;
+      const uint32_t ph = (uint32_t)(kb / DQ_GROUPS) & 1u;
       // qweight and scale tiles of the stage have landed
       ok = __all_sync(0xffffffffu,
                       mbar_wait_bounded<true>(&bar->wfull[j], ph, abort_flag, kWaitLimitNs));
@@ -273,32 +298,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (lane == 0) record_timeout(err, bar);
         break;
       }
-      const uint8_t* qw = qw_tile + j * W_STAGE_BYTES;
-      const uint8_t* sc = s_tile + j * W_STAGE_BYTES;
+      // the stage's 16 packed rows, one 64-k half (32 TMEM columns) at a time
       uint32_t cells[32];
 #pragma unroll
-      for (int r = 0; r < BK / 8; ++r) {
-        // scale row of packed row r inside the stage (0 unless the group is
-        // smaller than the 64-k stage)
-        const int gl = group_shift >= 6 ? 0 : (r * 8) >> group_shift;
-        const uint16_t sv = *reinterpret_cast<const uint16_t*>(sc + gl * S_ROW_BYTES);
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(qw + r * (BW * 4));
-        uint32_t nat[4];
-        dequant_word_natural(w, half2_broadcast(sv), nat);
+      for (int h = 0; h < 2; ++h) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) cells[4 * r + q] = nat[q];
+        for (int r8 = 0; r8 < 8; ++r8) {
+          const int r = 8 * h + r8;
+          // scale row of packed row r inside the stage (0 unless the group is
+          // smaller than the 128-k stage)
+          const int gl = group_shift >= 7 ? 0 : (r * 8) >> group_shift;
+          const uint16_t sv = *reinterpret_cast<const uint16_t*>(sc + gl * S_ROW_BYTES);
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(qw + r * (BW * 4));
+          uint32_t nat[4];
+          dequant_word_natural(w, half2_broadcast(sv), nat);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) cells[4 * r8 + q] = nat[q];
+        }
+        if (h == 0) {
+          // the A slot is free once the pair MMAs of its previous use completed
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded<true>(&bar->aempty[j], ph ^ 1u,
+                                                               abort_flag, kWaitLimitNs));
+          if (!ok) break;
+          tc_fence_after();
+        } else {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar->wempty[j]);  // weight tiles of the stage read
+        }
+        tmem_st_32x32b_x32(tmem + lane_addr + A_COL + j * A_STAGE_COLS + 32 * h, cells);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->wempty[j]);  // weight tiles of the stage read
-      // the A slot is free once the pair MMAs of its previous use completed
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded<true>(&bar->aempty[j], ph ^ 1u, abort_flag,
-                                                           kWaitLimitNs));
       if (!ok) {
         if (lane == 0) record_timeout(err, bar);
         break;
       }
-      tc_fence_after();
-      tmem_st_32x32b_x32(tmem + lane_addr + A_COL + j * A_STAGE_COLS, cells);
       tmem_wait_st();  // the whole warp's cells are in TMEM
       tc_fence_before();
       __syncwarp();
@@ -350,8 +382,20 @@ cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint1
                           const DeviceInfo& dev) {
   using L = PairLayout<BT>;
   CUtensorMap x_map, qw_map, s_map;
-  if (!tensor_map_2d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M,
-                     (uint64_t)K * 2, BK, L::HT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  // X as [K/64][M][64] (one copy of both 64-k halves per stage) when K is a
+  // multiple of 64, else as [M][K] (one copy per half); rows at or beyond M
+  // and k at or beyond K read as zero either way
+  int x3d = 0;
+  if (K % 64 == 0) {
+    const uint64_t dims[3] = {64, (uint64_t)M, (uint64_t)(K / 64)};
+    const uint64_t strides[2] = {(uint64_t)K * 2, 128};
+    const uint32_t box[3] = {64, (uint32_t)L::HT, 2};
+    x3d = tensor_map_3d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, dims, strides, box,
+                        CU_TENSOR_MAP_SWIZZLE_128B) ? 1 : 0;
+  }
+  if ((!x3d && !tensor_map_2d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K,
+                              (uint64_t)M, (uint64_t)K * 2, 64, L::HT,
+                              CU_TENSOR_MAP_SWIZZLE_128B)) ||
       !tensor_map_2d(&qw_map, qweight, CU_TENSOR_MAP_DATA_TYPE_INT32, (uint64_t)N,
                      (uint64_t)(K / 8), (uint64_t)N * 4, BW, BK / 8, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !tensor_map_2d(&s_map, scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, (uint64_t)N,
@@ -373,7 +417,7 @@ cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint1
   const dim3 grid(ctas_n, (unsigned)((M + BT - 1) / BT), 1);
   prefill_pair_kernel<BT><<<grid, THREADS, smem, stream>>>(x_map, qw_map, s_map, y, (int)M,
                                                            (int)K, (int)N, group_shift,
-                                                           scale_rows, dev.error_word);
+                                                           scale_rows, x3d, dev.error_word);
   return cudaGetLastError();
 }
 
@@ -385,7 +429,7 @@ cudaError_t launch_prefill_pair(const uint16_t* x, const int32_t* qweight,
                                 const DeviceInfo& dev) {
   const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
                                ? 1 : (K + (int64_t(1) << group_shift) - 1) >> group_shift;
-  const int scale_rows = group_shift >= 6 ? 1 : (BK >> group_shift);
+  const int scale_rows = group_shift >= 7 ? 1 : (BK >> group_shift);
   if (M <= 128)
     return launch_pair_t<128>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups,
                               stream, dev);

@@ -257,6 +257,18 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst_smem, const CUtensorM
       : "memory");
 }
 
+// 3-D tile load into this CTA's shared memory, bytes counted on an mbarrier
+// of either CTA of the pair (as tma_load_2d_pair).
+__device__ __forceinline__ void tma_load_3d_pair(void* dst_smem, const CUtensorMap* map,
+                                                 int32_t c0, int32_t c1, int32_t c2,
+                                                 uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst_smem)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
