@@ -12,7 +12,7 @@
 //
 // * each CTA dequantises its own 128 weight columns into its own TMEM (A rows
 //   0..127 live in the even CTA, rows 128..255 in the odd one);
-// * each CTA loads only HALF of the X tile (BT/2 token rows x 64 k per
+// * each CTA loads only HALF of the X tile (BT/2 token rows x 128 k per
 //   stage); the pair MMA reads B rows 0..BT/2-1 from the even CTA and the
 //   rest from the odd CTA, so every X byte crosses from L2 once per pair
 //   instead of once per CTA;
@@ -26,6 +26,15 @@
 // memory is where most of the power of this kernel goes: with half of it the
 // SMs hold a higher clock under the board's power limit.
 //
+// The kernel is persistent: one cluster per SM pair walks the tiles (column
+// pair fastest), and every ring continues across tiles.  The accumulator is
+// drained by the dequantisation warps between two of their stages: each
+// group reads its quarter of the tokens from TMEM, hands the accumulator back
+// to the MMA warp at once, then rounds to FP16 into a shared-memory staging
+// tile that one TMA store writes to Y.  So the next tile's copies,
+// dequantisation and MMAs overlap the previous tile's epilogue, and no CTA
+// launch, TMEM allocation or pipeline fill is paid per tile.
+//
 // Every wait is bounded in time; on expiry the CTA records GPTQ_ERR_TIMEOUT
 // in the device error word and winds down.  Both CTAs always reach the final
 // cluster barrier, so neither leaves while the other may still signal it.
@@ -33,6 +42,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -46,10 +56,10 @@ namespace {
 
 constexpr int BW = 128;   // weight columns per CTA (TMEM lanes); 256 per pair (MMA M)
 constexpr int BK = 128;   // k per pipeline stage (eight k16 MMAs)
-constexpr int XS = 4;     // X ring stages (half tile per CTA)
+constexpr int XS = 3;     // X ring stages (half tile per CTA)
 constexpr int WS = 4;     // weight-tile ring stages (qweight + scales of 128 k)
 constexpr int AS = 4;     // A slots in TMEM (128 k each)
-constexpr int DQ_GROUPS = 4;             // dequantisation groups: group g takes stages kb = g mod 4
+constexpr int DQ_GROUPS = 4;             // dequantisation groups: group g takes stages g mod 4
 constexpr int DQ_WARPS = 4 * DQ_GROUPS;  // one warp per TMEM lane quarter in each group
 constexpr int DQ_WARP0 = 3;  // warps 0, 1, 2: X producer, MMA issuer, weight producer
 constexpr int THREADS = (DQ_WARP0 + DQ_WARPS) * 32;
@@ -65,32 +75,43 @@ constexpr uint16_t kPairMask = 0x3;        // both CTAs of the cluster
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 static_assert(A_COL + AS * A_STAGE_COLS <= TMEM_COLS, "TMEM budget");
-static_assert(AS == WS && XS == WS && WS == DQ_GROUPS,
-              "stage kb uses X, weight and A slot kb mod 4, dequantised by group kb mod 4");
+static_assert(AS == WS && WS == DQ_GROUPS,
+              "stage g uses weight and A slot g mod 4 and is dequantised by group g mod 4");
 
 // Shared-memory layout for a pair token tile of BT (BT/2 X rows per CTA).
 // An X stage is two 64-k halves, each BT/2 rows of 128 bytes (128-byte
-// swizzle), the second right after the first.
+// swizzle), the second right after the first.  The staging area holds this
+// CTA's 128 columns x BT tokens of Y in FP16: one block of BT/4 tokens x 32
+// columns (token-major, 64-byte rows) per dequantisation warp, which stores
+// it to Y on its own.
 template <int BT>
 struct PairLayout {
   static constexpr int HT = BT / 2;
+  static constexpr int TPG = BT / DQ_GROUPS;  // tokens drained per group
   static constexpr int X_HALF_BYTES = HT * 64 * 2;
   static constexpr int X_STAGE_BYTES = 2 * X_HALF_BYTES;
   static constexpr int W_OFF = XS * X_STAGE_BYTES;
-  static constexpr int BAR_OFF = W_OFF + WS * W_STAGE_BYTES;
+  static constexpr int Y_OFF = W_OFF + WS * W_STAGE_BYTES;
+  static constexpr int Y_WARP_BYTES = TPG * 32 * 2;
+  static constexpr int Y_GROUP_BYTES = 4 * Y_WARP_BYTES;
+  static constexpr int BAR_OFF = Y_OFF + DQ_GROUPS * Y_GROUP_BYTES;
   static constexpr size_t kSmemBytes = 1024 + (size_t)BAR_OFF + 512;
   static_assert(X_HALF_BYTES % 1024 == 0, "128-byte swizzle atoms stay aligned");
+  static_assert(Y_OFF % 128 == 0 && Y_WARP_BYTES % 128 == 0, "store sources aligned");
+  static_assert(TPG % 32 == 0, "drained in 32-column TMEM loads");
 };
 
-// Both CTAs hold the full set; xfull and afull are only used in the even CTA.
+// Both CTAs hold the full set; xfull, afull and dempty are only used in the
+// even CTA.
 struct PairBarriers {
-  uint64_t xfull[XS];   // both halves of the X tile landed (even CTA)
+  uint64_t xfull[XS];   // both halves of the X stage landed (even CTA)
   uint64_t xempty[XS];  // pair MMAs reading the X stage done
   uint64_t wfull[WS];   // this CTA's qweight and scale tiles landed
   uint64_t wempty[WS];  // weight tiles read by this CTA's group warps
   uint64_t afull[AS];   // A slot written by the group warps of both CTAs (even CTA)
   uint64_t aempty[AS];  // pair MMAs reading the A slot done
-  uint64_t dfull;       // all MMAs of the tile done
+  uint64_t dfull;       // all MMAs of the current tile done
+  uint64_t dempty;      // accumulator read out by every group warp of both CTAs (even CTA)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -110,20 +131,38 @@ __device__ __forceinline__ bool elect_one() {
   return p != 0;
 }
 
+// The tiles of one cluster: tile = cluster + i * clusters for i = 0, 1, ...;
+// column pair fastest.
+struct TileWalk {
+  int cluster, clusters, n_pairs, tiles;
+  __device__ int count() const {
+    return cluster < tiles ? (tiles - cluster + clusters - 1) / clusters : 0;
+  }
+  __device__ void coords(int i, int bt, uint32_t rank, int& n0, int& t0) const {
+    const int tile = cluster + i * clusters;
+    n0 = (2 * (tile % n_pairs) + (int)rank) * BW;
+    t0 = (tile / n_pairs) * bt;
+  }
+};
+
 // scale_rows: scale rows one 128-k stage touches (1, or 128/group for groups
 // below 128); stages start on 128-k boundaries, so they align with groups.
 // x3d: X is read through a [K/64][M][64] view, one copy per stage (K a
 // multiple of 64); otherwise through [M][K], one copy per 64-k half.
+// n_pairs, tiles: column pairs (of 256) and pair tiles (n_pairs x token
+// tiles); cluster c takes tiles c, c + clusters, ...
 template <int BT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap x_map,
                         const __grid_constant__ CUtensorMap qw_map,
-                        const __grid_constant__ CUtensorMap s_map, uint16_t* __restrict__ y,
-                        int M, int K, int N, int group_shift, int scale_rows, int x3d,
+                        const __grid_constant__ CUtensorMap s_map,
+                        const __grid_constant__ CUtensorMap y_map, int M, int K, int N,
+                        int group_shift, int scale_rows, int x3d, int n_pairs, int tiles,
                         int* err) {
   static_assert(BT == 128 || BT == 256, "pair token tile");
   using L = PairLayout<BT>;
   constexpr int HT = L::HT;
+  constexpr int TPG = L::TPG;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base; the same offset in both CTAs, so that one MMA
   // descriptor and one barrier offset name the matching buffers of the pair
@@ -135,14 +174,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0: even CTA (issues the MMAs), 1: odd CTA
   const bool even = rank == 0;
-  const int n0 = blockIdx.x * BW;
-  const int t0 = blockIdx.y * BT;
-  const int KB = (K + BK - 1) / BK;
-  // Does the odd CTA's half of the token tile hold any row below M?  If not,
-  // it loads nothing (no copy box lies wholly outside X) and the even CTA
-  // expects only its own bytes; the MMA then reads stale shared memory for
-  // token columns that are never stored.
-  const bool odd_rows = t0 + HT < M;
+  const TileWalk walk{(int)(blockIdx.x >> 1), (int)(gridDim.x >> 1), n_pairs, tiles};
+  const int NT = walk.count();          // tiles of this cluster
+  const int KB = (K + BK - 1) / BK;     // stages per tile
+  const int G = NT * KB;                // stages of this cluster, over all its tiles
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < XS; ++s) {
@@ -155,7 +190,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&bar->afull[j], 2 * 4);   // those warps in both CTAs
       mbar_init(&bar->aempty[j], 1);      // one pair commit
     }
-    mbar_init(&bar->dfull, 1);
+    mbar_init(&bar->dfull, 1);                 // one pair commit per tile
+    mbar_init(&bar->dempty, 2 * DQ_WARPS);     // every group warp of both CTAs
     bar->abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -163,6 +199,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     prefetch_tensormap(&x_map);
     prefetch_tensormap(&qw_map);
     prefetch_tensormap(&s_map);
+    prefetch_tensormap(&y_map);
   }
   __syncwarp();
   if (warp == 1) {
@@ -178,25 +215,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   // the even CTA's barriers that both CTAs signal
   const uint32_t xfull_even = map_to_rank(smem_u32(&bar->xfull[0]), 0);
   const uint32_t afull_even = map_to_rank(smem_u32(&bar->afull[0]), 0);
+  const uint32_t dempty_even = map_to_rank(smem_u32(&bar->dempty), 0);
 
   if (warp == 0 || warp == 2) {
     // ---------------- TMA producers: X half (warp 0), weights (warp 2) ----------------
-    if (lane == 0) {
+    if (lane == 0 && NT > 0) {
       const bool xp = warp == 0;
       const int depth = xp ? XS : WS;
+      int it = 0, kb = 0, n0, t0;
+      walk.coords(0, BT, rank, n0, t0);
+      // Does the odd CTA's half of the token tile hold any row below M?  If
+      // not, it loads nothing (no copy box lies wholly outside X) and the
+      // even CTA expects only its own bytes; the MMA then reads stale shared
+      // memory for token columns that are never stored.
+      bool odd_rows = t0 + HT < M;
       int issued = 0;
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % depth;
-        const uint32_t ph = (uint32_t)(kb / depth) & 1u;
+      for (int g = 0; g < G; ++g) {
+        const int s = g % depth;
+        const uint32_t ph = (uint32_t)(g / depth) & 1u;
         uint64_t* emp = xp ? &bar->xempty[s] : &bar->wempty[s];
         if (!mbar_wait_bounded(emp, ph ^ 1u, abort_flag, kWaitLimitNs)) {
           record_timeout(err, bar);
           break;
         }
+        const int k0 = kb * BK;
         if (xp) {
           // the second 64-k half holds k below K (else it is neither loaded
           // nor multiplied)
-          const int k0 = kb * BK;
           const bool hi = k0 + 64 < K;
           const uint32_t bytes = (x3d || hi) ? L::X_STAGE_BYTES : L::X_HALF_BYTES;
           if (even) mbar_arrive_expect_tx(&bar->xfull[s], (odd_rows ? 2u : 1u) * bytes);
@@ -214,13 +259,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         } else if (n0 < N) {
           uint8_t* wst = smem + L::W_OFF + s * W_STAGE_BYTES;
           mbar_arrive_expect_tx(&bar->wfull[s], QW_STAGE_BYTES + scale_rows * S_ROW_BYTES);
-          tma_load_2d(wst, &qw_map, n0, kb * (BK / 8), &bar->wfull[s]);
-          tma_load_2d(wst + QW_STAGE_BYTES, &s_map, n0, (int)(((int64_t)kb * BK) >> group_shift),
+          tma_load_2d(wst, &qw_map, n0, k0 / 8, &bar->wfull[s]);
+          tma_load_2d(wst + QW_STAGE_BYTES, &s_map, n0, (int)((int64_t)k0 >> group_shift),
                       &bar->wfull[s]);
         } else {
           mbar_arrive(&bar->wfull[s]);  // padding CTA: no columns, nothing to load
         }
         ++issued;
+        if (++kb == KB) {
+          kb = 0;
+          if (++it < NT) {
+            walk.coords(it, BT, rank, n0, t0);
+            odd_rows = t0 + HT < M;
+          }
+        }
       }
       if (*abort_flag && (!xp || even)) {
         // drain: wait for the last loads issued into each slot (the odd
@@ -238,59 +290,125 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (even) {
       const uint32_t idesc = idesc_f16_f32(2 * BW, BT);
       bool ok = true;
-      for (int kb = 0; kb < KB && ok; ++kb) {
-        const int s = kb % XS, a = kb % AS;
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait_bounded(&bar->xfull[s], (uint32_t)(kb / XS) & 1u, abort_flag,
-                                          kWaitLimitNs) &&
-                            mbar_wait_bounded(&bar->afull[a], (uint32_t)(kb / AS) & 1u,
-                                              abort_flag, kWaitLimitNs));
-        if (!ok) break;
-        tc_fence_after();
-        const uint64_t b_desc0 = smem_desc_sw128(smem_u32(xs + s * L::X_STAGE_BYTES));
-        const uint32_t a_base = tmem + A_COL + a * A_STAGE_COLS;
-        const int nk = kb * BK + 64 < K ? BK / 16 : 4;  // k16 steps holding k below K
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            if (kk < nk)
-              mma_f16_ts_pair(tmem + D_COL, a_base + kk * 8,
-                              b_desc0 + (uint64_t)(((kk >> 2) * L::X_HALF_BYTES +
-                                                    (kk & 3) * 32) >> 4),
-                              idesc, (kb | kk) != 0 ? 1u : 0u);
-          mma_commit_pair(&bar->xempty[s], kPairMask);
-          mma_commit_pair(&bar->aempty[a], kPairMask);
+      int g = 0, it = 0;
+      for (; it < NT && ok; ++it) {
+        if (it > 0) {
+          // the previous tile's accumulator has been read out by every group
+          // warp of both CTAs
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar->dempty, (uint32_t)(it - 1) & 1u,
+                                                         abort_flag, kWaitLimitNs));
+          if (!ok) break;
+          tc_fence_after();
         }
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          const int s = g % XS, a = g % AS;
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait_bounded(&bar->xfull[s], (uint32_t)(g / XS) & 1u, abort_flag,
+                                            kWaitLimitNs) &&
+                              mbar_wait_bounded(&bar->afull[a], (uint32_t)(g / AS) & 1u,
+                                                abort_flag, kWaitLimitNs));
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t b_desc0 = smem_desc_sw128(smem_u32(xs + s * L::X_STAGE_BYTES));
+          const uint32_t a_base = tmem + A_COL + a * A_STAGE_COLS;
+          const int nk = kb * BK + 64 < K ? BK / 16 : 4;  // k16 steps holding k below K
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              if (kk < nk)
+                mma_f16_ts_pair(tmem + D_COL, a_base + kk * 8,
+                                b_desc0 + (uint64_t)(((kk >> 2) * L::X_HALF_BYTES +
+                                                      (kk & 3) * 32) >> 4),
+                                idesc, (kb | kk) != 0 ? 1u : 0u);
+            mma_commit_pair(&bar->xempty[s], kPairMask);
+            mma_commit_pair(&bar->aempty[a], kPairMask);
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (elect_one()) mma_commit_pair(&bar->dfull, kPairMask);  // tile done
         __syncwarp();
       }
-      if (!ok && lane == 0) record_timeout(err, bar);
-      if (elect_one()) mma_commit_pair(&bar->dfull, kPairMask);
-      __syncwarp();
       if (!ok) {
+        if (lane == 0) record_timeout(err, bar);
+        // wait for the MMAs already issued before anyone frees TMEM
+        if (elect_one()) mma_commit_pair(&bar->dfull, kPairMask);
+        __syncwarp();
         int never = 0;
-        mbar_wait_bounded(&bar->dfull, 0, &never, kDrainLimitNs);
+        mbar_wait_bounded(&bar->dfull, (uint32_t)it & 1u, &never, kDrainLimitNs);
       }
     }
     __syncwarp();  // the whole warp reaches the cluster barrier below together
   } else {
-    // ---------------- dequantisation, then epilogue ----------------
+    // ---------------- dequantisation and accumulator read-out ----------------
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
-    const int grp = (warp - DQ_WARP0) >> 2;  // stages kb = grp mod DQ_GROUPS
-    const int n = n0 + 32 * quarter + lane;
-    const bool col_ok = n < N;
+    const int grp = (warp - DQ_WARP0) >> 2;  // stages g = grp mod DQ_GROUPS
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
+    const int col = 32 * quarter + lane;     // this thread's column in the tile
+    const int j = grp;                       // this group's weight slot and A slot
+    const uint8_t* qw = smem + L::W_OFF + j * W_STAGE_BYTES + col * 4;
+    const uint8_t* sc = smem + L::W_OFF + j * W_STAGE_BYTES + QW_STAGE_BYTES + col * 2;
+    uint8_t* ystage = smem + L::Y_OFF + grp * L::Y_GROUP_BYTES + quarter * L::Y_WARP_BYTES;
 
-    // this thread's column in the stage's qweight and scale tiles
-    const int col = 32 * quarter + lane;
-    const uint8_t* qw_tile = smem + L::W_OFF + col * 4;
-    const uint8_t* s_tile = smem + L::W_OFF + QW_STAGE_BYTES + col * 2;
+    // Reads out tile d's accumulator (this warp's 32 lanes x its group's TPG
+    // tokens), hands it back to the MMA warp, and stores the FP16 values to
+    // Y through this warp's staging block.  False if the wait expired.
+    auto drain = [&](int d) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded<true>(&bar->dfull, (uint32_t)d & 1u,
+                                                           abort_flag, kWaitLimitNs)))
+        return false;
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      tmem_ld_32x32b_x32(tmem + lane_addr + D_COL + grp * TPG, v0);
+      if constexpr (TPG == 64) tmem_ld_32x32b_x32(tmem + lane_addr + D_COL + grp * TPG + 32, v1);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(dempty_even);  // the MMAs may overwrite it now
+      int dn0, dt0;
+      walk.coords(d, BT, rank, dn0, dt0);
+      if (lane == 0) bulk_wait_read_all();  // the block's previous store has read it
+      __syncwarp();
+      uint16_t* ys = reinterpret_cast<uint16_t*>(ystage);
+#pragma unroll
+      for (int q = 0; q < 32; ++q)
+        ys[q * 32 + lane] = __half_as_ushort(__float2half_rn(__uint_as_float(v0[q])));
+      if constexpr (TPG == 64) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          ys[(32 + q) * 32 + lane] = __half_as_ushort(__float2half_rn(__uint_as_float(v1[q])));
+      }
+      fence_proxy_async_smem();  // the staging writes are visible to the store
+      __syncwarp();
+      const int c0 = dn0 + 32 * quarter, tok0 = dt0 + grp * TPG;
+      if (lane == 0 && c0 < N && tok0 < M) {
+        tma_store_2d(&y_map, ystage, c0, tok0);
+        bulk_commit_group();
+      }
+      return true;
+    };
 
     bool ok = true;
-    const int j = grp;  // this group's weight slot and A slot
-    const uint8_t* qw = qw_tile + j * W_STAGE_BYTES;
-    const uint8_t* sc = s_tile + j * W_STAGE_BYTES;
-    for (int kb = grp; kb < KB; kb += DQ_GROUPS) {
-      const uint32_t ph = (uint32_t)(kb / DQ_GROUPS) & 1u;
+    int drained = 0;  // tiles whose accumulator this warp has read out
+    for (int g = grp; g < G; g += DQ_GROUPS) {
+      // Read out every finished tile before this stage.  One must be read
+      // out first if this stage's A slot was last used by a later tile, whose
+      // MMAs wait for the accumulator.
+      const int it = g / KB;
+      while (drained < it) {
+        const bool forced = g - AS >= (drained + 1) * KB;
+        const bool done = __shfl_sync(
+            0xffffffffu, (int)mbar_test_wait(smem_u32(&bar->dfull), (uint32_t)drained & 1u), 0);
+        if (!forced && !done) break;
+        ok = drain(drained);
+        if (!ok) break;
+        ++drained;
+      }
+      if (!ok) {
+        if (lane == 0) record_timeout(err, bar);
+        break;
+      }
+      const uint32_t ph = (uint32_t)(g / DQ_GROUPS) & 1u;
       // qweight and scale tiles of the stage have landed
       ok = __all_sync(0xffffffffu,
                       mbar_wait_bounded<true>(&bar->wfull[j], ph, abort_flag, kWaitLimitNs));
@@ -336,32 +454,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(afull_even + 8u * (uint32_t)j);
     }
-
-    if (ok) {
-      ok = mbar_wait_bounded<true>(&bar->dfull, 0, abort_flag, kWaitLimitNs);
-      ok = __all_sync(0xffffffffu, ok);
+    // the tiles not read out yet
+    while (ok && drained < NT) {
+      ok = drain(drained);
       if (!ok && lane == 0) record_timeout(err, bar);
+      ++drained;
     }
-    if (ok) {
-      // group g writes tokens [g*BT/4, (g+1)*BT/4) of the tile, 16 at a time
-      tc_fence_after();
-      constexpr int TPG = BT / DQ_GROUPS;
-#pragma unroll 1
-      for (int chunk = 0; chunk < TPG / 16; ++chunk) {
-        const int tok0 = TPG * grp + 16 * chunk;
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(tmem + lane_addr + D_COL + tok0, r);
-        tmem_wait_ld();
-        if (col_ok) {
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const int t = t0 + tok0 + q;
-            if (t < M)
-              y[(int64_t)t * N + n] = __half_as_ushort(__float2half_rn(__uint_as_float(r[q])));
-          }
-        }
-      }
-    }
+    if (lane == 0) bulk_wait_all();  // this warp's stores have completed
+    __syncwarp();
   }
 
   // neither CTA leaves (or frees TMEM) while the pair's MMAs, loads or
@@ -381,7 +481,7 @@ cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint1
                           int scale_rows, int64_t n_groups, cudaStream_t stream,
                           const DeviceInfo& dev) {
   using L = PairLayout<BT>;
-  CUtensorMap x_map, qw_map, s_map;
+  CUtensorMap x_map, qw_map, s_map, y_map;
   // X as [K/64][M][64] (one copy of both 64-k halves per stage) when K is a
   // multiple of 64, else as [M][K] (one copy per half); rows at or beyond M
   // and k at or beyond K read as zero either way
@@ -400,7 +500,10 @@ cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint1
                      (uint64_t)(K / 8), (uint64_t)N * 4, BW, BK / 8, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !tensor_map_2d(&s_map, scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, (uint64_t)N,
                      (uint64_t)n_groups, (uint64_t)N * 2, BW, (uint32_t)scale_rows,
-                     CU_TENSOR_MAP_SWIZZLE_NONE))
+                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      // Y blocks of 32 columns x BT/4 tokens, one per dequantisation warp
+      !tensor_map_2d(&y_map, y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)N, (uint64_t)M,
+                     (uint64_t)N * 2, 32, L::TPG, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   constexpr size_t smem = L::kSmemBytes;
   static std::once_flag attr_once[64];
@@ -411,13 +514,14 @@ cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint1
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   });
   if (attr_err[d] != cudaSuccess) return attr_err[d];
-  // an even number of 128-column CTAs: with an odd count the last pair's odd
-  // CTA has no columns, loads no weights and stores nothing
-  const unsigned ctas_n = (unsigned)(((N + BW - 1) / BW + 1) & ~int64_t(1));
-  const dim3 grid(ctas_n, (unsigned)((M + BT - 1) / BT), 1);
-  prefill_pair_kernel<BT><<<grid, THREADS, smem, stream>>>(x_map, qw_map, s_map, y, (int)M,
-                                                           (int)K, (int)N, group_shift,
-                                                           scale_rows, x3d, dev.error_word);
+  // column pairs of 2 x 128 (with an odd count of 128-column tiles the last
+  // pair's odd CTA has no columns: it loads no weights and stores nothing)
+  const int64_t n_pairs = ((N + BW - 1) / BW + 1) / 2;
+  const int64_t tiles = n_pairs * ((M + BT - 1) / BT);
+  const int64_t clusters = std::min<int64_t>(tiles, std::max(1, dev.num_sms / 2));
+  prefill_pair_kernel<BT><<<dim3((unsigned)(2 * clusters)), THREADS, smem, stream>>>(
+      x_map, qw_map, s_map, y_map, (int)M, (int)K, (int)N, group_shift, scale_rows, x3d,
+      (int)n_pairs, (int)tiles, dev.error_word);
   return cudaGetLastError();
 }
 
