@@ -356,22 +356,21 @@ cudaError_t launch_t(const uint16_t* x, const int32_t* qweight, const uint16_t* 
 
 }  // namespace
 
-// The token tile follows M (64 or 128 tokens per CTA, then 256 per CTA pair),
-// so that small M does not pay for MMAs over empty token columns.
+// Up to 32 tokens (reached only when prefill is forced: the dispatcher sends
+// M <= 32 to the decode kernel) one CTA per 128 columns x 64 tokens; above
+// that the pair kernel, whose token tile (128 or 256) follows M.
 cudaError_t launch_prefill(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                            uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
                            cudaStream_t stream, const DeviceInfo& dev) {
   const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
                                ? 1 : (K + (int64_t(1) << group_shift) - 1) >> group_shift;
   const int scale_rows = group_shift >= 6 ? 1 : (BK >> group_shift);
-  if (M <= 64)
-    return launch_t<64>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups, stream,
-                        dev);
-  if (M <= 128)
-    return launch_t<128>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups, stream,
-                         dev);
-  // above 128 tokens the CTA-pair kernel takes over: half the X traffic per SM
-  return launch_prefill_pair(x, qweight, scales, y, M, K, N, group_shift, stream, dev);
+  // above 32 tokens the persistent CTA-pair kernel takes over (128- or
+  // 256-token pair tiles): half the X traffic per SM, no per-tile launch
+  if (M > 32)
+    return launch_prefill_pair(x, qweight, scales, y, M, K, N, group_shift, stream, dev);
+  return launch_t<64>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups, stream,
+                      dev);
 }
 
 }  // namespace gptq

@@ -56,9 +56,9 @@ namespace {
 
 constexpr int BW = 128;   // weight columns per CTA (TMEM lanes); 256 per pair (MMA M)
 constexpr int BK = 128;   // k per pipeline stage (eight k16 MMAs)
-constexpr int XS = 3;     // X ring stages (half tile per CTA)
-constexpr int WS = 4;     // weight-tile ring stages (qweight + scales of 128 k)
-constexpr int AS = 4;     // A slots in TMEM (128 k each)
+constexpr int XS_MAX = 4;   // X ring stages (half tile per CTA), at most
+constexpr int WS_MAX = 12;  // weight-tile ring stages (qweight + scales of 128 k), at most
+constexpr int AS = 4;       // A slots in TMEM (128 k each)
 constexpr int DQ_GROUPS = 4;             // dequantisation groups: group g takes stages g mod 4
 constexpr int DQ_WARPS = 4 * DQ_GROUPS;  // one warp per TMEM lane quarter in each group
 constexpr int DQ_WARP0 = 3;  // warps 0, 1, 2: X producer, MMA issuer, weight producer
@@ -75,10 +75,12 @@ constexpr uint16_t kPairMask = 0x3;        // both CTAs of the cluster
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 static_assert(A_COL + AS * A_STAGE_COLS <= TMEM_COLS, "TMEM budget");
-static_assert(AS == WS && WS == DQ_GROUPS,
-              "stage g uses weight and A slot g mod 4 and is dequantised by group g mod 4");
+static_assert(AS == DQ_GROUPS, "stage g uses A slot g mod 4 and is dequantised by group g mod 4");
 
-// Shared-memory layout for a pair token tile of BT (BT/2 X rows per CTA).
+// Ring depths and shared-memory layout for a pair token tile of BT (BT/2 X
+// rows per CTA).  The weight ring is as deep as shared memory allows: below
+// a few token tiles every weight stage comes from HBM, and the bytes a CTA
+// keeps in flight set its streaming rate.
 // An X stage is two 64-k halves, each BT/2 rows of 128 bytes (128-byte
 // swizzle), the second right after the first.  The staging area holds this
 // CTA's 128 columns x BT tokens of Y in FP16: one block of BT/4 tokens x 32
@@ -86,6 +88,8 @@ static_assert(AS == WS && WS == DQ_GROUPS,
 // it to Y on its own.
 template <int BT>
 struct PairLayout {
+  static constexpr int XS = BT == 256 ? 3 : 4;
+  static constexpr int WS = BT == 256 ? 4 : 8;
   static constexpr int HT = BT / 2;
   static constexpr int TPG = BT / DQ_GROUPS;  // tokens drained per group
   static constexpr int X_HALF_BYTES = HT * 64 * 2;
@@ -99,15 +103,17 @@ struct PairLayout {
   static_assert(X_HALF_BYTES % 1024 == 0, "128-byte swizzle atoms stay aligned");
   static_assert(Y_OFF % 128 == 0 && Y_WARP_BYTES % 128 == 0, "store sources aligned");
   static_assert(TPG % 32 == 0, "drained in 32-column TMEM loads");
+  static_assert(XS <= XS_MAX && WS <= WS_MAX && WS % DQ_GROUPS == 0,
+                "weight slot g mod WS is always used by group g mod 4");
 };
 
 // Both CTAs hold the full set; xfull, afull and dempty are only used in the
 // even CTA.
 struct PairBarriers {
-  uint64_t xfull[XS];   // both halves of the X stage landed (even CTA)
-  uint64_t xempty[XS];  // pair MMAs reading the X stage done
-  uint64_t wfull[WS];   // this CTA's qweight and scale tiles landed
-  uint64_t wempty[WS];  // weight tiles read by this CTA's group warps
+  uint64_t xfull[XS_MAX];   // both halves of the X stage landed (even CTA)
+  uint64_t xempty[XS_MAX];  // pair MMAs reading the X stage done
+  uint64_t wfull[WS_MAX];   // this CTA's qweight and scale tiles landed
+  uint64_t wempty[WS_MAX];  // weight tiles read by this CTA's group warps
   uint64_t afull[AS];   // A slot written by the group warps of both CTAs (even CTA)
   uint64_t aempty[AS];  // pair MMAs reading the A slot done
   uint64_t dfull;       // all MMAs of the current tile done
@@ -163,6 +169,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   using L = PairLayout<BT>;
   constexpr int HT = L::HT;
   constexpr int TPG = L::TPG;
+  constexpr int XS = L::XS;
+  constexpr int WS = L::WS;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base; the same offset in both CTAs, so that one MMA
   // descriptor and one barrier offset name the matching buffers of the pair
@@ -187,7 +195,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int j = 0; j < WS; ++j) {
       mbar_init(&bar->wfull[j], 1);
       mbar_init(&bar->wempty[j], 4);      // the four warps of the slot's group
-      mbar_init(&bar->afull[j], 2 * 4);   // those warps in both CTAs
+    }
+    for (int j = 0; j < AS; ++j) {
+      mbar_init(&bar->afull[j], 2 * 4);   // the slot's group warps in both CTAs
       mbar_init(&bar->aempty[j], 1);      // one pair commit
     }
     mbar_init(&bar->dfull, 1);                 // one pair commit per tile
@@ -219,35 +229,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
   if (warp == 0 || warp == 2) {
     // ---------------- TMA producers: X half (warp 0), weights (warp 2) ----------------
+    // One thread each.  The loops are kept lean (ring depth known at compile
+    // time, slot and phase advanced incrementally, per-tile values hoisted):
+    // below a few hundred tokens the MMAs are short and the issue rate of
+    // these threads sets the pace.
     if (lane == 0 && NT > 0) {
-      const bool xp = warp == 0;
-      const int depth = xp ? XS : WS;
       int it = 0, kb = 0, n0, t0;
       walk.coords(0, BT, rank, n0, t0);
-      // Does the odd CTA's half of the token tile hold any row below M?  If
-      // not, it loads nothing (no copy box lies wholly outside X) and the
-      // even CTA expects only its own bytes; the MMA then reads stale shared
-      // memory for token columns that are never stored.
-      bool odd_rows = t0 + HT < M;
+      int s = 0;
+      uint32_t ph = 0;
       int issued = 0;
-      for (int g = 0; g < G; ++g) {
-        const int s = g % depth;
-        const uint32_t ph = (uint32_t)(g / depth) & 1u;
-        uint64_t* emp = xp ? &bar->xempty[s] : &bar->wempty[s];
-        if (!mbar_wait_bounded(emp, ph ^ 1u, abort_flag, kWaitLimitNs)) {
-          record_timeout(err, bar);
-          break;
-        }
-        const int k0 = kb * BK;
-        if (xp) {
+      if (warp == 0) {
+        // Does the odd CTA's half of the token tile hold any row below M?
+        // If not, it loads nothing (no copy box lies wholly outside X) and
+        // the even CTA expects only its own bytes; the MMA then reads stale
+        // shared memory for token columns that are never stored.
+        bool odd_rows = t0 + HT < M;
+        bool load = even || odd_rows;
+        uint32_t copies = odd_rows ? 2u : 1u;
+        int row = t0 + (int)rank * HT;
+        for (int g = 0; g < G; ++g) {
+          if (!mbar_wait_bounded(&bar->xempty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
+            record_timeout(err, bar);
+            break;
+          }
+          const int k0 = kb * BK;
           // the second 64-k half holds k below K (else it is neither loaded
           // nor multiplied)
           const bool hi = k0 + 64 < K;
-          const uint32_t bytes = (x3d || hi) ? L::X_STAGE_BYTES : L::X_HALF_BYTES;
-          if (even) mbar_arrive_expect_tx(&bar->xfull[s], (odd_rows ? 2u : 1u) * bytes);
-          if (even || odd_rows) {
+          if (even)
+            mbar_arrive_expect_tx(&bar->xfull[s],
+                                  copies * ((x3d || hi) ? L::X_STAGE_BYTES : L::X_HALF_BYTES));
+          if (load) {
             uint8_t* dst = xs + s * L::X_STAGE_BYTES;
-            const int row = t0 + (int)rank * HT;
             const uint32_t bar_c = xfull_even + 8u * (uint32_t)s;
             if (x3d) {
               tma_load_3d_pair(dst, &x_map, 0, row, k0 / 64, bar_c);
@@ -256,32 +270,66 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               if (hi) tma_load_2d_pair(dst + L::X_HALF_BYTES, &x_map, k0 + 64, row, bar_c);
             }
           }
-        } else if (n0 < N) {
-          uint8_t* wst = smem + L::W_OFF + s * W_STAGE_BYTES;
-          mbar_arrive_expect_tx(&bar->wfull[s], QW_STAGE_BYTES + scale_rows * S_ROW_BYTES);
-          tma_load_2d(wst, &qw_map, n0, k0 / 8, &bar->wfull[s]);
-          tma_load_2d(wst + QW_STAGE_BYTES, &s_map, n0, (int)((int64_t)k0 >> group_shift),
-                      &bar->wfull[s]);
-        } else {
-          mbar_arrive(&bar->wfull[s]);  // padding CTA: no columns, nothing to load
-        }
-        ++issued;
-        if (++kb == KB) {
-          kb = 0;
-          if (++it < NT) {
-            walk.coords(it, BT, rank, n0, t0);
-            odd_rows = t0 + HT < M;
+          ++issued;
+          if (++s == XS) {
+            s = 0;
+            ph ^= 1u;
+          }
+          if (++kb == KB) {
+            kb = 0;
+            if (++it < NT) {
+              walk.coords(it, BT, rank, n0, t0);
+              odd_rows = t0 + HT < M;
+              load = even || odd_rows;
+              copies = odd_rows ? 2u : 1u;
+              row = t0 + (int)rank * HT;
+            }
           }
         }
-      }
-      if (*abort_flag && (!xp || even)) {
-        // drain: wait for the last loads issued into each slot (the odd
-        // CTA's X loads complete on the even CTA's barriers, which the even
-        // CTA drains)
-        int never = 0;
-        for (int j = issued - 1; j >= 0 && j >= issued - depth; --j)
-          mbar_wait_bounded(xp ? &bar->xfull[j % depth] : &bar->wfull[j % depth],
-                            (uint32_t)(j / depth) & 1u, &never, kDrainLimitNs);
+        if (*abort_flag && even) {
+          // drain: wait for the last loads issued into each slot (the odd
+          // CTA's X loads complete on the even CTA's barriers, which the
+          // even CTA drains)
+          int never = 0;
+          for (int j = issued - 1; j >= 0 && j >= issued - XS; --j)
+            mbar_wait_bounded(&bar->xfull[j % XS], (uint32_t)(j / XS) & 1u, &never,
+                              kDrainLimitNs);
+        }
+      } else {
+        const uint32_t wbytes = QW_STAGE_BYTES + scale_rows * S_ROW_BYTES;
+        uint8_t* wst = smem + L::W_OFF;
+        for (int g = 0; g < G; ++g) {
+          if (!mbar_wait_bounded(&bar->wempty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
+            record_timeout(err, bar);
+            break;
+          }
+          if (n0 < N) {
+            const int k0 = kb * BK;
+            mbar_arrive_expect_tx(&bar->wfull[s], wbytes);
+            tma_load_2d(wst, &qw_map, n0, k0 / 8, &bar->wfull[s]);
+            tma_load_2d(wst + QW_STAGE_BYTES, &s_map, n0, (int)((int64_t)k0 >> group_shift),
+                        &bar->wfull[s]);
+          } else {
+            mbar_arrive(&bar->wfull[s]);  // padding CTA: no columns, nothing to load
+          }
+          ++issued;
+          wst += W_STAGE_BYTES;
+          if (++s == WS) {
+            s = 0;
+            ph ^= 1u;
+            wst = smem + L::W_OFF;
+          }
+          if (++kb == KB) {
+            kb = 0;
+            if (++it < NT) walk.coords(it, BT, rank, n0, t0);
+          }
+        }
+        if (*abort_flag) {
+          int never = 0;
+          for (int j = issued - 1; j >= 0 && j >= issued - WS; --j)
+            mbar_wait_bounded(&bar->wfull[j % WS], (uint32_t)(j / WS) & 1u, &never,
+                              kDrainLimitNs);
+        }
       }
     }
     __syncwarp();  // the whole warp reaches the cluster barrier below together
@@ -345,9 +393,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int grp = (warp - DQ_WARP0) >> 2;  // stages g = grp mod DQ_GROUPS
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
     const int col = 32 * quarter + lane;     // this thread's column in the tile
-    const int j = grp;                       // this group's weight slot and A slot
-    const uint8_t* qw = smem + L::W_OFF + j * W_STAGE_BYTES + col * 4;
-    const uint8_t* sc = smem + L::W_OFF + j * W_STAGE_BYTES + QW_STAGE_BYTES + col * 2;
+    const int j = grp;                       // this group's A slot
+    // this thread's column in weight slot 0 (slot jw adds jw * W_STAGE_BYTES)
+    const uint8_t* qw0 = smem + L::W_OFF + col * 4;
+    const uint8_t* sc0 = smem + L::W_OFF + QW_STAGE_BYTES + col * 2;
     uint8_t* ystage = smem + L::Y_OFF + grp * L::Y_GROUP_BYTES + quarter * L::Y_WARP_BYTES;
 
     // Reads out tile d's accumulator (this warp's 32 lanes x its group's TPG
@@ -408,10 +457,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (lane == 0) record_timeout(err, bar);
         break;
       }
-      const uint32_t ph = (uint32_t)(g / DQ_GROUPS) & 1u;
+      const uint32_t ph = (uint32_t)(g / DQ_GROUPS) & 1u;  // A slot phase
+      const int jw = g % WS;                                // weight slot
+      const uint32_t pw = (uint32_t)(g / WS) & 1u;
+      const uint8_t* qw = qw0 + jw * W_STAGE_BYTES;
+      const uint8_t* sc = sc0 + jw * W_STAGE_BYTES;
       // qweight and scale tiles of the stage have landed
       ok = __all_sync(0xffffffffu,
-                      mbar_wait_bounded<true>(&bar->wfull[j], ph, abort_flag, kWaitLimitNs));
+                      mbar_wait_bounded<true>(&bar->wfull[jw], pw, abort_flag, kWaitLimitNs));
       if (!ok) {
         if (lane == 0) record_timeout(err, bar);
         break;
@@ -441,7 +494,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           tc_fence_after();
         } else {
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bar->wempty[j]);  // weight tiles of the stage read
+          if (lane == 0) mbar_arrive(&bar->wempty[jw]);  // weight tiles of the stage read
         }
         tmem_st_32x32b_x32(tmem + lane_addr + A_COL + j * A_STAGE_COLS + 32 * h, cells);
       }
