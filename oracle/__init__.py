@@ -10,6 +10,13 @@ and Quickstart", "Defaults and compatibility decisions"):
     q[k,n] = (uint32(qweight[k//8, n]) >> 4*(k%8)) & 0xF
     W[k,n] = fp16_RNE((q[k,n] - 8) * scales[k//G, n])
     Y[m,n] = sum_k x[m,k] * W[k,n]            (binary64, k ascending)
+
+With a LoRA adapter (GPTQ-Pro README, "Runtime contract": adapters on the
+linear path; GPTQModel README, "PEFT LoRA Training and Adapter Loading": the
+adapter stays separate from the packed weights), read with PEFT's layouts and
+the adapter's scaling already in lora_b:
+    T[m,j] = fp16_RNE(sum_k x[m,k] * lora_a[j,k])          lora_a [r, K]
+    Y[m,n] += sum_j T[m,j] * lora_b[n,j]                    lora_b [N, r]
 """
 from __future__ import annotations
 
@@ -67,6 +74,8 @@ def _load():
                                                 _i64, _p, _p, _p]
             lib.oracle_gemm_rows.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32,
                                              _i64, _p, _p]
+            lib.oracle_lora_down.argtypes = [_p, _p, _i64, _i64, _i64, _p]
+            lib.oracle_lora_up_add.argtypes = [_p, _p, _i64, _i64, _i64, _p, _p]
             _lib = lib
     return _lib
 
@@ -198,3 +207,47 @@ def gemm_rows(x, qweight, scales, group, ms) -> np.ndarray:
     _load().oracle_gemm_rows(_ptr(xb), _ptr(qw), _ptr(s), M, K, N, group,
                              ms.size, _ptr(ms), _ptr(out))
     return out
+
+
+def lora_down(x: np.ndarray, lora_a: np.ndarray) -> np.ndarray:
+    """T = fp16(x . lora_a^T) as float16 [M, r] (binary64 sums)."""
+    xb = _bits16(x)
+    a = _bits16(lora_a)
+    M, K = xb.shape
+    r = a.shape[0]
+    if a.shape[1] != K:
+        raise ValueError("x and lora_a disagree on K")
+    t = np.empty((M, r), dtype=np.uint16)
+    _load().oracle_lora_down(_ptr(xb), _ptr(a), M, K, r, _ptr(t))
+    return t.view(np.float16)
+
+
+def lora_up_add(t: np.ndarray, lora_b: np.ndarray, y: np.ndarray, ms=None) -> np.ndarray:
+    """y[i, :] += t[ms[i], :] . lora_b^T in binary64 (ms = all rows by default)."""
+    tb = _bits16(t)
+    b = _bits16(lora_b)
+    M, r = tb.shape
+    N = b.shape[0]
+    if b.shape[1] != r:
+        raise ValueError("t and lora_b disagree on the rank")
+    ms = np.arange(M, dtype=np.int64) if ms is None else np.asarray(ms, dtype=np.int64)
+    ms = _c(ms, np.int64)
+    if ms.size and (ms.min() < 0 or ms.max() >= M):
+        raise IndexError("row index out of range")
+    out = _c(np.asarray(y, dtype=np.float64), np.float64)
+    if out.shape != (ms.size, N):
+        raise ValueError("y has the wrong shape")
+    _load().oracle_lora_up_add(_ptr(tb), _ptr(b), r, N, ms.size, _ptr(ms), _ptr(out))
+    return out
+
+
+def gemm_lora(x, qweight, scales, group, lora_a, lora_b) -> np.ndarray:
+    """Y = x . W + fp16(x . lora_a^T) . lora_b^T in binary64, float64 [M, N]."""
+    return lora_up_add(lora_down(x, lora_a), lora_b, gemm(x, qweight, scales, group))
+
+
+def gemm_lora_rows(x, qweight, scales, group, lora_a, lora_b, ms) -> np.ndarray:
+    """Rows ms of gemm_lora, for problems too large to compute whole."""
+    ms = np.asarray(ms, dtype=np.int64)
+    xs = np.ascontiguousarray(np.asarray(x)[ms])
+    return lora_up_add(lora_down(xs, lora_a), lora_b, gemm_rows(x, qweight, scales, group, ms))

@@ -233,3 +233,42 @@ void oracle_gemm_rows(const uint16_t* x, const int32_t* qweight,
         }
     }
 }
+
+/* ---- LoRA adapter on the linear path ------------------------------------
+ *
+ * GPTQ-Pro README, "Runtime contract" (adapters: LoRA on the GPTQ-Pro linear
+ * path) and GPTQModel README, "PEFT LoRA Training and Adapter Loading" (the
+ * adapter stays separate from the packed weights).  Read as the usual LoRA
+ * delta with PEFT's layouts and the adapter's scaling already in lora_b:
+ *     T[m,j] = fp16_RNE( sum_k x[m,k] * lora_a[j,k] )      lora_a [r, K]
+ *     Y[m,n] = sum_k x[m,k] * W[k,n] + sum_j T[m,j] * lora_b[n,j]   lora_b [N, r]
+ * T is rounded to FP16 (the adapter's dtype); Y is the binary64 sum.
+ */
+
+/* t (FP16 bits) [M, r] = fp16(x . lora_a^T), binary64 sums, k ascending. */
+void oracle_lora_down(const uint16_t* x, const uint16_t* lora_a, int64_t M, int64_t K,
+                      int64_t r, uint16_t* t)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t j = 0; j < r; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += oracle_half_to_double(x[m * K + k]) * oracle_half_to_double(lora_a[j * K + k]);
+            t[m * r + j] = oracle_double_to_half(acc);
+        }
+}
+
+/* y [count, N] (binary64) += t[ms[i], :] . lora_b^T, j ascending. */
+void oracle_lora_up_add(const uint16_t* t, const uint16_t* lora_b, int64_t r, int64_t N,
+                        int64_t count, const int64_t* ms, double* y)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; ++i)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < r; ++j)
+                acc += oracle_half_to_double(t[ms[i] * r + j]) * oracle_half_to_double(lora_b[n * r + j]);
+            y[i * N + n] += acc;
+        }
+}

@@ -242,3 +242,87 @@ def test_validation_errors():
     with pytest.raises(IndexError):
         oracle.gemm_entries(np.zeros((1, 16), np.float16), qw, np.zeros((1, 8), np.float16),
                             -1, [1], [0])
+
+
+# ---- LoRA adapter ----------------------------------------------------------
+
+def _lora_problem(M, K, N, r, seed, G=32):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    qw = oracle.pack(rng.integers(0, 16, size=(K, N)).astype(np.uint8))
+    s = rng.uniform(1e-3, 2e-2, size=(oracle.num_groups(K, G), N)).astype(np.float16)
+    a = (rng.standard_normal((r, K)) * 0.05).astype(np.float16)
+    b = (rng.standard_normal((N, r)) * 0.05).astype(np.float16)
+    return x, qw, s, G, a, b
+
+
+def test_lora_down_integer_inputs_match_numpy_bitwise():
+    """Integer inputs: every product and sum is exact, so any summation order
+    gives the same binary64 value and the FP16 rounding must agree."""
+    rng = np.random.default_rng(1)
+    x = rng.integers(-8, 9, size=(5, 64)).astype(np.float16)
+    a = rng.integers(-8, 9, size=(16, 64)).astype(np.float16)
+    ref = (x.astype(np.float64) @ a.astype(np.float64).T).astype(np.float16)
+    assert np.array_equal(oracle.lora_down(x, a).view(np.uint16), ref.view(np.uint16))
+
+
+def test_lora_down_random_within_one_ulp_of_numpy():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((7, 96)).astype(np.float16)
+    a = rng.standard_normal((32, 96)).astype(np.float16)
+    ours = oracle.lora_down(x, a).astype(np.float64)
+    ref = (x.astype(np.float64) @ a.astype(np.float64).T)
+    ulp = np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64)
+    assert np.all(np.abs(ours - ref) <= ulp)
+
+
+@pytest.mark.parametrize("M,K,N,r", [(1, 16, 8, 16), (3, 48, 24, 16), (4, 64, 40, 32)])
+def test_gemm_lora_against_numpy_einsum(M, K, N, r):
+    x, qw, s, G, a, b = _lora_problem(M, K, N, r, seed=M + K)
+    t = (x.astype(np.float64) @ a.astype(np.float64).T).astype(np.float16)
+    w = oracle.dequant(qw, s, G).astype(np.float64)
+    ref = np.einsum("mk,kn->mn", x.astype(np.float64), w) + \
+        np.einsum("mj,nj->mn", t.astype(np.float64), b.astype(np.float64))
+    ours = oracle.gemm_lora(x, qw, s, G, a, b)
+    assert np.allclose(ours, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_lora_zero_up_projection_leaves_the_layer_unchanged():
+    x, qw, s, G, a, b = _lora_problem(3, 64, 16, 16, seed=3)
+    b[:] = 0
+    assert np.array_equal(oracle.gemm_lora(x, qw, s, G, a, b), oracle.gemm(x, qw, s, G))
+
+
+def test_lora_one_hot_down_copies_x_columns():
+    """lora_a rows one-hot at k_j: T[:, j] is exactly x[:, k_j]."""
+    x, qw, s, G, a, b = _lora_problem(4, 64, 16, 16, seed=4)
+    ks = np.random.default_rng(4).integers(0, 64, size=16)
+    a[:] = 0
+    a[np.arange(16), ks] = 1
+    t = oracle.lora_down(x, a)
+    assert np.array_equal(t.view(np.uint16), x[:, ks].view(np.uint16))
+
+
+def test_lora_one_hot_up_adds_one_t_column():
+    """lora_b rows one-hot at j_n: Y_lora - Y is exactly T[:, j_n]."""
+    x, qw, s, G, a, b = _lora_problem(4, 64, 24, 16, seed=5)
+    js = np.random.default_rng(5).integers(0, 16, size=24)
+    b[:] = 0
+    b[np.arange(24), js] = 1
+    t = oracle.lora_down(x, a).astype(np.float64)
+    delta = oracle.gemm_lora(x, qw, s, G, a, b) - oracle.gemm(x, qw, s, G)
+    assert np.array_equal(delta, t[:, js])
+
+
+def test_lora_rank_one_is_an_outer_product():
+    x, qw, s, G, a, b = _lora_problem(5, 32, 16, 1, seed=6)
+    t = oracle.lora_down(x, a).astype(np.float64)
+    delta = oracle.gemm_lora(x, qw, s, G, a, b) - oracle.gemm(x, qw, s, G)
+    assert np.allclose(delta, np.outer(t[:, 0], b[:, 0].astype(np.float64)), rtol=0, atol=1e-12)
+
+
+def test_gemm_lora_rows_match_the_whole_result():
+    x, qw, s, G, a, b = _lora_problem(6, 64, 16, 16, seed=7)
+    full = oracle.gemm_lora(x, qw, s, G, a, b)
+    rows = oracle.gemm_lora_rows(x, qw, s, G, a, b, [5, 0, 3])
+    assert np.array_equal(rows, full[[5, 0, 3]])
