@@ -70,6 +70,7 @@ typedef enum {
 #define GPTQ_MAX_M 8388608
 #define GPTQ_DECODE_MAX_M 32
 #define GPTQ_MAX_GROUPED 8     /* linears per gptq_w4a16_gemm_grouped call */
+#define GPTQ_MAX_LORA_RANK 256 /* largest adapter rank of gptq_w4a16_gemm_lora */
 
 /*
  * Y = X . dequant(qweight, scales).
@@ -134,6 +135,34 @@ GPTQ_API int gptq_w4a16_gemm_grouped(const uint16_t* x, const int32_t* const* qw
                                      const uint16_t* const* scales, const int64_t* Ns,
                                      int32_t count, int64_t M, int64_t K, int32_t group,
                                      uint16_t* const* ys, void* stream);
+
+/*
+ * The layer with a LoRA adapter on its path:
+ *   T = fp16(X . lora_a^T)                       [M, rank]
+ *   Y = fp16(X . dequant(qweight, scales) + T . lora_b^T)
+ * The GPTQ-Pro README ("Runtime contract") puts LoRA adapters on the linear
+ * path; the GPTQModel README ("PEFT LoRA Training and Adapter Loading") keeps
+ * the adapter separate from the packed weights.  Read with PEFT's layouts:
+ *   lora_a   [rank, K] FP16 bits, device (lora_A.weight)
+ *   lora_b   [N, rank] FP16 bits, device (lora_B.weight), with the adapter's
+ *            scaling (alpha / rank) already multiplied in
+ *   rank     16 .. GPTQ_MAX_LORA_RANK, a multiple of 16
+ *   t_work   [M, rank] FP16 bits, device, caller-owned: receives T (the
+ *            adapter's down-projection, rounded to FP16 like the adapter's
+ *            own output); must not overlap any other argument
+ * T is summed in FP32 and rounded to FP16; T . lora_b^T is added to the
+ * layer's FP32 accumulator (the adapter's rank is extra K of the same
+ * tensor-core product) and Y is rounded once.  Two launches on `stream`: T,
+ * then the layer; every M runs on the prefill path.  Other arguments, checks
+ * and errors as gptq_w4a16_gemm, plus GPTQ_ERR_NULL for a NULL lora_a, lora_b
+ * or t_work (when M > 0), GPTQ_ERR_SHAPE for a rank out of range, and
+ * GPTQ_ERR_ALIAS when t_work or y overlaps any other buffer.
+ */
+GPTQ_API int gptq_w4a16_gemm_lora(const uint16_t* x, const int32_t* qweight,
+                                  const uint16_t* scales, int64_t M, int64_t K, int64_t N,
+                                  int32_t group, const uint16_t* lora_a,
+                                  const uint16_t* lora_b, int64_t rank, uint16_t* t_work,
+                                  uint16_t* y, void* stream);
 
 /*
  * W[K, N] = dequant(qweight, scales) as FP16 bits, each value rounded once from

@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libgptq_w4a16.so")
 KERNEL_AUTO, KERNEL_DECODE, KERNEL_PREFILL = 0, 1, 2
 DECODE_MAX_M = 32
 MAX_GROUPED = 8
+MAX_LORA_RANK = 256
 GROUP_SIZES = (-1, 16, 32, 64, 128, 256, 512, 1024)
 
 STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_NULL", 2: "GPTQ_ERR_SHAPE", 3: "GPTQ_ERR_GROUP",
@@ -28,8 +29,8 @@ STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_NULL", 2: "GPTQ_ERR_SHAPE", 3: "GPTQ_ERR_GR
 
 # Every entry point declared in include/gptq_w4a16.h.
 EXPORTS = ("gptq_w4a16_gemm", "gptq_w4a16_gemm_kernel", "gptq_w4a16_gemm_decode_splits",
-           "gptq_w4a16_gemm_grouped", "gptq_dequant", "gptq_w4a16_select", "gptq_status_string", "gptq_device_error",
-           "gptq_version")
+           "gptq_w4a16_gemm_grouped", "gptq_w4a16_gemm_lora", "gptq_dequant",
+           "gptq_w4a16_select", "gptq_status_string", "gptq_device_error", "gptq_version")
 
 
 class GptqError(RuntimeError):
@@ -62,6 +63,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.gptq_w4a16_gemm_decode_splits.argtypes = gemm_args + [_i32]
             lib.gptq_w4a16_gemm_grouped.argtypes = [_p, _p, _p, _p, _i32, _i64, _i64, _i32,
                                                     _p, _p]
+            lib.gptq_w4a16_gemm_lora.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32, _p, _p,
+                                                 _i64, _p, _p, _p]
             lib.gptq_dequant.argtypes = [_p, _p, _i64, _i64, _i32, _p, _p]
             lib.gptq_w4a16_select.argtypes = [_i64, _i64, _i64, _i32,
                                               ctypes.POINTER(_i32), ctypes.POINTER(_i32)]
@@ -71,7 +74,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.gptq_version.restype = ctypes.c_char_p
             for name in ("gptq_w4a16_gemm", "gptq_w4a16_gemm_kernel",
                          "gptq_w4a16_gemm_decode_splits", "gptq_w4a16_gemm_grouped",
-                         "gptq_dequant",
+                         "gptq_w4a16_gemm_lora", "gptq_dequant",
                          "gptq_w4a16_select", "gptq_device_error"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
@@ -188,6 +191,46 @@ def gemm_grouped(x: torch.Tensor, qweights, scales, group: int, outs=None,
     _check(lib.gptq_w4a16_gemm_grouped(_ptr(x), qa, sa, na, count, M, K, group, ya,
                                        _stream_handle(stream, dev)))
     return outs
+
+
+def gemm_lora(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, group: int,
+              lora_a: torch.Tensor, lora_b: torch.Tensor, t_work: torch.Tensor | None = None,
+              out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y = x . dequant(qweight, scales) + fp16(x . lora_a^T) . lora_b^T (FP16),
+    lora_a [rank, K], lora_b [N, rank] with the adapter's scaling applied;
+    t_work [M, rank] receives fp16(x . lora_a^T)."""
+    lib = load()
+    dev = qweight.device
+    _require(qweight, "qweight", lambda d: d == torch.int32, None)
+    _require(scales, "scales", lambda d: d == torch.float16, dev)
+    _require(x, "x", lambda d: d == torch.float16, dev)
+    _require(lora_a, "lora_a", lambda d: d == torch.float16, dev)
+    _require(lora_b, "lora_b", lambda d: d == torch.float16, dev)
+    if x.dim() != 2 or lora_a.dim() != 2 or lora_b.dim() != 2:
+        raise ValueError("x, lora_a and lora_b must be 2-D")
+    M, K = x.shape
+    N = qweight.shape[1]
+    rank = lora_a.shape[0]
+    if qweight.shape[0] * 8 != K or lora_a.shape[1] != K:
+        raise ValueError(f"qweight or lora_a do not match K={K}")
+    if tuple(lora_b.shape) != (N, rank):
+        raise ValueError(f"lora_b has shape {tuple(lora_b.shape)}, expected {(N, rank)}")
+    if t_work is None:
+        t_work = torch.empty((M, rank), dtype=torch.float16, device=dev)
+    else:
+        _require(t_work, "t_work", lambda d: d == torch.float16, dev)
+        if tuple(t_work.shape) != (M, rank):
+            raise ValueError(f"t_work has shape {tuple(t_work.shape)}, expected {(M, rank)}")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=dev)
+    else:
+        _require(out, "out", lambda d: d == torch.float16, dev)
+        if tuple(out.shape) != (M, N):
+            raise ValueError(f"out has shape {tuple(out.shape)}, expected {(M, N)}")
+    _check(lib.gptq_w4a16_gemm_lora(_ptr(x), _ptr(qweight), _ptr(scales), M, K, N, group,
+                                    _ptr(lora_a), _ptr(lora_b), rank, _ptr(t_work), _ptr(out),
+                                    _stream_handle(stream, dev)))
+    return out
 
 
 def dequant(qweight: torch.Tensor, scales: torch.Tensor, group: int,

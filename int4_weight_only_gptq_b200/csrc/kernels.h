@@ -55,5 +55,16 @@ cudaError_t launch_prefill_pair(const uint16_t* x, const int32_t* qweight,
                                 const uint16_t* scales, uint16_t* y, int64_t M, int64_t K,
                                 int64_t N, int group_shift, cudaStream_t stream,
                                 const DeviceInfo& dev);
+// The same with a LoRA adapter: t = fp16(x . lora_a^T) [M, rank] (from
+// launch_lora_down), lora_b [N, rank]; T . lora_b^T is added to the
+// accumulator as rank/32 extra stages per tile.
+cudaError_t launch_prefill_pair_lora(const uint16_t* x, const int32_t* qweight,
+                                     const uint16_t* scales, uint16_t* y, int64_t M, int64_t K,
+                                     int64_t N, int group_shift, const uint16_t* t,
+                                     const uint16_t* lora_b, int64_t rank, cudaStream_t stream,
+                                     const DeviceInfo& dev);
+// t [M, r] = fp16(x . lora_a^T), lora_a [r, K] (the adapter's down-projection).
+cudaError_t launch_lora_down(const uint16_t* x, const uint16_t* lora_a, uint16_t* t, int64_t M,
+                             int64_t K, int64_t r, cudaStream_t stream, const DeviceInfo& dev);
 
 }  // namespace gptq

@@ -35,6 +35,13 @@
 // dequantisation and MMAs overlap the previous tile's epilogue, and no CTA
 // launch, TMEM allocation or pipeline fill is paid per tile.
 //
+// With a LoRA adapter (GPTQ-Pro README, "Runtime contract": adapters on the
+// linear path) each tile gets rank/32 more stages after its K stages: the
+// weight producer loads 32 columns of lora_b (FP16, copied into the TMEM A
+// slot as they are), the X producer loads the same 32 columns of T =
+// fp16(X . lora_a^T), and the MMAs add T . lora_b^T into the same FP32
+// accumulator, so Y is rounded once.
+//
 // Every wait is bounded in time; on expiry the CTA records GPTQ_ERR_TIMEOUT
 // in the device error word and winds down.  Both CTAs always reach the final
 // cluster barrier, so neither leaves while the other may still signal it.
@@ -67,6 +74,12 @@ constexpr int QW_STAGE_BYTES = BW * (BK / 8) * 4;  // 128 columns x 16 packed ro
 constexpr int S_ROW_BYTES = BW * 2;                // one scale row of the tile: 256 B
 constexpr int S_STAGE_MAX_ROWS = BK / 16;          // group 16: eight rows per stage
 constexpr int W_STAGE_BYTES = QW_STAGE_BYTES + S_STAGE_MAX_ROWS * S_ROW_BYTES;
+// A LoRA stage: 32 of the adapter's rank.  Its weight tile is lora_b's 128
+// rows x 32 FP16 (64-byte rows, no swizzle); its token tile is T's rows x 64
+// columns (128-byte swizzle; the 32 columns past the stage are not used).
+constexpr int LORA_R = 32;
+constexpr int LORA_W_BYTES = BW * LORA_R * 2;
+static_assert(LORA_W_BYTES <= W_STAGE_BYTES, "a LoRA weight tile fits a weight slot");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t D_COL = 0;              // accumulator: columns [0, BT)
 constexpr uint32_t A_COL = 256;            // A slots: [256, 256 + 4 * 64)
@@ -157,14 +170,18 @@ struct TileWalk {
 // multiple of 64); otherwise through [M][K], one copy per 64-k half.
 // n_pairs, tiles: column pairs (of 256) and pair tiles (n_pairs x token
 // tiles); cluster c takes tiles c, c + clusters, ...
+// lora_stages: LoRA stages per tile (0 without an adapter); t_map and b_map
+// then describe T [M, rank] and lora_b [N, rank].
 template <int BT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap x_map,
                         const __grid_constant__ CUtensorMap qw_map,
                         const __grid_constant__ CUtensorMap s_map,
-                        const __grid_constant__ CUtensorMap y_map, int M, int K, int N,
+                        const __grid_constant__ CUtensorMap y_map,
+                        const __grid_constant__ CUtensorMap t_map,
+                        const __grid_constant__ CUtensorMap b_map, int M, int K, int N,
                         int group_shift, int scale_rows, int x3d, int n_pairs, int tiles,
-                        int* err) {
+                        int lora_stages, int* err) {
   static_assert(BT == 128 || BT == 256, "pair token tile");
   using L = PairLayout<BT>;
   constexpr int HT = L::HT;
@@ -184,7 +201,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const bool even = rank == 0;
   const TileWalk walk{(int)(blockIdx.x >> 1), (int)(gridDim.x >> 1), n_pairs, tiles};
   const int NT = walk.count();          // tiles of this cluster
-  const int KB = (K + BK - 1) / BK;     // stages per tile
+  const int KW = (K + BK - 1) / BK;     // weight stages per tile
+  const int KB = KW + lora_stages;      // stages per tile (weights, then LoRA)
   const int G = NT * KB;                // stages of this cluster, over all its tiles
 
   if (threadIdx.x == 0) {
@@ -210,6 +228,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     prefetch_tensormap(&qw_map);
     prefetch_tensormap(&s_map);
     prefetch_tensormap(&y_map);
+    if (lora_stages > 0) {
+      prefetch_tensormap(&t_map);
+      prefetch_tensormap(&b_map);
+    }
   }
   __syncwarp();
   if (warp == 1) {
@@ -253,22 +275,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             record_timeout(err, bar);
             break;
           }
-          const int k0 = kb * BK;
-          // the second 64-k half holds k below K (else it is neither loaded
-          // nor multiplied)
-          const bool hi = k0 + 64 < K;
-          if (even)
-            mbar_arrive_expect_tx(&bar->xfull[s],
-                                  copies * ((x3d || hi) ? L::X_STAGE_BYTES : L::X_HALF_BYTES));
-          if (load) {
-            uint8_t* dst = xs + s * L::X_STAGE_BYTES;
-            const uint32_t bar_c = xfull_even + 8u * (uint32_t)s;
-            if (x3d) {
-              tma_load_3d_pair(dst, &x_map, 0, row, k0 / 64, bar_c);
-            } else {
-              tma_load_2d_pair(dst, &x_map, k0, row, bar_c);
-              if (hi) tma_load_2d_pair(dst + L::X_HALF_BYTES, &x_map, k0 + 64, row, bar_c);
+          uint8_t* dst = xs + s * L::X_STAGE_BYTES;
+          const uint32_t bar_c = xfull_even + 8u * (uint32_t)s;
+          if (kb < KW) {
+            const int k0 = kb * BK;
+            // the second 64-k half holds k below K (else it is neither loaded
+            // nor multiplied)
+            const bool hi = k0 + 64 < K;
+            if (even)
+              mbar_arrive_expect_tx(&bar->xfull[s],
+                                    copies * ((x3d || hi) ? L::X_STAGE_BYTES : L::X_HALF_BYTES));
+            if (load) {
+              if (x3d) {
+                tma_load_3d_pair(dst, &x_map, 0, row, k0 / 64, bar_c);
+              } else {
+                tma_load_2d_pair(dst, &x_map, k0, row, bar_c);
+                if (hi) tma_load_2d_pair(dst + L::X_HALF_BYTES, &x_map, k0 + 64, row, bar_c);
+              }
             }
+          } else {
+            // LoRA stage: 64 columns of T from column 32 * (kb - KW)
+            if (even) mbar_arrive_expect_tx(&bar->xfull[s], copies * L::X_HALF_BYTES);
+            if (load) tma_load_2d_pair(dst, &t_map, LORA_R * (kb - KW), row, bar_c);
           }
           ++issued;
           if (++s == XS) {
@@ -303,12 +331,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             record_timeout(err, bar);
             break;
           }
-          if (n0 < N) {
+          if (n0 < N && kb < KW) {
             const int k0 = kb * BK;
             mbar_arrive_expect_tx(&bar->wfull[s], wbytes);
             tma_load_2d(wst, &qw_map, n0, k0 / 8, &bar->wfull[s]);
             tma_load_2d(wst + QW_STAGE_BYTES, &s_map, n0, (int)((int64_t)k0 >> group_shift),
                         &bar->wfull[s]);
+          } else if (n0 < N) {
+            // LoRA stage: lora_b rows n0.. , columns 32 * (kb - KW) ..
+            mbar_arrive_expect_tx(&bar->wfull[s], LORA_W_BYTES);
+            tma_load_2d(wst, &b_map, LORA_R * (kb - KW), n0, &bar->wfull[s]);
           } else {
             mbar_arrive(&bar->wfull[s]);  // padding CTA: no columns, nothing to load
           }
@@ -359,7 +391,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           tc_fence_after();
           const uint64_t b_desc0 = smem_desc_sw128(smem_u32(xs + s * L::X_STAGE_BYTES));
           const uint32_t a_base = tmem + A_COL + a * A_STAGE_COLS;
-          const int nk = kb * BK + 64 < K ? BK / 16 : 4;  // k16 steps holding k below K
+          // k16 steps: those holding k below K, or a LoRA stage's 32 ranks
+          const int nk = kb >= KW ? LORA_R / 16 : (kb * BK + 64 < K ? BK / 16 : 4);
           if (elect_one()) {
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
@@ -469,6 +502,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (lane == 0) record_timeout(err, bar);
         break;
       }
+      if (g - it * KB >= KW) {
+        // LoRA stage: this column's 32 lora_b values, copied as they are
+        // (pairs of ranks per 32-bit cell, as the dequantised weights)
+        const uint4* brow = reinterpret_cast<const uint4*>(smem + L::W_OFF + jw * W_STAGE_BYTES +
+                                                           col * (LORA_R * 2));
+        uint32_t cells[LORA_R / 2];
+#pragma unroll
+        for (int v = 0; v < LORA_R / 8; ++v) {
+          const uint4 q = brow[v];
+          cells[4 * v] = q.x;
+          cells[4 * v + 1] = q.y;
+          cells[4 * v + 2] = q.z;
+          cells[4 * v + 3] = q.w;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->wempty[jw]);
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded<true>(&bar->aempty[j], ph ^ 1u,
+                                                             abort_flag, kWaitLimitNs));
+        if (!ok) {
+          if (lane == 0) record_timeout(err, bar);
+          break;
+        }
+        tc_fence_after();
+        tmem_st_32x32b_x16(tmem + lane_addr + A_COL + j * A_STAGE_COLS, cells);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(afull_even + 8u * (uint32_t)j);
+        continue;
+      }
       // the stage's 16 packed rows, one 64-k half (32 TMEM columns) at a time
       uint32_t cells[32];
 #pragma unroll
@@ -531,10 +594,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 template <int BT>
 cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                           uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
-                          int scale_rows, int64_t n_groups, cudaStream_t stream,
+                          int scale_rows, int64_t n_groups, const uint16_t* t,
+                          const uint16_t* lora_b, int64_t rank, cudaStream_t stream,
                           const DeviceInfo& dev) {
   using L = PairLayout<BT>;
-  CUtensorMap x_map, qw_map, s_map, y_map;
+  CUtensorMap x_map, qw_map, s_map, y_map, t_map, b_map;
   // X as [K/64][M][64] (one copy of both 64-k halves per stage) when K is a
   // multiple of 64, else as [M][K] (one copy per half); rows at or beyond M
   // and k at or beyond K read as zero either way
@@ -558,6 +622,20 @@ cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint1
       !tensor_map_2d(&y_map, y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)N, (uint64_t)M,
                      (uint64_t)N * 2, 32, L::TPG, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
+  int lora_stages = 0;
+  if (rank > 0) {
+    // T [M, rank]: 64 columns x BT/2 rows per copy (128-byte swizzle, the
+    // B operand); lora_b [N, rank]: 32 columns x 128 rows (plain rows)
+    if (!tensor_map_2d(&t_map, t, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)rank, (uint64_t)M,
+                       (uint64_t)rank * 2, 64, L::HT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !tensor_map_2d(&b_map, lora_b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)rank,
+                       (uint64_t)N, (uint64_t)rank * 2, LORA_R, BW, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    lora_stages = (int)((rank + LORA_R - 1) / LORA_R);
+  } else {
+    t_map = x_map;  // not read without an adapter
+    b_map = qw_map;
+  }
   constexpr size_t smem = L::kSmemBytes;
   static std::once_flag attr_once[64];
   static cudaError_t attr_err[64];
@@ -573,25 +651,34 @@ cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint1
   const int64_t tiles = n_pairs * ((M + BT - 1) / BT);
   const int64_t clusters = std::min<int64_t>(tiles, std::max(1, dev.num_sms / 2));
   prefill_pair_kernel<BT><<<dim3((unsigned)(2 * clusters)), THREADS, smem, stream>>>(
-      x_map, qw_map, s_map, y_map, (int)M, (int)K, (int)N, group_shift, scale_rows, x3d,
-      (int)n_pairs, (int)tiles, dev.error_word);
+      x_map, qw_map, s_map, y_map, t_map, b_map, (int)M, (int)K, (int)N, group_shift, scale_rows,
+      x3d, (int)n_pairs, (int)tiles, lora_stages, dev.error_word);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_prefill_pair(const uint16_t* x, const int32_t* qweight,
-                                const uint16_t* scales, uint16_t* y, int64_t M, int64_t K,
-                                int64_t N, int group_shift, cudaStream_t stream,
-                                const DeviceInfo& dev) {
+cudaError_t launch_prefill_pair_lora(const uint16_t* x, const int32_t* qweight,
+                                     const uint16_t* scales, uint16_t* y, int64_t M, int64_t K,
+                                     int64_t N, int group_shift, const uint16_t* t,
+                                     const uint16_t* lora_b, int64_t rank, cudaStream_t stream,
+                                     const DeviceInfo& dev) {
   const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
                                ? 1 : (K + (int64_t(1) << group_shift) - 1) >> group_shift;
   const int scale_rows = group_shift >= 7 ? 1 : (BK >> group_shift);
   if (M <= 128)
     return launch_pair_t<128>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups,
-                              stream, dev);
-  return launch_pair_t<256>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups,
-                            stream, dev);
+                              t, lora_b, rank, stream, dev);
+  return launch_pair_t<256>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups, t,
+                            lora_b, rank, stream, dev);
+}
+
+cudaError_t launch_prefill_pair(const uint16_t* x, const int32_t* qweight,
+                                const uint16_t* scales, uint16_t* y, int64_t M, int64_t K,
+                                int64_t N, int group_shift, cudaStream_t stream,
+                                const DeviceInfo& dev) {
+  return launch_prefill_pair_lora(x, qweight, scales, y, M, K, N, group_shift, nullptr, nullptr,
+                                  0, stream, dev);
 }
 
 }  // namespace gptq

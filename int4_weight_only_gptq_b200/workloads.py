@@ -97,6 +97,35 @@ def make_problem(M: int, K: int, N: int, group: int, *, seed: int = 0,
                    scales=scales)
 
 
+@dataclasses.dataclass
+class Adapter:
+    """A LoRA adapter for a K -> N linear (PEFT's layouts)."""
+    rank: int
+    lora_a: np.ndarray   # float16 [rank, K]
+    lora_b: np.ndarray   # float16 [N, rank], the adapter's scaling applied
+
+    def extra_bytes(self, M: int) -> int:
+        """Bytes the adapter adds to the layer: lora_a, lora_b, and T [M, rank]
+        written once and read once."""
+        return self.lora_a.size * 2 + self.lora_b.size * 2 + 2 * M * self.rank * 2
+
+    def extra_flops(self, M: int) -> int:
+        K, N = self.lora_a.shape[1], self.lora_b.shape[0]
+        return 2 * M * K * self.rank + 2 * M * self.rank * N
+
+
+def make_adapter(K: int, N: int, rank: int, *, seed: int = 0, b_std: float = 0.05) -> Adapter:
+    """Draw one seeded adapter: lora_a ~ N(0, 1/K) (so that T = x . lora_a^T
+    has unit variance for unit-variance x) and lora_b ~ N(0, b_std^2), both
+    drawn in float64 and rounded to float16.  The pages give no adapter
+    statistics; these keep the adapter's term a tenth or so of the layer's.
+    Its own stream: PCG64 seeded with (seed, 1), lora_a drawn before lora_b."""
+    rng = np.random.Generator(np.random.PCG64([seed, 1]))
+    a = rng.standard_normal(size=(rank, K)) / math.sqrt(K)
+    b = rng.standard_normal(size=(N, rank)) * b_std
+    return Adapter(rank=rank, lora_a=a.astype(np.float16), lora_b=b.astype(np.float16))
+
+
 # The five synthetic workloads, restated from their prose descriptions.
 def tiny(M: int = 1, seed: int = 0) -> Problem:
     """W4A16 GEMM, M in {1, 4}, K=512, N=256, group=128, scales U[1e-3, 2e-2]."""

@@ -157,3 +157,44 @@ def test_grouped_empty_m_and_no_device(lib):
     assert call_grouped(lib, M=0, x=0, ys=(0, 0)) == 0
     if not torch.cuda.is_available():
         assert call_grouped(lib) == 5
+
+
+# ---- gptq_w4a16_gemm_lora: host-side checks ----------------------------------
+# Fake device addresses: lora_a [32, 512] (32 KB), lora_b [256, 32] (16 KB),
+# t_work [4, 32] (256 B); disjoint from the ones above.
+
+LA, LB, TW = 0x1800000, 0x1C00000, 0x2000000
+
+
+def call_lora(lib, x=X, qw=QW, s=S, M=4, K=512, N=256, g=128, a=LA, b=LB, rank=32, t=TW,
+              y=Y):
+    v = ctypes.c_void_p
+    return lib.gptq_w4a16_gemm_lora(v(x), v(qw), v(s), M, K, N, g, v(a), v(b), rank, v(t), v(y),
+                                    None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(rank=0), 2), (dict(rank=8), 2), (dict(rank=40), 2), (dict(rank=272), 2),
+    (dict(K=520), 2), (dict(N=252), 2), (dict(g=100), 3),
+    (dict(a=0), 1), (dict(b=0), 1), (dict(qw=0), 1), (dict(t=0), 1), (dict(x=0), 1),
+    (dict(y=0), 1),
+    (dict(a=LA + 2), 4), (dict(b=LB + 8), 4), (dict(t=TW + 2), 4), (dict(x=X + 2), 4),
+    (dict(t=X), 8),            # T would overwrite x
+    (dict(t=LA + 64), 8),      # T would overwrite lora_a
+    (dict(t=LB), 8),           # T would overwrite lora_b
+    (dict(y=TW), 8),           # Y would overwrite T
+    (dict(y=LB), 8),           # Y would overwrite lora_b
+    (dict(t=QW + 16), 8),
+])
+def test_lora_argument_checks(lib, kw, status):
+    assert call_lora(lib, **kw) == status
+
+
+def test_lora_empty_m_and_no_device(lib):
+    import torch
+    assert call_lora(lib, M=0, x=0, t=0, y=0) == 0
+    # the adapter and rank are still checked when M == 0
+    assert call_lora(lib, M=0, x=0, t=0, y=0, rank=24) == 2
+    assert call_lora(lib, M=0, x=0, t=0, y=0, a=0) == 1
+    if not torch.cuda.is_available():
+        assert call_lora(lib) == 5

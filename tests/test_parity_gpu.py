@@ -367,3 +367,125 @@ def test_grouped_qkv_full_size():
     ys = run_grouped(ps)
     for i, (p, y) in enumerate(zip(ps, ys)):
         check_rows(p, y, [0], f"grouped q/k/v linear {i}")
+
+
+# ---- LoRA adapter on the linear path (gptq_w4a16_gemm_lora) --------------------
+
+def run_lora(p, ad, t_out=False):
+    x, qw, s = dev(p)
+    a = torch.from_numpy(ad.lora_a.view(np.int16)).view(torch.float16).cuda()
+    b = torch.from_numpy(ad.lora_b.view(np.int16)).view(torch.float16).cuda()
+    t = torch.empty((p.M, ad.rank), dtype=torch.float16, device="cuda")
+    y = B.gemm_lora(x, qw, s, p.group, a, b, t_work=t)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    return (y.cpu().numpy(), t.cpu().numpy()) if t_out else y.cpu().numpy()
+
+
+def check_t(t_gpu, x, lora_a):
+    """T on the GPU is an FP32 sum rounded to FP16; the oracle's is a binary64
+    sum rounded to FP16.  They may differ by the FP32 summation error bound
+    (K-1) * 2^-24 * sum_k |x_k a_jk| plus one FP16 ulp of the result."""
+    t_ref = oracle.lora_down(x, lora_a).astype(np.float64)
+    K = x.shape[1]
+    bound = (np.spacing(np.abs(t_ref).astype(np.float16)).astype(np.float64) +
+             (K - 1) * 2.0 ** -24 *
+             (np.abs(x.astype(np.float64)) @ np.abs(lora_a.astype(np.float64)).T))
+    assert np.all(np.abs(t_gpu.astype(np.float64) - t_ref) <= bound), \
+        "T differs from fp16(x . lora_a^T) by more than the FP32 summation bound"
+
+
+@pytest.mark.parametrize("M,K,N,G,r", [
+    (1, 512, 256, 128, 16), (5, 1024, 264, 32, 32), (16, 2048, 136, -1, 64),
+    (33, 528, 136, 128, 48),            # 128-token pair tile, ragged K, rank not a multiple of 32
+    (128, 1040, 392, 16, 128),          # odd number of column tiles (padding CTA)
+    (200, 2048, 392, 64, 64),           # 256-token pair tile, odd CTA's half partly filled
+    (300, 96, 264, 32, 256),            # largest rank, single k stage
+    (2048, 5120, 512, 128, 32),         # several token tiles per cluster
+])
+def test_lora_parity(M, K, N, G, r):
+    p = W.make_problem(M, K, N, G, seed=M + r)
+    ad = W.make_adapter(K, N, r, seed=M + r)
+    y, t = run_lora(p, ad, t_out=True)
+    check_t(t, p.x, ad.lora_a)
+    ref = oracle.gemm_lora(p.x, p.qweight, p.scales, G, ad.lora_a, ad.lora_b)
+    err = rel_err(y, ref)
+    print(f"[parity] lora M={M} K={K} N={N} G={G} r={r}: {err:.3e}")
+    assert np.all(np.isfinite(y))
+    assert err <= TOL
+
+
+@pytest.mark.parametrize("M", [1, 40, 300])
+def test_lora_integer_exact_inputs_bitwise(M):
+    """Integer x and codes, power-of-two scales, sparse +-1 lora_a and lora_b
+    in multiples of 2^-6: T and every product and partial sum are exact, so
+    any summation order must reproduce the oracle's rounding bit for bit."""
+    rng = np.random.default_rng(M)
+    K, N, r = 1024, 264, 32
+    p = W.make_problem(M, K, N, 64, seed=M)
+    p.x[:] = rng.integers(-4, 5, size=p.x.shape).astype(np.float16)
+    p.scales[:] = np.float16(2.0 ** -6)
+    ad = W.make_adapter(K, N, r, seed=M)
+    ad.lora_a[:] = (rng.integers(-1, 2, size=ad.lora_a.shape) *
+                    (rng.random(ad.lora_a.shape) < 1 / 16)).astype(np.float16)
+    ad.lora_b[:] = (rng.integers(-8, 9, size=ad.lora_b.shape) * 2.0 ** -6).astype(np.float16)
+    y, t = run_lora(p, ad, t_out=True)
+    t_ref = oracle.lora_down(p.x, ad.lora_a)
+    assert np.array_equal(t.view(np.uint16), t_ref.view(np.uint16))
+    ref = oracle.round_to_half(oracle.gemm_lora(p.x, p.qweight, p.scales, 64, ad.lora_a,
+                                                ad.lora_b))
+    assert np.array_equal(y.view(np.uint16), ref.view(np.uint16))
+
+
+def test_lora_zero_adapter_equals_the_plain_layer_bitwise():
+    """lora_b = 0 adds exact zeros to the same accumulator: above 32 tokens the
+    plain call runs the same kernel, so Y must be identical."""
+    p = W.make_problem(200, 2048, 392, 128, seed=21)
+    ad = W.make_adapter(2048, 392, 32, seed=21)
+    ad.lora_b[:] = 0
+    assert np.array_equal(run_lora(p, ad).view(np.uint16), run(p).view(np.uint16))
+
+
+def test_lora_one_hot_reproduces_weight_row_plus_t_column_bitwise():
+    """x one-hot at k*, lora_a one-hot at k_j, lora_b one-hot at j_n: Y[m, n]
+    is fp16(W[k*, n] + [k_{j_n} == k*]), with every step exact."""
+    M, K, N, r = 64, 1024, 264, 32
+    p = W.make_problem(M, K, N, 32, seed=8)
+    rng = np.random.default_rng(8)
+    ks = rng.integers(0, K, size=M)
+    p.x[:] = 0
+    p.x[np.arange(M), ks] = 1
+    ad = W.make_adapter(K, N, r, seed=8)
+    kj = rng.integers(0, K, size=r)
+    kj[:8] = ks[:8]                     # some adapter rows hit the rows' own k
+    ad.lora_a[:] = 0
+    ad.lora_a[np.arange(r), kj] = 1
+    jn = rng.integers(0, r, size=N)
+    ad.lora_b[:] = 0
+    ad.lora_b[np.arange(N), jn] = 1
+    y = run_lora(p, ad)
+    w = oracle.dequant(p.qweight, p.scales, 32).astype(np.float64)
+    hit = (kj[jn][None, :] == ks[:, None]).astype(np.float64)
+    ref = oracle.round_to_half(w[ks] + hit)
+    assert np.array_equal(y.view(np.uint16), ref.view(np.uint16))
+
+
+def test_lora_deterministic():
+    p = W.make_problem(16, 5120, 1024, 128, seed=9)
+    ad = W.make_adapter(5120, 1024, 64, seed=9)
+    a, b = run_lora(p, ad), run_lora(p, ad)
+    assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+
+
+@pytest.mark.parametrize("M", [1, 16, 2048])
+def test_lora_up_projection_full_size(M):
+    p = W.prefill(M) if M > 16 else (W.decode_up() if M == 1 else W.make_problem(
+        16, 5120, 17408, 128, seed=0))
+    ad = W.make_adapter(p.K, p.N, 32, seed=M)
+    y = run_lora(p, ad)
+    rows = sorted({0, M // 2, M - 1})
+    ref = oracle.gemm_lora_rows(p.x, p.qweight, p.scales, p.group, ad.lora_a, ad.lora_b, rows)
+    err = rel_err(y[rows], ref)
+    print(f"[parity] lora up-projection M={M}: {err:.3e} over rows {rows}")
+    assert np.all(np.isfinite(y[rows]))
+    assert err <= TOL
