@@ -281,6 +281,35 @@ def time_grouped(lib, torch, ps, steps, warmup, l2_bytes):
     return e0.elapsed_time(e1) / steps
 
 
+def time_lora(lib, torch, p, ad, steps, warmup, l2_bytes):
+    """Device time per call (ms) of back-to-back gptq_w4a16_gemm_lora calls
+    (the adapter's down-projection launch and the layer launch), rotating
+    weight copies past the L2 like time_gemm."""
+    copies = copies_for(p, l2_bytes) if l2_bytes else 1
+    sets = to_device(p, torch, copies)
+    a = torch.from_numpy(ad.lora_a.view(np.int16)).view(torch.float16).cuda()
+    b = torch.from_numpy(ad.lora_b.view(np.int16)).view(torch.float16).cuda()
+    t = torch.empty((p.M, ad.rank), dtype=torch.float16, device="cuda")
+    sh = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    v = ctypes.c_void_p
+    argv = [(v(x.data_ptr()), v(qw.data_ptr()), v(s.data_ptr()), p.M, p.K, p.N, p.group,
+             v(a.data_ptr()), v(b.data_ptr()), ad.rank, v(t.data_ptr()), v(y.data_ptr()), sh)
+            for (x, qw, s, y) in sets]
+    fn = lib.gptq_w4a16_gemm_lora
+    for i in range(warmup):
+        st = fn(*argv[i % copies])
+        if st:
+            raise RuntimeError(f"lora gemm status {st}")
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        fn(*argv[i % copies])
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -446,6 +475,22 @@ def run_sweep(lib, torch, l2, hbm, tf):
             gbs = sum(p.algorithmic_bytes for p in ps) / (ms * 1e-3) / 1e9
             res[f"grouped_{name}_M{M}"] = {"ms": round(ms, 5), "GB/s": round(gbs, 1),
                                            "frac_hbm": round(gbs / hbm, 3)}
+    # LoRA adapter (rank 32) on the up-projection: both launches of one call;
+    # the plain layer at the same M is timed beside it
+    for M in (1, 16, 2048):
+        p = W.make_problem(M, 5120, 17408, 128, seed=0)
+        ad = W.make_adapter(5120, 17408, 32, seed=0)
+        steps = 200 if M <= 16 else 30
+        ms = time_lora(lib, torch, p, ad, steps, 10, l2)
+        plain, _ = time_gemm(lib, torch, p, steps, 10, l2_bytes=l2)
+        entry = {"ms": round(ms, 5), "plain_ms": round(plain, 5)}
+        if M <= 16:
+            gbs = (p.algorithmic_bytes + ad.extra_bytes(M)) / (ms * 1e-3) / 1e9
+            entry.update({"GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)})
+        else:
+            tfl = (p.flops + ad.extra_flops(M)) / (ms * 1e-3) / 1e12
+            entry.update({"TFLOP/s": round(tfl, 1), "frac_tensor": round(tfl / tf, 3)})
+        res[f"lora_r32_up_M{M}"] = entry
     return res
 
 

@@ -7,14 +7,17 @@
 //
 // This product is at most rank/N of the layer's work (well under 1 % for the
 // usual ranks), so it runs on the FP32 cores: one CTA computes 32 tokens x 32
-// ranks, streaming 64-k chunks of X and lora_a through shared memory.  When
-// there are fewer tiles than SMs, the CTAs of a thread-block cluster split K
-// and the partial sums are added in a fixed order (rank 0, 1, ...) through
-// distributed shared memory, so T is the same on every call.
+// ranks, streaming 64-k chunks of X and lora_a through shared memory (as
+// FP32, the next chunk fetched into registers while the current one is
+// used).  When there are fewer tiles than twice the SMs, the CTAs of a
+// thread-block cluster (up to 16) split K and the partial sums are added in a
+// fixed order (rank 0, 1, ...) through distributed shared memory, so T is the
+// same on every call.
 
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -28,16 +31,42 @@ constexpr int RT = 32;           // ranks per CTA (one per lane)
 constexpr int KC = 64;           // k per shared-memory chunk
 constexpr int THREADS = 256;     // warp w: tokens 4w .. 4w+3; lane: one rank
 constexpr int TOK_PER_WARP = MT / (THREADS / 32);
-constexpr int A_ROW_WORDS = KC / 2 + 1;  // padded: lane j reads row j conflict-free
-constexpr int kMaxSplits = 8;
+constexpr int A_ROW = KC + 4;    // padded FP32 row: 16-byte loads by 8 lanes hit 32 banks
+constexpr int WORDS = MT * KC / 2 / THREADS;  // 32-bit words of each chunk per thread
+constexpr int kMaxSplits = 16;
+static_assert(RT * KC / 2 / THREADS == WORDS, "X and lora_a chunks have the same size");
+
+// This thread's words of chunk c: X rows m0.., lora_a rows j0.. (zero outside
+// M, r and K).
+__device__ __forceinline__ void load_chunk(const uint16_t* __restrict__ x,
+                                           const uint16_t* __restrict__ a, int M, int K, int r,
+                                           int m0, int j0, int c, uint32_t (&xv)[WORDS],
+                                           uint32_t (&av)[WORDS]) {
+  const int k0 = c * KC;
+#pragma unroll
+  for (int u = 0; u < WORDS; ++u) {
+    const int i = threadIdx.x + u * THREADS;
+    const int row = i / (KC / 2), k = k0 + 2 * (i % (KC / 2));
+    const int m = m0 + row, j = j0 + row;
+    xv[u] = (m < M && k < K) ? __ldg(reinterpret_cast<const unsigned int*>(x + (int64_t)m * K + k))
+                             : 0u;
+    av[u] = (j < r && k < K) ? __ldg(reinterpret_cast<const unsigned int*>(a + (int64_t)j * K + k))
+                             : 0u;
+  }
+}
 
 __global__ void __launch_bounds__(THREADS)
     lora_down_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a,
                      uint16_t* __restrict__ t, int M, int K, int r, int splits) {
-  __shared__ uint32_t xs[MT][KC / 2];       // X chunk, half2 per word
-  __shared__ uint32_t as[RT][A_ROW_WORDS];  // lora_a chunk, half2 per word (padded rows)
+  __shared__ __align__(16) float xs[MT][KC];     // X chunk in FP32
+  __shared__ __align__(16) float as[RT][A_ROW];  // lora_a chunk in FP32 (padded rows)
   __shared__ float part[THREADS][TOK_PER_WARP];
 
+  // The layer launch that reads T may start now: it waits for this grid's
+  // completion before its first read of T, and every CTA of this grid is
+  // resident once all have passed this point, so the early start cannot keep
+  // any of them from an SM.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * MT, j0 = blockIdx.y * RT;
   const int split = splits > 1 ? (int)cluster_ctarank() : 0;  // the cluster spans z
@@ -47,34 +76,31 @@ __global__ void __launch_bounds__(THREADS)
   const int c_begin = split * per, c_end = min(chunks, c_begin + per);
 
   float acc[TOK_PER_WARP] = {};
+  uint32_t xv[WORDS], av[WORDS];
+  if (c_begin < c_end) load_chunk(x, a, M, K, r, m0, j0, c_begin, xv, av);
   for (int c = c_begin; c < c_end; ++c) {
-    const int k0 = c * KC;
-    // X chunk: 32 rows x 64 k, 32-bit words (zero outside M and K)
-    for (int i = threadIdx.x; i < MT * KC / 2; i += THREADS) {
+    // store this chunk (FP32), then fetch the next one while computing
+#pragma unroll
+    for (int u = 0; u < WORDS; ++u) {
+      const int i = threadIdx.x + u * THREADS;
       const int row = i / (KC / 2), w = i % (KC / 2);
-      const int m = m0 + row, k = k0 + 2 * w;
-      uint32_t v = 0;
-      if (m < M && k < K) v = *reinterpret_cast<const uint32_t*>(x + (int64_t)m * K + k);
-      xs[row][w] = v;
-    }
-    // lora_a chunk: 32 ranks x 64 k (zero outside r and K)
-    for (int i = threadIdx.x; i < RT * KC / 2; i += THREADS) {
-      const int row = i / (KC / 2), w = i % (KC / 2);
-      const int j = j0 + row, k = k0 + 2 * w;
-      uint32_t v = 0;
-      if (j < r && k < K) v = *reinterpret_cast<const uint32_t*>(a + (int64_t)j * K + k);
-      as[row][w] = v;
+      const float2 xf = __half22float2(*reinterpret_cast<const __half2*>(&xv[u]));
+      const float2 af = __half22float2(*reinterpret_cast<const __half2*>(&av[u]));
+      *reinterpret_cast<float2*>(&xs[row][2 * w]) = xf;
+      *reinterpret_cast<float2*>(&as[row][2 * w]) = af;
     }
     __syncthreads();
-#pragma unroll 8
-    for (int w = 0; w < KC / 2; ++w) {
-      const float2 av = __half22float2(*reinterpret_cast<const __half2*>(&as[lane][w]));
+    if (c + 1 < c_end) load_chunk(x, a, M, K, r, m0, j0, c + 1, xv, av);
+#pragma unroll 4
+    for (int k = 0; k < KC; k += 4) {
+      const float4 a4 = *reinterpret_cast<const float4*>(&as[lane][k]);
 #pragma unroll
       for (int q = 0; q < TOK_PER_WARP; ++q) {
-        const float2 xv =
-            __half22float2(*reinterpret_cast<const __half2*>(&xs[TOK_PER_WARP * warp + q][w]));
-        acc[q] = fmaf(xv.x, av.x, acc[q]);
-        acc[q] = fmaf(xv.y, av.y, acc[q]);
+        const float4 x4 = *reinterpret_cast<const float4*>(&xs[TOK_PER_WARP * warp + q][k]);
+        acc[q] = fmaf(x4.x, a4.x, acc[q]);
+        acc[q] = fmaf(x4.y, a4.y, acc[q]);
+        acc[q] = fmaf(x4.z, a4.z, acc[q]);
+        acc[q] = fmaf(x4.w, a4.w, acc[q]);
       }
     }
     __syncthreads();
@@ -115,9 +141,20 @@ cudaError_t launch_lora_down(const uint16_t* x, const uint16_t* lora_a, uint16_t
   const unsigned gm = (unsigned)((M + MT - 1) / MT), gr = (unsigned)((r + RT - 1) / RT);
   const int64_t tiles = (int64_t)gm * gr;
   const int chunks = (int)((K + KC - 1) / KC);
-  // split K over a cluster when the tiles alone cannot fill the SMs
-  int splits = (int)std::min<int64_t>(kMaxSplits, std::max<int64_t>(1, dev.num_sms / tiles));
+  // split K over a cluster when the tiles alone cannot fill the SMs twice
+  int splits = (int)std::min<int64_t>(kMaxSplits, std::max<int64_t>(1, 2 * dev.num_sms / tiles));
   splits = std::min(splits, chunks);
+  if (splits > 8) {
+    // clusters above the portable size of 8 have to be allowed per kernel
+    static std::once_flag once[64];
+    static cudaError_t attr_err[64];
+    const int d = dev.device & 63;
+    std::call_once(once[d], [&] {
+      attr_err[d] = cudaFuncSetAttribute(lora_down_kernel,
+                                         cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    });
+    if (attr_err[d] != cudaSuccess) splits = 8;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(gm, gr, (unsigned)splits);
   cfg.blockDim = dim3(THREADS, 1, 1);

@@ -270,6 +270,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         bool load = even || odd_rows;
         uint32_t copies = odd_rows ? 2u : 1u;
         int row = t0 + (int)rank * HT;
+        bool t_ready = false;
         for (int g = 0; g < G; ++g) {
           if (!mbar_wait_bounded(&bar->xempty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
             record_timeout(err, bar);
@@ -294,7 +295,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               }
             }
           } else {
-            // LoRA stage: 64 columns of T from column 32 * (kb - KW)
+            // LoRA stage: 64 columns of T from column 32 * (kb - KW).  T comes
+            // from the launch before this one, which may still be running
+            // (programmatic dependent launch): wait for it once, here.
+            if (!t_ready) {
+              asm volatile("griddepcontrol.wait;" ::: "memory");
+              t_ready = true;
+            }
             if (even) mbar_arrive_expect_tx(&bar->xfull[s], copies * L::X_HALF_BYTES);
             if (load) tma_load_2d_pair(dst, &t_map, LORA_R * (kb - KW), row, bar_c);
           }
@@ -650,10 +657,22 @@ cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint1
   const int64_t n_pairs = ((N + BW - 1) / BW + 1) / 2;
   const int64_t tiles = n_pairs * ((M + BT - 1) / BT);
   const int64_t clusters = std::min<int64_t>(tiles, std::max(1, dev.num_sms / 2));
-  prefill_pair_kernel<BT><<<dim3((unsigned)(2 * clusters)), THREADS, smem, stream>>>(
-      x_map, qw_map, s_map, y_map, t_map, b_map, (int)M, (int)K, (int)N, group_shift, scale_rows,
-      x3d, (int)n_pairs, (int)tiles, lora_stages, dev.error_word);
-  return cudaGetLastError();
+  // With an adapter this launch may start while the one computing T still
+  // runs (only the first read of T waits for it); the weights and X do not
+  // depend on that launch.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = lora_stages > 0 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, prefill_pair_kernel<BT>, x_map, qw_map, s_map, y_map, t_map,
+                            b_map, (int)M, (int)K, (int)N, group_shift, scale_rows, x3d,
+                            (int)n_pairs, (int)tiles, lora_stages, dev.error_word);
 }
 
 }  // namespace
