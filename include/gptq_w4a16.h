@@ -71,6 +71,7 @@ typedef enum {
 #define GPTQ_DECODE_MAX_M 32
 #define GPTQ_MAX_GROUPED 8     /* linears per gptq_w4a16_gemm_grouped call */
 #define GPTQ_MAX_LORA_RANK 256 /* largest adapter rank of gptq_w4a16_gemm_lora */
+#define GPTQ_LORA_SCRATCH_BYTES (8 << 20) /* T buffer of gptq_w4a16_gemm_lora_noalloc */
 
 /*
  * Y = X . dequant(qweight, scales).
@@ -163,6 +164,28 @@ GPTQ_API int gptq_w4a16_gemm_lora(const uint16_t* x, const int32_t* qweight,
                                   int32_t group, const uint16_t* lora_a,
                                   const uint16_t* lora_b, int64_t rank, uint16_t* t_work,
                                   uint16_t* y, void* stream);
+
+/*
+ * gptq_w4a16_gemm_lora without a caller-provided T buffer.  The pages have no
+ * counterpart of this entry point: it exists for callers that cannot hand
+ * the library device scratch.  T [M, rank] is kept in one fixed device buffer
+ * inside the library (GPTQ_LORA_SCRATCH_BYTES per device, part of the
+ * library's static device memory), so the call allocates nothing.
+ *   M * rank * 2 must not exceed GPTQ_LORA_SCRATCH_BYTES, else GPTQ_ERR_SHAPE
+ *   (checked before anything is enqueued).
+ * T is written in full before it is read, so nothing in the buffer has to
+ * start at zero.  Every call on a device uses the same buffer: two calls
+ * whose executions may overlap (streams without an ordering between them, or
+ * host threads enqueueing concurrently on different streams) race on it and
+ * can return wrong results; calls ordered on one stream are safe.  Results
+ * are bit-identical to gptq_w4a16_gemm_lora.  Other arguments, checks and
+ * errors as gptq_w4a16_gemm_lora (without t_work).
+ */
+GPTQ_API int gptq_w4a16_gemm_lora_noalloc(const uint16_t* x, const int32_t* qweight,
+                                          const uint16_t* scales, int64_t M, int64_t K,
+                                          int64_t N, int32_t group, const uint16_t* lora_a,
+                                          const uint16_t* lora_b, int64_t rank, uint16_t* y,
+                                          void* stream);
 
 /*
  * W[K, N] = dequant(qweight, scales) as FP16 bits, each value rounded once from

@@ -9,9 +9,9 @@ and fails loudly if it is missing.
 """
 __version__ = "0.1.0"
 
-_BINDING_NAMES = {"gemm", "gemm_grouped", "gemm_lora", "dequant", "select", "device_error", "version",
+_BINDING_NAMES = {"gemm", "gemm_grouped", "gemm_lora", "gemm_lora_noalloc", "dequant", "select", "device_error", "version",
                   "load", "GptqError", "KERNEL_AUTO", "KERNEL_DECODE", "KERNEL_PREFILL",
-                  "DECODE_MAX_M", "MAX_GROUPED", "MAX_LORA_RANK", "GROUP_SIZES"}
+                  "DECODE_MAX_M", "MAX_GROUPED", "MAX_LORA_RANK", "LORA_SCRATCH_BYTES", "GROUP_SIZES"}
 
 
 def __getattr__(name):

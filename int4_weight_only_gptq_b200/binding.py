@@ -21,6 +21,7 @@ KERNEL_AUTO, KERNEL_DECODE, KERNEL_PREFILL = 0, 1, 2
 DECODE_MAX_M = 32
 MAX_GROUPED = 8
 MAX_LORA_RANK = 256
+LORA_SCRATCH_BYTES = 8 << 20
 GROUP_SIZES = (-1, 16, 32, 64, 128, 256, 512, 1024)
 
 STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_NULL", 2: "GPTQ_ERR_SHAPE", 3: "GPTQ_ERR_GROUP",
@@ -29,7 +30,8 @@ STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_NULL", 2: "GPTQ_ERR_SHAPE", 3: "GPTQ_ERR_GR
 
 # Every entry point declared in include/gptq_w4a16.h.
 EXPORTS = ("gptq_w4a16_gemm", "gptq_w4a16_gemm_kernel", "gptq_w4a16_gemm_decode_splits",
-           "gptq_w4a16_gemm_grouped", "gptq_w4a16_gemm_lora", "gptq_dequant",
+           "gptq_w4a16_gemm_grouped", "gptq_w4a16_gemm_lora", "gptq_w4a16_gemm_lora_noalloc",
+           "gptq_dequant",
            "gptq_w4a16_select", "gptq_status_string", "gptq_device_error", "gptq_version")
 
 
@@ -65,6 +67,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                                     _p, _p]
             lib.gptq_w4a16_gemm_lora.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32, _p, _p,
                                                  _i64, _p, _p, _p]
+            lib.gptq_w4a16_gemm_lora_noalloc.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32,
+                                                         _p, _p, _i64, _p, _p]
             lib.gptq_dequant.argtypes = [_p, _p, _i64, _i64, _i32, _p, _p]
             lib.gptq_w4a16_select.argtypes = [_i64, _i64, _i64, _i32,
                                               ctypes.POINTER(_i32), ctypes.POINTER(_i32)]
@@ -74,7 +78,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.gptq_version.restype = ctypes.c_char_p
             for name in ("gptq_w4a16_gemm", "gptq_w4a16_gemm_kernel",
                          "gptq_w4a16_gemm_decode_splits", "gptq_w4a16_gemm_grouped",
-                         "gptq_w4a16_gemm_lora", "gptq_dequant",
+                         "gptq_w4a16_gemm_lora", "gptq_w4a16_gemm_lora_noalloc",
+                         "gptq_dequant",
                          "gptq_w4a16_select", "gptq_device_error"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
@@ -230,6 +235,32 @@ def gemm_lora(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, grou
     _check(lib.gptq_w4a16_gemm_lora(_ptr(x), _ptr(qweight), _ptr(scales), M, K, N, group,
                                     _ptr(lora_a), _ptr(lora_b), rank, _ptr(t_work), _ptr(out),
                                     _stream_handle(stream, dev)))
+    return out
+
+
+def gemm_lora_noalloc(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
+                      group: int, lora_a: torch.Tensor, lora_b: torch.Tensor,
+                      out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """gemm_lora with T kept in the library's static device buffer (no work
+    tensor; M * rank * 2 <= LORA_SCRATCH_BYTES; calls that may overlap in time
+    share the buffer and race)."""
+    lib = load()
+    dev = qweight.device
+    _require(qweight, "qweight", lambda d: d == torch.int32, None)
+    _require(scales, "scales", lambda d: d == torch.float16, dev)
+    _require(x, "x", lambda d: d == torch.float16, dev)
+    _require(lora_a, "lora_a", lambda d: d == torch.float16, dev)
+    _require(lora_b, "lora_b", lambda d: d == torch.float16, dev)
+    M, K = x.shape
+    N = qweight.shape[1]
+    rank = lora_a.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=dev)
+    else:
+        _require(out, "out", lambda d: d == torch.float16, dev)
+    _check(lib.gptq_w4a16_gemm_lora_noalloc(_ptr(x), _ptr(qweight), _ptr(scales), M, K, N,
+                                            group, _ptr(lora_a), _ptr(lora_b), rank, _ptr(out),
+                                            _stream_handle(stream, dev)))
     return out
 
 

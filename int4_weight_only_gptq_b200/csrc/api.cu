@@ -18,6 +18,10 @@ namespace {
 // One error word per device, written only by kernels that give up a wait.
 __device__ int g_error_word;
 
+// The T buffer of gptq_w4a16_gemm_lora_noalloc: static device memory of the
+// library, one per device, shared by every such call on that device.
+__device__ __align__(256) uint16_t g_lora_scratch[GPTQ_LORA_SCRATCH_BYTES / 2];
+
 constexpr int kMaxDevices = 64;
 std::once_flag g_dev_once[kMaxDevices];
 DeviceInfo g_dev[kMaxDevices];
@@ -54,6 +58,13 @@ int query_device(const DeviceInfo** out) {
       return;
     }
     info.error_word = static_cast<int*>(p);
+    void* q = nullptr;
+    if (cudaGetSymbolAddress(&q, g_lora_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      g_dev_status[d] = GPTQ_ERR_DEVICE;
+      return;
+    }
+    info.lora_scratch = static_cast<uint16_t*>(q);
     g_dev[d] = info;
     g_dev_status[d] = GPTQ_OK;
   });
@@ -128,6 +139,50 @@ int gemm_impl(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
     e = launch_decode(x, qweight, scales, y, M, K, N, gs, splits, s, *dev);
   else
     e = launch_prefill(x, qweight, scales, y, M, K, N, gs, s, *dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  return GPTQ_OK;
+}
+
+// The adapter path.  t_work: caller-owned T buffer, or (static_t) the
+// library's static one.
+int lora_impl(const uint16_t* x, const int32_t* qweight, const uint16_t* scales, int64_t M,
+              int64_t K, int64_t N, int32_t group, const uint16_t* lora_a,
+              const uint16_t* lora_b, int64_t rank, uint16_t* t_work, bool static_t, uint16_t* y,
+              void* stream) {
+  int st = check_shape(M, K, N, group);
+  if (st != GPTQ_OK) return st;
+  if (rank < 16 || rank > GPTQ_MAX_LORA_RANK || rank % 16 != 0) return GPTQ_ERR_SHAPE;
+  if (static_t && M * rank * 2 > (int64_t)GPTQ_LORA_SCRATCH_BYTES) return GPTQ_ERR_SHAPE;
+  if (!qweight || !scales || !lora_a || !lora_b) return GPTQ_ERR_NULL;
+  if (M == 0) return GPTQ_OK;
+  if (!x || !y || (!static_t && !t_work)) return GPTQ_ERR_NULL;
+  if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(y) ||
+      !aligned16(lora_a) || !aligned16(lora_b) || (!static_t && !aligned16(t_work)))
+    return GPTQ_ERR_ALIGN;
+  const int64_t xb = M * K * 2, qb = K / 8 * N * 4, sb = num_groups(K, group) * N * 2;
+  const int64_t ab = rank * K * 2, bb = N * rank * 2, tb = M * rank * 2, yb = M * N * 2;
+  // y and t_work are written: neither may overlap anything else (the static
+  // buffer overlaps no caller buffer)
+  if (overlaps(y, yb, x, xb) || overlaps(y, yb, qweight, qb) || overlaps(y, yb, scales, sb) ||
+      overlaps(y, yb, lora_a, ab) || overlaps(y, yb, lora_b, bb))
+    return GPTQ_ERR_ALIAS;
+  if (!static_t &&
+      (overlaps(y, yb, t_work, tb) || overlaps(t_work, tb, x, xb) ||
+       overlaps(t_work, tb, qweight, qb) || overlaps(t_work, tb, scales, sb) ||
+       overlaps(t_work, tb, lora_a, ab) || overlaps(t_work, tb, lora_b, bb)))
+    return GPTQ_ERR_ALIAS;
+  const DeviceInfo* dev = nullptr;
+  st = query_device(&dev);
+  if (st != GPTQ_OK) return st;
+  if (static_t) t_work = dev->lora_scratch;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_lora_down(x, lora_a, t_work, M, K, rank, s, *dev);
+  if (e == cudaSuccess)
+    e = launch_prefill_pair_lora(x, qweight, scales, y, M, K, N, group_shift_of(group), t_work,
+                                 lora_b, rank, s, *dev);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return GPTQ_ERR_CUDA;
@@ -214,38 +269,18 @@ int gptq_w4a16_gemm_lora(const uint16_t* x, const int32_t* qweight, const uint16
                          int64_t M, int64_t K, int64_t N, int32_t group, const uint16_t* lora_a,
                          const uint16_t* lora_b, int64_t rank, uint16_t* t_work, uint16_t* y,
                          void* stream) {
-  int st = check_shape(M, K, N, group);
-  if (st != GPTQ_OK) return st;
-  if (rank < 16 || rank > GPTQ_MAX_LORA_RANK || rank % 16 != 0) return GPTQ_ERR_SHAPE;
-  if (!qweight || !scales || !lora_a || !lora_b) return GPTQ_ERR_NULL;
-  if (M == 0) return GPTQ_OK;
-  if (!x || !y || !t_work) return GPTQ_ERR_NULL;
-  if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(y) ||
-      !aligned16(lora_a) || !aligned16(lora_b) || !aligned16(t_work))
-    return GPTQ_ERR_ALIGN;
-  const int64_t xb = M * K * 2, qb = K / 8 * N * 4, sb = num_groups(K, group) * N * 2;
-  const int64_t ab = rank * K * 2, bb = N * rank * 2, tb = M * rank * 2, yb = M * N * 2;
-  // y and t_work are written: neither may overlap anything else
-  if (overlaps(y, yb, x, xb) || overlaps(y, yb, qweight, qb) || overlaps(y, yb, scales, sb) ||
-      overlaps(y, yb, lora_a, ab) || overlaps(y, yb, lora_b, bb) || overlaps(y, yb, t_work, tb) ||
-      overlaps(t_work, tb, x, xb) || overlaps(t_work, tb, qweight, qb) ||
-      overlaps(t_work, tb, scales, sb) || overlaps(t_work, tb, lora_a, ab) ||
-      overlaps(t_work, tb, lora_b, bb))
-    return GPTQ_ERR_ALIAS;
-  const DeviceInfo* dev = nullptr;
-  st = query_device(&dev);
-  if (st != GPTQ_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_lora_down(x, lora_a, t_work, M, K, rank, s, *dev);
-  if (e == cudaSuccess)
-    e = launch_prefill_pair_lora(x, qweight, scales, y, M, K, N, group_shift_of(group), t_work,
-                                 lora_b, rank, s, *dev);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return GPTQ_ERR_CUDA;
-  }
-  return GPTQ_OK;
+  return lora_impl(x, qweight, scales, M, K, N, group, lora_a, lora_b, rank, t_work, false, y,
+                   stream);
 }
+
+int gptq_w4a16_gemm_lora_noalloc(const uint16_t* x, const int32_t* qweight,
+                                 const uint16_t* scales, int64_t M, int64_t K, int64_t N,
+                                 int32_t group, const uint16_t* lora_a, const uint16_t* lora_b,
+                                 int64_t rank, uint16_t* y, void* stream) {
+  return lora_impl(x, qweight, scales, M, K, N, group, lora_a, lora_b, rank, nullptr, true, y,
+                   stream);
+}
+
 
 int gptq_dequant(const int32_t* qweight, const uint16_t* scales, int64_t K, int64_t N,
                  int32_t group, uint16_t* w_out, void* stream) {

@@ -14,6 +14,7 @@ struct DeviceInfo {
   int smem_optin = 0;   // max dynamic shared memory per block (opt-in)
   int l2_bytes = 0;
   int* error_word = nullptr;  // device address of this device's error word
+  uint16_t* lora_scratch = nullptr;  // device address of the static T buffer
 };
 
 // Error codes written to the device error word (match gptq_status values).
