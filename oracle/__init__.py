@@ -17,6 +17,13 @@ adapter stays separate from the packed weights), read with PEFT's layouts and
 the adapter's scaling already in lora_b:
     T[m,j] = fp16_RNE(sum_k x[m,k] * lora_a[j,k])          lora_a [r, K]
     Y[m,n] += sum_j T[m,j] * lora_b[n,j]                    lora_b [N, r]
+
+With asymmetric zero points (GPTQModel wiki, "Defaults and compatibility
+decisions": sym; GPTQ-Pro README: asymmetric weights outside that fork's
+contract), read with GPTQ's packed qzeros [n_groups, N/8] (eight codes per
+int32 along N, lowest nibble = lowest n), each zero taken as stored:
+    z[g,n] = (uint32(qzeros[g, n//8]) >> 4*(n%8)) & 0xF
+    W[k,n] = fp16_RNE((q[k,n] - z[k//G, n]) * scales[k//G, n])
 """
 from __future__ import annotations
 
@@ -75,6 +82,9 @@ def _load():
             lib.oracle_gemm_rows.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32,
                                              _i64, _p, _p]
             lib.oracle_lora_down.argtypes = [_p, _p, _i64, _i64, _i64, _p]
+            lib.oracle_dequant_asym.argtypes = [_p, _p, _p, _i64, _i64, _i32, _p]
+            lib.oracle_gemm_asym_rows.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32,
+                                                  _i64, _p, _p]
             lib.oracle_lora_up_add.argtypes = [_p, _p, _i64, _i64, _i64, _p, _p]
             _lib = lib
     return _lib
@@ -251,3 +261,53 @@ def gemm_lora_rows(x, qweight, scales, group, lora_a, lora_b, ms) -> np.ndarray:
     ms = np.asarray(ms, dtype=np.int64)
     xs = np.ascontiguousarray(np.asarray(x)[ms])
     return lora_up_add(lora_down(xs, lora_a), lora_b, gemm_rows(x, qweight, scales, group, ms))
+
+
+def pack_zeros(zcodes: np.ndarray) -> np.ndarray:
+    """Zero codes [n_groups, N] (0..15) -> qzeros int32 [n_groups, N/8], eight
+    codes per word along N, lowest nibble = lowest n."""
+    z = np.asarray(zcodes, dtype=np.uint32)
+    G, N = z.shape
+    if N % 8:
+        raise ValueError("N must be a multiple of 8")
+    words = np.zeros((G, N // 8), dtype=np.uint32)
+    for j in range(8):
+        words |= (z[:, j::8] & 0xF) << (4 * j)
+    return words.view(np.int32)
+
+
+def dequant_asym(qweight, scales, qzeros, group) -> np.ndarray:
+    """W = fp16((q - z) * s) as float16 [K, N]."""
+    qw = _c(qweight, np.int32)
+    s = _bits16(scales)
+    qz = _c(qzeros, np.int32)
+    K, N = qw.shape[0] * 8, qw.shape[1]
+    if s.shape != (num_groups(K, group), N) or qz.shape != (s.shape[0], N // 8):
+        raise ValueError("scales or qzeros do not match K, N and the group")
+    w = np.empty((K, N), dtype=np.uint16)
+    _load().oracle_dequant_asym(_ptr(qw), _ptr(s), _ptr(qz), K, N, group, _ptr(w))
+    return w.view(np.float16)
+
+
+def gemm_asym_rows(x, qweight, scales, qzeros, group, ms) -> np.ndarray:
+    """Rows ms of Y = x . W_asym in binary64, float64 [len(ms), N]."""
+    xb = _bits16(x)
+    qw = _c(qweight, np.int32)
+    s = _bits16(scales)
+    qz = _c(qzeros, np.int32)
+    M, K = xb.shape
+    N = qw.shape[1]
+    if qz.shape != (s.shape[0], N // 8):
+        raise ValueError("qzeros do not match the scales")
+    ms = _c(np.asarray(ms, dtype=np.int64), np.int64)
+    if ms.size and (ms.min() < 0 or ms.max() >= M):
+        raise IndexError("row index out of range")
+    out = np.empty((ms.size, N), dtype=np.float64)
+    _load().oracle_gemm_asym_rows(_ptr(xb), _ptr(qw), _ptr(s), _ptr(qz), M, K, N, group,
+                                  ms.size, _ptr(ms), _ptr(out))
+    return out
+
+
+def gemm_asym(x, qweight, scales, qzeros, group) -> np.ndarray:
+    """Y = x . W_asym in binary64, float64 [M, N]."""
+    return gemm_asym_rows(x, qweight, scales, qzeros, group, np.arange(np.asarray(x).shape[0]))

@@ -272,3 +272,60 @@ void oracle_lora_up_add(const uint16_t* t, const uint16_t* lora_b, int64_t r, in
             y[i * N + n] += acc;
         }
 }
+
+/* ---- asymmetric zero points ----------------------------------------------
+ *
+ * GPTQModel wiki "Installation and Quickstart", "Defaults and compatibility
+ * decisions" (sym is True by default, and not every backend accepts
+ * asymmetric weights) and GPTQ-Pro README, "Runtime contract" (asymmetric
+ * weights lie outside that fork's contract).  Read with GPTQ's packed
+ * zero points, eight 4-bit codes per int32 along N (lowest nibble = lowest
+ * n, as the weights along K), each taken as stored:
+ *     z[g,n] = (uint32(qzeros[g, n/8]) >> 4*(n%8)) & 0xF   qzeros [n_groups, N/8]
+ *     W[k,n] = fp16_RNE((q[k,n] - z[g(k),n]) * scales[g(k),n])
+ * With every z = 8 this is the symmetric layer above.
+ */
+
+static int zero_at(const int32_t* qzeros, int64_t N, int64_t g, int64_t n)
+{
+    uint32_t word = (uint32_t)qzeros[g * (N / 8) + n / 8];
+    return (int)((word >> (4 * (n % 8))) & 0xFu);
+}
+
+static uint16_t dequant_asym_at(const int32_t* qweight, const uint16_t* scales,
+                                const int32_t* qzeros, int64_t N, int32_t group, int64_t k,
+                                int64_t n)
+{
+    int64_t g = group_of(k, group);
+    double q = (double)code_at(qweight, N, k, n);
+    double z = (double)zero_at(qzeros, N, g, n);
+    double s = oracle_half_to_double(scales[g * N + n]);
+    return oracle_double_to_half((q - z) * s);   /* exact product, one rounding */
+}
+
+void oracle_dequant_asym(const int32_t* qweight, const uint16_t* scales, const int32_t* qzeros,
+                         int64_t K, int64_t N, int32_t group, uint16_t* w)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t k = 0; k < K; ++k)
+        for (int64_t n = 0; n < N; ++n)
+            w[k * N + n] = dequant_asym_at(qweight, scales, qzeros, N, group, k, n);
+}
+
+/* Y rows ms[0..count) of the asymmetric layer, binary64 [count, N]. */
+void oracle_gemm_asym_rows(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                           const int32_t* qzeros, int64_t M, int64_t K, int64_t N,
+                           int32_t group, int64_t count, const int64_t* ms, double* out)
+{
+    (void)M;
+    #pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t i = 0; i < count; ++i) out[i * N + n] = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double w = oracle_half_to_double(
+                dequant_asym_at(qweight, scales, qzeros, N, group, k, n));
+            for (int64_t i = 0; i < count; ++i)
+                out[i * N + n] += oracle_half_to_double(x[ms[i] * K + k]) * w;
+        }
+    }
+}

@@ -326,3 +326,73 @@ def test_gemm_lora_rows_match_the_whole_result():
     full = oracle.gemm_lora(x, qw, s, G, a, b)
     rows = oracle.gemm_lora_rows(x, qw, s, G, a, b, [5, 0, 3])
     assert np.array_equal(rows, full[[5, 0, 3]])
+
+
+# ---- asymmetric zero points ----------------------------------------------------
+
+def _asym_problem(M, K, N, G, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    qw = oracle.pack(rng.integers(0, 16, size=(K, N)).astype(np.uint8))
+    ng = oracle.num_groups(K, G)
+    s = rng.uniform(1e-3, 2e-2, size=(ng, N)).astype(np.float16)
+    z = rng.integers(0, 16, size=(ng, N))
+    return x, qw, s, oracle.pack_zeros(z), z
+
+
+def test_asym_with_every_zero_eight_is_the_symmetric_layer():
+    x, qw, s, _, _ = _asym_problem(4, 96, 24, 32, seed=1)
+    qz = oracle.pack_zeros(np.full(s.shape, 8))
+    assert np.array_equal(oracle.dequant_asym(qw, s, qz, 32).view(np.uint16),
+                          oracle.dequant(qw, s, 32).view(np.uint16))
+    assert np.array_equal(oracle.gemm_asym(x, qw, s, qz, 32), oracle.gemm(x, qw, s, 32))
+
+
+def test_asym_dequant_every_code_and_zero_against_numpy():
+    """All 16 x 16 (code, zero) pairs with many scales: (q - z) * s is exact in
+    float32 (5-bit integer times an 11-bit significand), so numpy's float32
+    product rounded by numpy to float16 is the independent reference."""
+    rng = np.random.default_rng(2)
+    svals = np.concatenate([rng.uniform(1e-4, 8.0, 62), [2.0 ** -14, 65504.0]]).astype(np.float16)
+    K, N = 16 * 16, 64                       # row k: code k % 16; group k // 16: zero (k // 16)
+    codes = np.tile((np.arange(K) % 16)[:, None], (1, N)).astype(np.uint8)
+    qw = oracle.pack(codes)
+    s = np.tile(svals[None, :], (16, 1))     # group g: the same 64 scales
+    z = np.tile(np.arange(16)[:, None], (1, N))
+    w = oracle.dequant_asym(qw, s, oracle.pack_zeros(z), 16)
+    q = codes.astype(np.float32)
+    zz = np.repeat(z, 16, axis=0).astype(np.float32)
+    ref = ((q - zz) * np.repeat(s, 16, axis=0).astype(np.float32)).astype(np.float16)
+    assert np.array_equal(w.view(np.uint16), ref.view(np.uint16))
+
+
+def test_asym_zero_nibble_lands_on_one_group_and_column():
+    x, qw, s, _, _ = _asym_problem(2, 128, 32, 32, seed=3)
+    base = np.zeros(s.shape, dtype=np.int64)
+    w0 = oracle.dequant_asym(qw, s, oracle.pack_zeros(base), 32)
+    z = base.copy()
+    z[2, 13] = 5
+    w1 = oracle.dequant_asym(qw, s, oracle.pack_zeros(z), 32)
+    diff = np.argwhere(w0.view(np.uint16) != w1.view(np.uint16))
+    assert diff.size and set(diff[:, 1]) == {13} and set(diff[:, 0] // 32) == {2}
+
+
+def test_asym_code_equal_to_zero_gives_exact_zero():
+    K, N, G = 64, 16, 16
+    rng = np.random.default_rng(4)
+    z = rng.integers(0, 16, size=(K // G, N))
+    codes = np.repeat(z, G, axis=0).astype(np.uint8)
+    s = rng.uniform(1e-3, 2e-2, size=z.shape).astype(np.float16)
+    x = rng.standard_normal((3, K)).astype(np.float16)
+    y = oracle.gemm_asym(x, oracle.pack(codes), s, oracle.pack_zeros(z), G)
+    assert np.array_equal(y, np.zeros_like(y))
+
+
+@pytest.mark.parametrize("M,K,N,G", [(1, 16, 8, -1), (3, 48, 24, 16), (2, 96, 40, 32)])
+def test_gemm_asym_against_numpy_einsum(M, K, N, G):
+    x, qw, s, qz, z = _asym_problem(M, K, N, G, seed=M + K)
+    codes = oracle.unpack(qw).astype(np.float64)
+    g = np.arange(K) // (K if G == -1 else G)
+    w = ((codes - z[g]) * s[g].astype(np.float64)).astype(np.float16).astype(np.float64)
+    ref = np.einsum("mk,kn->mn", x.astype(np.float64), w)
+    assert np.allclose(oracle.gemm_asym(x, qw, s, qz, G), ref, rtol=1e-12, atol=1e-12)
