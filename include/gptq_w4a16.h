@@ -138,6 +138,28 @@ GPTQ_API int gptq_w4a16_gemm_grouped(const uint16_t* x, const int32_t* const* qw
                                      uint16_t* const* ys, void* stream);
 
 /*
+ * The layer with asymmetric zero points (GPTQ's sym=False weights):
+ *   Y = X . W,  W[k,n] = fp16((q[k,n] - z[k/G, n]) * scales[k/G, n])
+ *   z[g,n] = (uint32(qzeros[g, n/8]) >> 4*(n%8)) & 0xF
+ * The GPTQModel wiki ("Installation and Quickstart", "Defaults and
+ * compatibility decisions") defaults sym to True and notes that not every
+ * backend accepts asymmetric weights; the GPTQ-Pro README puts them outside
+ * its contract.  Read with GPTQ's packed zero points, each taken as stored:
+ *   qzeros   [n_groups, N/8] int32, device, eight 4-bit zeros per word along
+ *            N (lowest nibble = lowest n), 16-byte aligned
+ *   N        a multiple of 32 (zero-point rows are copied in 16-byte units)
+ * (q - z) is exact and scaled with one rounding, as in the symmetric layer;
+ * with every z = 8 the result equals gptq_w4a16_gemm's.  Every M runs on the
+ * prefill path.  Other arguments, checks and errors as gptq_w4a16_gemm, plus
+ * GPTQ_ERR_NULL for a NULL qzeros, GPTQ_ERR_SHAPE for N % 32 != 0, and
+ * GPTQ_ERR_ALIAS when y overlaps qzeros.
+ */
+GPTQ_API int gptq_w4a16_gemm_asym(const uint16_t* x, const int32_t* qweight,
+                                  const uint16_t* scales, const int32_t* qzeros, int64_t M,
+                                  int64_t K, int64_t N, int32_t group, uint16_t* y,
+                                  void* stream);
+
+/*
  * The layer with a LoRA adapter on its path:
  *   T = fp16(X . lora_a^T)                       [M, rank]
  *   Y = fp16(X . dequant(qweight, scales) + T . lora_b^T)

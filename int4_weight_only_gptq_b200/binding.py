@@ -30,7 +30,8 @@ STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_NULL", 2: "GPTQ_ERR_SHAPE", 3: "GPTQ_ERR_GR
 
 # Every entry point declared in include/gptq_w4a16.h.
 EXPORTS = ("gptq_w4a16_gemm", "gptq_w4a16_gemm_kernel", "gptq_w4a16_gemm_decode_splits",
-           "gptq_w4a16_gemm_grouped", "gptq_w4a16_gemm_lora", "gptq_w4a16_gemm_lora_noalloc",
+           "gptq_w4a16_gemm_grouped", "gptq_w4a16_gemm_asym", "gptq_w4a16_gemm_lora",
+           "gptq_w4a16_gemm_lora_noalloc",
            "gptq_dequant",
            "gptq_w4a16_select", "gptq_status_string", "gptq_device_error", "gptq_version")
 
@@ -67,6 +68,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                                     _p, _p]
             lib.gptq_w4a16_gemm_lora.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32, _p, _p,
                                                  _i64, _p, _p, _p]
+            lib.gptq_w4a16_gemm_asym.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32, _p, _p]
             lib.gptq_w4a16_gemm_lora_noalloc.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32,
                                                          _p, _p, _i64, _p, _p]
             lib.gptq_dequant.argtypes = [_p, _p, _i64, _i64, _i32, _p, _p]
@@ -78,7 +80,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.gptq_version.restype = ctypes.c_char_p
             for name in ("gptq_w4a16_gemm", "gptq_w4a16_gemm_kernel",
                          "gptq_w4a16_gemm_decode_splits", "gptq_w4a16_gemm_grouped",
-                         "gptq_w4a16_gemm_lora", "gptq_w4a16_gemm_lora_noalloc",
+                         "gptq_w4a16_gemm_asym", "gptq_w4a16_gemm_lora",
+                         "gptq_w4a16_gemm_lora_noalloc",
                          "gptq_dequant",
                          "gptq_w4a16_select", "gptq_device_error"):
                 getattr(lib, name).restype = ctypes.c_int
@@ -196,6 +199,31 @@ def gemm_grouped(x: torch.Tensor, qweights, scales, group: int, outs=None,
     _check(lib.gptq_w4a16_gemm_grouped(_ptr(x), qa, sa, na, count, M, K, group, ya,
                                        _stream_handle(stream, dev)))
     return outs
+
+
+def gemm_asym(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
+              qzeros: torch.Tensor, group: int, out: torch.Tensor | None = None,
+              stream=None) -> torch.Tensor:
+    """Y = x . W, W = fp16((q - z) * s) with zeros packed in qzeros
+    [n_groups, N/8] int32 (eight per word along N); N % 32 == 0."""
+    lib = load()
+    dev = qweight.device
+    _require(qweight, "qweight", lambda d: d == torch.int32, None)
+    _require(scales, "scales", lambda d: d == torch.float16, dev)
+    _require(qzeros, "qzeros", lambda d: d == torch.int32, dev)
+    _require(x, "x", lambda d: d == torch.float16, dev)
+    M, K = x.shape
+    N = qweight.shape[1]
+    if tuple(qzeros.shape) != (scales.shape[0], N // 8):
+        raise ValueError(f"qzeros has shape {tuple(qzeros.shape)}, expected "
+                         f"{(scales.shape[0], N // 8)}")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=dev)
+    else:
+        _require(out, "out", lambda d: d == torch.float16, dev)
+    _check(lib.gptq_w4a16_gemm_asym(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(qzeros), M, K,
+                                    N, group, _ptr(out), _stream_handle(stream, dev)))
+    return out
 
 
 def gemm_lora(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, group: int,

@@ -265,6 +265,35 @@ int gptq_w4a16_gemm_grouped(const uint16_t* x, const int32_t* const* qweights,
   return GPTQ_OK;
 }
 
+int gptq_w4a16_gemm_asym(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                         const int32_t* qzeros, int64_t M, int64_t K, int64_t N, int32_t group,
+                         uint16_t* y, void* stream) {
+  int st = check_shape(M, K, N, group);
+  if (st != GPTQ_OK) return st;
+  if (N % 32 != 0) return GPTQ_ERR_SHAPE;
+  if (!qweight || !scales || !qzeros) return GPTQ_ERR_NULL;
+  if (M == 0) return GPTQ_OK;
+  if (!x || !y) return GPTQ_ERR_NULL;
+  if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(qzeros) ||
+      !aligned16(y))
+    return GPTQ_ERR_ALIGN;
+  const int64_t ng = num_groups(K, group), yb = M * N * 2;
+  if (overlaps(y, yb, x, M * K * 2) || overlaps(y, yb, qweight, K / 8 * N * 4) ||
+      overlaps(y, yb, scales, ng * N * 2) || overlaps(y, yb, qzeros, ng * (N / 8) * 4))
+    return GPTQ_ERR_ALIAS;
+  const DeviceInfo* dev = nullptr;
+  st = query_device(&dev);
+  if (st != GPTQ_OK) return st;
+  const cudaError_t e = launch_prefill_pair_asym(x, qweight, scales, qzeros, y, M, K, N,
+                                                 group_shift_of(group),
+                                                 static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  return GPTQ_OK;
+}
+
 int gptq_w4a16_gemm_lora(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                          int64_t M, int64_t K, int64_t N, int32_t group, const uint16_t* lora_a,
                          const uint16_t* lora_b, int64_t rank, uint16_t* t_work, uint16_t* y,

@@ -77,6 +77,35 @@ __device__ __forceinline__ void dequant_word_natural(uint32_t w, uint32_t s2, ui
   n[3] = prmt(p[2], p[3], 0x7632);  // (k6, k7)
 }
 
+// With a zero point z (0..15) per weight instead of the constant 8: the
+// subtrahends are half2(1024 + z) for the low nibble pairs and the addends
+// half2(-(64 + z)) for the high pairs (bit patterns 0x6400 + z and
+// 0xD400 + 16 z), so every value q - z (in -15..15) is again exact and the
+// scale multiply rounds once.  z = 8 gives the constants of unpack_centered.
+__device__ __forceinline__ uint32_t zero_sub_low(uint32_t z) {
+  const uint32_t h = 0x6400u + z;
+  return h | (h << 16);
+}
+__device__ __forceinline__ uint32_t zero_add_high(uint32_t z) {
+  const uint32_t h = 0xD400u + 16u * z;
+  return h | (h << 16);
+}
+
+// dequant_word_natural with the zero point given as those two constants.
+__device__ __forceinline__ void dequant_word_natural_z(uint32_t w, uint32_t s2, uint32_t zlo,
+                                                       uint32_t zhi, uint32_t n[4]) {
+  const uint32_t w8 = w >> 8;
+  uint32_t p[4];
+  p[0] = hmul2_rn(hsub2_rn(lop3_and_or(w, 0x000F000Fu, kMagic1024), zlo), s2);
+  p[1] = hmul2_rn(hfma2_rn(lop3_and_or(w, 0x00F000F0u, kMagic1024), kOneSixteenth, zhi), s2);
+  p[2] = hmul2_rn(hsub2_rn(lop3_and_or(w8, 0x000F000Fu, kMagic1024), zlo), s2);
+  p[3] = hmul2_rn(hfma2_rn(lop3_and_or(w8, 0x00F000F0u, kMagic1024), kOneSixteenth, zhi), s2);
+  n[0] = prmt(p[0], p[1], 0x5410);  // (k0, k1)
+  n[1] = prmt(p[2], p[3], 0x5410);  // (k2, k3)
+  n[2] = prmt(p[0], p[1], 0x7632);  // (k4, k5)
+  n[3] = prmt(p[2], p[3], 0x7632);  // (k6, k7)
+}
+
 __device__ __forceinline__ uint32_t half2_broadcast(uint16_t h) {
   return (uint32_t)h | ((uint32_t)h << 16);
 }

@@ -64,6 +64,12 @@ cudaError_t launch_prefill_pair_lora(const uint16_t* x, const int32_t* qweight,
                                      int64_t N, int group_shift, const uint16_t* t,
                                      const uint16_t* lora_b, int64_t rank, cudaStream_t stream,
                                      const DeviceInfo& dev);
+// The pair kernel with asymmetric zero points: qzeros [n_groups, N/8] int32,
+// eight 4-bit zeros per word along N (N % 32 == 0).
+cudaError_t launch_prefill_pair_asym(const uint16_t* x, const int32_t* qweight,
+                                     const uint16_t* scales, const int32_t* qzeros, uint16_t* y,
+                                     int64_t M, int64_t K, int64_t N, int group_shift,
+                                     cudaStream_t stream, const DeviceInfo& dev);
 // t [M, r] = fp16(x . lora_a^T), lora_a [r, K] (the adapter's down-projection).
 cudaError_t launch_lora_down(const uint16_t* x, const uint16_t* lora_a, uint16_t* t, int64_t M,
                              int64_t K, int64_t r, cudaStream_t stream, const DeviceInfo& dev);

@@ -35,6 +35,12 @@
 // dequantisation and MMAs overlap the previous tile's epilogue, and no CTA
 // launch, TMEM allocation or pipeline fill is paid per tile.
 //
+// With asymmetric zero points (ASYM; GPTQModel wiki, "Defaults and
+// compatibility decisions": sym) the weight producer also loads the stage's
+// rows of packed zeros (qzeros [n_groups, N/8], eight per int32 along N) and
+// the dequantisation subtracts each column's zero instead of 8, at the same
+// number of FP16 operations.
+//
 // With a LoRA adapter (GPTQ-Pro README, "Runtime contract": adapters on the
 // linear path) each tile gets rank/32 more stages after its K stages: the
 // weight producer loads 32 columns of lora_b (FP16, copied into the TMEM A
@@ -73,7 +79,9 @@ constexpr int THREADS = (DQ_WARP0 + DQ_WARPS) * 32;
 constexpr int QW_STAGE_BYTES = BW * (BK / 8) * 4;  // 128 columns x 16 packed rows: 8 KB
 constexpr int S_ROW_BYTES = BW * 2;                // one scale row of the tile: 256 B
 constexpr int S_STAGE_MAX_ROWS = BK / 16;          // group 16: eight rows per stage
-constexpr int W_STAGE_BYTES = QW_STAGE_BYTES + S_STAGE_MAX_ROWS * S_ROW_BYTES;
+constexpr int Z_ROW_BYTES = BW / 8 * 4;           // one row of packed zero points: 64 B
+constexpr int Z_OFF = QW_STAGE_BYTES + S_STAGE_MAX_ROWS * S_ROW_BYTES;  // zeros in a slot
+constexpr int W_STAGE_BYTES = Z_OFF + S_STAGE_MAX_ROWS * Z_ROW_BYTES;
 // A LoRA stage: 32 of the adapter's rank.  Its weight tile is lora_b's 128
 // rows x 32 FP16 (64-byte rows, no swizzle); its token tile is T's rows x 64
 // columns (128-byte swizzle; the 32 columns past the stage are not used).
@@ -172,11 +180,12 @@ struct TileWalk {
 // tiles); cluster c takes tiles c, c + clusters, ...
 // lora_stages: LoRA stages per tile (0 without an adapter); t_map and b_map
 // then describe T [M, rank] and lora_b [N, rank].
-template <int BT>
+template <int BT, bool ASYM>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap x_map,
                         const __grid_constant__ CUtensorMap qw_map,
                         const __grid_constant__ CUtensorMap s_map,
+                        const __grid_constant__ CUtensorMap qz_map,
                         const __grid_constant__ CUtensorMap y_map,
                         const __grid_constant__ CUtensorMap t_map,
                         const __grid_constant__ CUtensorMap b_map, int M, int K, int N,
@@ -228,6 +237,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     prefetch_tensormap(&qw_map);
     prefetch_tensormap(&s_map);
     prefetch_tensormap(&y_map);
+    if (ASYM) prefetch_tensormap(&qz_map);
     if (lora_stages > 0) {
       prefetch_tensormap(&t_map);
       prefetch_tensormap(&b_map);
@@ -331,7 +341,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                               kDrainLimitNs);
         }
       } else {
-        const uint32_t wbytes = QW_STAGE_BYTES + scale_rows * S_ROW_BYTES;
+        const uint32_t wbytes =
+            QW_STAGE_BYTES + scale_rows * (S_ROW_BYTES + (ASYM ? Z_ROW_BYTES : 0));
         uint8_t* wst = smem + L::W_OFF;
         for (int g = 0; g < G; ++g) {
           if (!mbar_wait_bounded(&bar->wempty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
@@ -344,6 +355,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             tma_load_2d(wst, &qw_map, n0, k0 / 8, &bar->wfull[s]);
             tma_load_2d(wst + QW_STAGE_BYTES, &s_map, n0, (int)((int64_t)k0 >> group_shift),
                         &bar->wfull[s]);
+            if (ASYM)
+              tma_load_2d(wst + Z_OFF, &qz_map, n0 / 8, (int)((int64_t)k0 >> group_shift),
+                          &bar->wfull[s]);
           } else if (n0 < N) {
             // LoRA stage: lora_b rows n0.. , columns 32 * (kb - KW) ..
             mbar_arrive_expect_tx(&bar->wfull[s], LORA_W_BYTES);
@@ -437,6 +451,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // this thread's column in weight slot 0 (slot jw adds jw * W_STAGE_BYTES)
     const uint8_t* qw0 = smem + L::W_OFF + col * 4;
     const uint8_t* sc0 = smem + L::W_OFF + QW_STAGE_BYTES + col * 2;
+    // this thread's packed zero word in weight slot 0 (eight columns per word)
+    const uint8_t* zr0 = smem + L::W_OFF + Z_OFF + (col / 8) * 4;
+    const uint32_t zshift = 4u * (uint32_t)(col % 8);
     uint8_t* ystage = smem + L::Y_OFF + grp * L::Y_GROUP_BYTES + quarter * L::Y_WARP_BYTES;
 
     // Reads out tile d's accumulator (this warp's 32 lanes x its group's TPG
@@ -552,7 +569,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           const uint16_t sv = *reinterpret_cast<const uint16_t*>(sc + gl * S_ROW_BYTES);
           const uint32_t w = *reinterpret_cast<const uint32_t*>(qw + r * (BW * 4));
           uint32_t nat[4];
-          dequant_word_natural(w, half2_broadcast(sv), nat);
+          if constexpr (ASYM) {
+            const uint32_t z = (*reinterpret_cast<const uint32_t*>(
+                                    zr0 + jw * W_STAGE_BYTES + gl * Z_ROW_BYTES) >> zshift) & 0xFu;
+            dequant_word_natural_z(w, half2_broadcast(sv), zero_sub_low(z), zero_add_high(z), nat);
+          } else {
+            dequant_word_natural(w, half2_broadcast(sv), nat);
+          }
 #pragma unroll
           for (int q = 0; q < 4; ++q) cells[4 * r8 + q] = nat[q];
         }
@@ -598,14 +621,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int BT>
+template <int BT, bool ASYM>
 cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
-                          uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
-                          int scale_rows, int64_t n_groups, const uint16_t* t,
+                          const int32_t* qzeros, uint16_t* y, int64_t M, int64_t K, int64_t N,
+                          int group_shift, int scale_rows, int64_t n_groups, const uint16_t* t,
                           const uint16_t* lora_b, int64_t rank, cudaStream_t stream,
                           const DeviceInfo& dev) {
   using L = PairLayout<BT>;
-  CUtensorMap x_map, qw_map, s_map, y_map, t_map, b_map;
+  CUtensorMap x_map, qw_map, s_map, y_map, t_map, b_map, qz_map;
   // X as [K/64][M][64] (one copy of both 64-k halves per stage) when K is a
   // multiple of 64, else as [M][K] (one copy per half); rows at or beyond M
   // and k at or beyond K read as zero either way
@@ -629,6 +652,15 @@ cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint1
       !tensor_map_2d(&y_map, y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)N, (uint64_t)M,
                      (uint64_t)N * 2, 32, L::TPG, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
+  if (ASYM) {
+    // zero points [n_groups, N/8] int32: 16 words (128 columns) x the stage's rows
+    if (!tensor_map_2d(&qz_map, qzeros, CU_TENSOR_MAP_DATA_TYPE_INT32, (uint64_t)(N / 8),
+                       (uint64_t)n_groups, (uint64_t)(N / 8) * 4, BW / 8, (uint32_t)scale_rows,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  } else {
+    qz_map = qw_map;  // not read for symmetric weights
+  }
   int lora_stages = 0;
   if (rank > 0) {
     // T [M, rank]: 64 columns x BT/2 rows per copy (128-byte swizzle, the
@@ -648,7 +680,7 @@ cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint1
   static cudaError_t attr_err[64];
   const int d = dev.device & 63;
   std::call_once(attr_once[d], [&] {
-    attr_err[d] = cudaFuncSetAttribute(prefill_pair_kernel<BT>,
+    attr_err[d] = cudaFuncSetAttribute(prefill_pair_kernel<BT, ASYM>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   });
   if (attr_err[d] != cudaSuccess) return attr_err[d];
@@ -670,9 +702,31 @@ cudaError_t launch_pair_t(const uint16_t* x, const int32_t* qweight, const uint1
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = lora_stages > 0 ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, prefill_pair_kernel<BT>, x_map, qw_map, s_map, y_map, t_map,
-                            b_map, (int)M, (int)K, (int)N, group_shift, scale_rows, x3d,
-                            (int)n_pairs, (int)tiles, lora_stages, dev.error_word);
+  return cudaLaunchKernelEx(&cfg, prefill_pair_kernel<BT, ASYM>, x_map, qw_map, s_map, qz_map,
+                            y_map, t_map, b_map, (int)M, (int)K, (int)N, group_shift, scale_rows,
+                            x3d, (int)n_pairs, (int)tiles, lora_stages, dev.error_word);
+}
+
+// Both pair tiles, symmetric or with zero points, with or without an adapter.
+cudaError_t launch_pair(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                        const int32_t* qzeros, uint16_t* y, int64_t M, int64_t K, int64_t N,
+                        int group_shift, const uint16_t* t, const uint16_t* lora_b, int64_t rank,
+                        cudaStream_t stream, const DeviceInfo& dev) {
+  const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
+                               ? 1 : (K + (int64_t(1) << group_shift) - 1) >> group_shift;
+  const int scale_rows = group_shift >= 7 ? 1 : (BK >> group_shift);
+  if (qzeros) {
+    if (M <= 128)
+      return launch_pair_t<128, true>(x, qweight, scales, qzeros, y, M, K, N, group_shift,
+                                      scale_rows, n_groups, t, lora_b, rank, stream, dev);
+    return launch_pair_t<256, true>(x, qweight, scales, qzeros, y, M, K, N, group_shift,
+                                    scale_rows, n_groups, t, lora_b, rank, stream, dev);
+  }
+  if (M <= 128)
+    return launch_pair_t<128, false>(x, qweight, scales, nullptr, y, M, K, N, group_shift,
+                                     scale_rows, n_groups, t, lora_b, rank, stream, dev);
+  return launch_pair_t<256, false>(x, qweight, scales, nullptr, y, M, K, N, group_shift,
+                                   scale_rows, n_groups, t, lora_b, rank, stream, dev);
 }
 
 }  // namespace
@@ -682,22 +736,24 @@ cudaError_t launch_prefill_pair_lora(const uint16_t* x, const int32_t* qweight,
                                      int64_t N, int group_shift, const uint16_t* t,
                                      const uint16_t* lora_b, int64_t rank, cudaStream_t stream,
                                      const DeviceInfo& dev) {
-  const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
-                               ? 1 : (K + (int64_t(1) << group_shift) - 1) >> group_shift;
-  const int scale_rows = group_shift >= 7 ? 1 : (BK >> group_shift);
-  if (M <= 128)
-    return launch_pair_t<128>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups,
-                              t, lora_b, rank, stream, dev);
-  return launch_pair_t<256>(x, qweight, scales, y, M, K, N, group_shift, scale_rows, n_groups, t,
-                            lora_b, rank, stream, dev);
+  return launch_pair(x, qweight, scales, nullptr, y, M, K, N, group_shift, t, lora_b, rank,
+                     stream, dev);
+}
+
+cudaError_t launch_prefill_pair_asym(const uint16_t* x, const int32_t* qweight,
+                                     const uint16_t* scales, const int32_t* qzeros, uint16_t* y,
+                                     int64_t M, int64_t K, int64_t N, int group_shift,
+                                     cudaStream_t stream, const DeviceInfo& dev) {
+  return launch_pair(x, qweight, scales, qzeros, y, M, K, N, group_shift, nullptr, nullptr, 0,
+                     stream, dev);
 }
 
 cudaError_t launch_prefill_pair(const uint16_t* x, const int32_t* qweight,
                                 const uint16_t* scales, uint16_t* y, int64_t M, int64_t K,
                                 int64_t N, int group_shift, cudaStream_t stream,
                                 const DeviceInfo& dev) {
-  return launch_prefill_pair_lora(x, qweight, scales, y, M, K, N, group_shift, nullptr, nullptr,
-                                  0, stream, dev);
+  return launch_pair(x, qweight, scales, nullptr, y, M, K, N, group_shift, nullptr, nullptr, 0,
+                     stream, dev);
 }
 
 }  // namespace gptq

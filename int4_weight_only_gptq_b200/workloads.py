@@ -126,6 +126,18 @@ def make_adapter(K: int, N: int, rank: int, *, seed: int = 0, b_std: float = 0.0
     return Adapter(rank=rank, lora_a=a.astype(np.float16), lora_b=b.astype(np.float16))
 
 
+def make_qzeros(n_groups: int, N: int, *, seed: int = 0) -> np.ndarray:
+    """Packed zero points int32 [n_groups, N/8] for the asymmetric layer,
+    drawn as whole words (uniform over all bit patterns, so every 4-bit zero
+    is uniform in 0..15 and independent), from their own stream: PCG64
+    seeded with (seed, 2)."""
+    if N % 8:
+        raise ValueError("N must be a multiple of 8")
+    rng = np.random.Generator(np.random.PCG64([seed, 2]))
+    words = rng.integers(0, 2 ** 32, size=(n_groups, N // 8), dtype=np.uint64).astype(np.uint32)
+    return words.view(np.int32)
+
+
 # The five synthetic workloads, restated from their prose descriptions.
 def tiny(M: int = 1, seed: int = 0) -> Problem:
     """W4A16 GEMM, M in {1, 4}, K=512, N=256, group=128, scales U[1e-3, 2e-2]."""

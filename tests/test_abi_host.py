@@ -198,3 +198,32 @@ def test_lora_empty_m_and_no_device(lib):
     assert call_lora(lib, M=0, x=0, t=0, y=0, a=0) == 1
     if not torch.cuda.is_available():
         assert call_lora(lib) == 5
+
+
+# ---- gptq_w4a16_gemm_asym: host-side checks ----------------------------------
+# Fake qzeros [4, 32] (512 B) for K=512, N=256, group 128.
+
+QZ = 0x2400000
+
+
+def call_asym(lib, x=X, qw=QW, s=S, qz=QZ, M=4, K=512, N=256, g=128, y=Y):
+    v = ctypes.c_void_p
+    return lib.gptq_w4a16_gemm_asym(v(x), v(qw), v(s), v(qz), M, K, N, g, v(y), None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(N=264), 2), (dict(N=8), 2), (dict(K=520), 2), (dict(g=100), 3),
+    (dict(qz=0), 1), (dict(qw=0), 1), (dict(x=0), 1), (dict(y=0), 1),
+    (dict(qz=QZ + 4), 4), (dict(y=Y + 2), 4),
+    (dict(y=QZ), 8), (dict(y=X), 8), (dict(y=S + 32), 8),
+])
+def test_asym_argument_checks(lib, kw, status):
+    assert call_asym(lib, **kw) == status
+
+
+def test_asym_empty_m_and_no_device(lib):
+    import torch
+    assert call_asym(lib, M=0, x=0, y=0) == 0
+    assert call_asym(lib, M=0, x=0, y=0, qz=0) == 1
+    if not torch.cuda.is_available():
+        assert call_asym(lib) == 5

@@ -489,3 +489,76 @@ def test_lora_up_projection_full_size(M):
     print(f"[parity] lora up-projection M={M}: {err:.3e} over rows {rows}")
     assert np.all(np.isfinite(y[rows]))
     assert err <= TOL
+
+
+# ---- asymmetric zero points (gptq_w4a16_gemm_asym) ------------------------------
+
+def run_asym(p, qzeros):
+    x, qw, s = dev(p)
+    qz = torch.from_numpy(qzeros).cuda()
+    y = B.gemm_asym(x, qw, s, qz, p.group)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    return y.cpu().numpy()
+
+
+@pytest.mark.parametrize("M,K,N,G", [
+    (1, 512, 256, 128), (7, 1024, 160, 32), (16, 2048, 288, -1),
+    (33, 528, 128, 16),                 # 128-token pair tile, ragged K and last group
+    (130, 1040, 416, 64),               # 256-token pair tile, odd number of column tiles
+    (300, 96, 224, 32),                 # a single k stage
+    (2048, 5120, 512, 128),             # several token tiles per cluster
+])
+def test_asym_parity(M, K, N, G):
+    p = W.make_problem(M, K, N, G, seed=M + K)
+    qz = W.make_qzeros(p.scales.shape[0], N, seed=M + K)
+    y = run_asym(p, qz)
+    ref = oracle.gemm_asym(p.x, p.qweight, p.scales, qz, G)
+    err = rel_err(y, ref)
+    print(f"[parity] asym M={M} K={K} N={N} G={G}: {err:.3e}")
+    assert np.all(np.isfinite(y))
+    assert err <= TOL
+
+
+def test_asym_with_every_zero_eight_equals_the_symmetric_layer_bitwise():
+    """Above 32 tokens the symmetric call runs the same pair kernel; with all
+    zeros 8 the dequantised values are identical, hence Y too."""
+    p = W.make_problem(200, 2048, 416, 128, seed=31)
+    qz = np.full((p.scales.shape[0], p.N // 8), 0x88888888, dtype=np.uint32).view(np.int32)
+    assert np.array_equal(run_asym(p, qz).view(np.uint16), run(p).view(np.uint16))
+
+
+@pytest.mark.parametrize("M", [1, 40, 300])
+def test_asym_integer_exact_inputs_bitwise(M):
+    rng = np.random.default_rng(M)
+    p = W.make_problem(M, 2048, 160, 64, seed=M)
+    p.x[:] = rng.integers(-4, 5, size=p.x.shape).astype(np.float16)
+    p.scales[:] = np.float16(2.0 ** -6)
+    qz = W.make_qzeros(p.scales.shape[0], p.N, seed=M)
+    y = run_asym(p, qz)
+    ref = oracle.round_to_half(oracle.gemm_asym(p.x, p.qweight, p.scales, qz, 64))
+    assert np.array_equal(y.view(np.uint16), ref.view(np.uint16))
+
+
+def test_asym_one_hot_x_reproduces_dequantised_rows_bitwise():
+    M, K, N, G = 64, 1024, 288, 32
+    p = W.make_problem(M, K, N, G, seed=12)
+    qz = W.make_qzeros(p.scales.shape[0], N, seed=12)
+    ks = np.random.default_rng(12).integers(0, K, size=M)
+    p.x[:] = 0
+    p.x[np.arange(M), ks] = 1
+    y = run_asym(p, qz)
+    w = oracle.dequant_asym(p.qweight, p.scales, qz, G)
+    assert np.array_equal(y.view(np.uint16), w[ks].view(np.uint16))
+
+
+@pytest.mark.parametrize("M", [1, 2048])
+def test_asym_up_projection_full_size(M):
+    p = W.decode_up() if M == 1 else W.prefill(M)
+    qz = W.make_qzeros(p.scales.shape[0], p.N, seed=M)
+    y = run_asym(p, qz)
+    rows = sorted({0, M // 2, M - 1})
+    ref = oracle.gemm_asym_rows(p.x, p.qweight, p.scales, qz, p.group, rows)
+    err = rel_err(y[rows], ref)
+    print(f"[parity] asym up-projection M={M}: {err:.3e} over rows {rows}")
+    assert err <= TOL
