@@ -281,6 +281,31 @@ def time_grouped(lib, torch, ps, steps, warmup, l2_bytes):
     return e0.elapsed_time(e1) / steps
 
 
+def time_asym(lib, torch, p, qzeros, steps, warmup, l2_bytes):
+    """Device time per call (ms) of back-to-back gptq_w4a16_gemm_asym calls,
+    rotating weight copies past the L2 like time_gemm."""
+    copies = copies_for(p, l2_bytes) if l2_bytes else 1
+    sets = to_device(p, torch, copies)
+    zs = [torch.from_numpy(qzeros).cuda() for _ in range(copies)]
+    sh = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    v = ctypes.c_void_p
+    argv = [(v(x.data_ptr()), v(qw.data_ptr()), v(s.data_ptr()), v(z.data_ptr()), p.M, p.K, p.N,
+             p.group, v(y.data_ptr()), sh) for (x, qw, s, y), z in zip(sets, zs)]
+    fn = lib.gptq_w4a16_gemm_asym
+    for i in range(warmup):
+        st = fn(*argv[i % copies])
+        if st:
+            raise RuntimeError(f"asym gemm status {st}")
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        fn(*argv[i % copies])
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
 def time_lora(lib, torch, p, ad, steps, warmup, l2_bytes):
     """Device time per call (ms) of back-to-back gptq_w4a16_gemm_lora calls
     (the adapter's down-projection launch and the layer launch), rotating
@@ -491,6 +516,21 @@ def run_sweep(lib, torch, l2, hbm, tf):
             tfl = (p.flops + ad.extra_flops(M)) / (ms * 1e-3) / 1e12
             entry.update({"TFLOP/s": round(tfl, 1), "frac_tensor": round(tfl / tf, 3)})
         res[f"lora_r32_up_M{M}"] = entry
+    # asymmetric zero points on the up-projection; the symmetric layer beside it
+    for M in (1, 16, 2048):
+        p = W.make_problem(M, 5120, 17408, 128, seed=0)
+        qz = W.make_qzeros(p.scales.shape[0], p.N, seed=0)
+        steps = 200 if M <= 16 else 30
+        ms = time_asym(lib, torch, p, qz, steps, 10, l2)
+        plain, _ = time_gemm(lib, torch, p, steps, 10, l2_bytes=l2)
+        entry = {"ms": round(ms, 5), "symmetric_ms": round(plain, 5)}
+        if M <= 16:
+            gbs = (p.algorithmic_bytes + qz.size * 4) / (ms * 1e-3) / 1e9
+            entry.update({"GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)})
+        else:
+            tfl = p.flops / (ms * 1e-3) / 1e12
+            entry.update({"TFLOP/s": round(tfl, 1), "frac_tensor": round(tfl / tf, 3)})
+        res[f"asym_up_M{M}"] = entry
     return res
 
 
