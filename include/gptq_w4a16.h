@@ -149,8 +149,9 @@ GPTQ_API int gptq_w4a16_gemm_grouped(const uint16_t* x, const int32_t* const* qw
  *            N (lowest nibble = lowest n), 16-byte aligned
  *   N        a multiple of 32 (zero-point rows are copied in 16-byte units)
  * (q - z) is exact and scaled with one rounding, as in the symmetric layer;
- * with every z = 8 the result equals gptq_w4a16_gemm's.  Every M runs on the
- * prefill path.  Other arguments, checks and errors as gptq_w4a16_gemm, plus
+ * with every z = 8 the result equals gptq_w4a16_gemm's.  The kernel follows
+ * M as in gptq_w4a16_gemm (decode up to GPTQ_DECODE_MAX_M, prefill above).
+ * Other arguments, checks and errors as gptq_w4a16_gemm, plus
  * GPTQ_ERR_NULL for a NULL qzeros, GPTQ_ERR_SHAPE for N % 32 != 0, and
  * GPTQ_ERR_ALIAS when y overlaps qzeros.
  */

@@ -284,9 +284,12 @@ int gptq_w4a16_gemm_asym(const uint16_t* x, const int32_t* qweight, const uint16
   const DeviceInfo* dev = nullptr;
   st = query_device(&dev);
   if (st != GPTQ_OK) return st;
-  const cudaError_t e = launch_prefill_pair_asym(x, qweight, scales, qzeros, y, M, K, N,
-                                                 group_shift_of(group),
-                                                 static_cast<cudaStream_t>(stream), *dev);
+  const int gs = group_shift_of(group);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = M <= GPTQ_DECODE_MAX_M
+                            ? launch_decode_asym(x, qweight, scales, qzeros, y, M, K, N, gs, s, *dev)
+                            : launch_prefill_pair_asym(x, qweight, scales, qzeros, y, M, K, N, gs,
+                                                       s, *dev);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return GPTQ_ERR_CUDA;

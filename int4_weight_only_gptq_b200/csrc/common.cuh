@@ -91,6 +91,16 @@ __device__ __forceinline__ uint32_t zero_add_high(uint32_t z) {
   return h | (h << 16);
 }
 
+// dequant_word_paired with the zero point given as those two constants.
+__device__ __forceinline__ void dequant_word_paired_z(uint32_t w, uint32_t s2, uint32_t zlo,
+                                                      uint32_t zhi, uint32_t p[4]) {
+  const uint32_t w8 = w >> 8;
+  p[0] = hmul2_rn(hsub2_rn(lop3_and_or(w, 0x000F000Fu, kMagic1024), zlo), s2);
+  p[1] = hmul2_rn(hfma2_rn(lop3_and_or(w, 0x00F000F0u, kMagic1024), kOneSixteenth, zhi), s2);
+  p[2] = hmul2_rn(hsub2_rn(lop3_and_or(w8, 0x000F000Fu, kMagic1024), zlo), s2);
+  p[3] = hmul2_rn(hfma2_rn(lop3_and_or(w8, 0x00F000F0u, kMagic1024), kOneSixteenth, zhi), s2);
+}
+
 // dequant_word_natural with the zero point given as those two constants.
 __device__ __forceinline__ void dequant_word_natural_z(uint32_t w, uint32_t s2, uint32_t zlo,
                                                        uint32_t zhi, uint32_t n[4]) {

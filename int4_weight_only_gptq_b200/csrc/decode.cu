@@ -75,6 +75,7 @@ constexpr int THREADS = (2 + DQ_WARPS) * 32;
 constexpr int X_ATOMS = BKS / 64;
 constexpr int QW_STAGE_BYTES = PRS * BW * 4;
 constexpr int S_ROW_BYTES = BW * 2;
+constexpr int Z_ROW_BYTES = BW / 8 * 4;  // one row of packed zero points (asymmetric weights)
 constexpr int kMaxStages = 8;
 constexpr int kRingBudget = 224 * 1024;
 constexpr int A_SLOTS = 3;
@@ -116,11 +117,13 @@ inline int align1024(int v) { return (v + 1023) & ~1023; }
 
 // Stages start on multiples of 512 k and groups are powers of two, so a
 // stage touches 512 / group scale rows (one for groups of 512 and more).
+// With zero points (asym) each stage also holds their rows after the scales.
 template <int BT>
-inline DecodeShape decode_shape(int group_shift) {
+inline DecodeShape decode_shape(int group_shift, bool asym = false) {
   DecodeShape d;
   d.scale_rows = group_shift >= 9 ? 1 : (BKS >> group_shift);
-  d.stage_bytes = align1024(TokGeo<BT>::S_OFF + d.scale_rows * S_ROW_BYTES);
+  d.stage_bytes = align1024(TokGeo<BT>::S_OFF +
+                            d.scale_rows * (S_ROW_BYTES + (asym ? Z_ROW_BYTES : 0)));
   const int s = kRingBudget / d.stage_bytes;
   d.stages = s > kMaxStages ? kMaxStages : s;
   d.smem_bytes = 1024 + d.stages * d.stage_bytes + 256;
@@ -197,11 +200,14 @@ __device__ __forceinline__ void permute_x_chunk(uint8_t* p) {
 // group 16, 4 for group 32, 8 (the thread's whole slice) for 64 and more.
 // x3d: X arrives as one 3-D box per stage (K a multiple of 64) instead of
 // one 2-D box per 64-k atom.
-template <int WPS, int BT>
+// ASYM: asymmetric weights (one linear): qz_map describes the packed zero
+// points [n_groups, N/8]; each stage holds their rows after the scales and
+// every column's zero replaces the 8 of the symmetric layer.
+template <int WPS, int BT, bool ASYM>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ LinearSet ls,
-                  int M, int K, int group_shift, int stages, int stage_bytes, int scale_rows,
-                  int x3d, int* err) {
+                  const __grid_constant__ CUtensorMap qz_map, int M, int K, int group_shift,
+                  int stages, int stage_bytes, int scale_rows, int x3d, int* err) {
   constexpr int X_ATOM_BYTES = TokGeo<BT>::X_ATOM_BYTES;
   constexpr int X_STAGE_BYTES = TokGeo<BT>::X_STAGE_BYTES;
   constexpr int QW_OFF = TokGeo<BT>::QW_OFF;
@@ -229,6 +235,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int st_end = (int)((int64_t)(blockIdx.y + 1) * NS / splits);
   const int n_st = st_end - st_begin;
   const int gs = min(group_shift, 30);        // group -1 (shift 62): row 0 throughout
+  const int z_off = S_OFF + scale_rows * S_ROW_BYTES;  // zero-point rows (ASYM)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -247,6 +254,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     prefetch_tensormap(&x_map);
     prefetch_tensormap(qw_map);
     prefetch_tensormap(s_map);
+    if (ASYM) prefetch_tensormap(&qz_map);
     // L2 prefetch of the first stages' weight tiles: safe before the wait
     const int pf = min(n_st, 2);
     for (int t = 0; t < pf; ++t) tma_prefetch_l2_2d(qw_map, n0, (st_begin + t) * PRS);
@@ -281,9 +289,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint8_t* st = smem + s * stage_bytes;
         const int k0 = (st_begin + t) * BKS;
         mbar_arrive_expect_tx(&bar->full[s],
-                              X_STAGE_BYTES + QW_STAGE_BYTES + scale_rows * S_ROW_BYTES);
+                              X_STAGE_BYTES + QW_STAGE_BYTES +
+                                  scale_rows * (S_ROW_BYTES + (ASYM ? Z_ROW_BYTES : 0)));
         tma_load_2d(st + QW_OFF, qw_map, n0, k0 >> 3, &bar->full[s]);
         tma_load_2d(st + S_OFF, s_map, n0, k0 >> gs, &bar->full[s]);
+        if (ASYM) tma_load_2d(st + z_off, &qz_map, n0 / 8, k0 >> gs, &bar->full[s]);
         if (x3d) {
           tma_load_3d(st, &x_map, 0, 0, k0 >> 6, &bar->full[s]);
         } else {
@@ -409,17 +419,27 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint8_t* qw = st + QW_OFF + row0 * (BW * 4) + col * 4;
           const uint8_t* sc = st + S_OFF + col * 2;
           uint32_t cells[4 * WPT];
-          uint32_t s2 = 0;
+          uint32_t s2 = 0, zlo = 0, zhi = 0;
 #pragma unroll
           for (int i = 0; i < WPT; ++i) {
             if (i % WPS == 0) {
               // scale row of packed row row0 + i inside the stage's scale tile
               const int row = (8 * (row0 + i)) >> gs;
               s2 = half2_broadcast(*reinterpret_cast<const uint16_t*>(sc + row * S_ROW_BYTES));
+              if constexpr (ASYM) {
+                const uint32_t zw = *reinterpret_cast<const uint32_t*>(
+                    st + z_off + row * Z_ROW_BYTES + (col / 8) * 4);
+                const uint32_t z = (zw >> (4 * (col % 8))) & 0xFu;
+                zlo = zero_sub_low(z);
+                zhi = zero_add_high(z);
+              }
             }
             const uint32_t w = *reinterpret_cast<const uint32_t*>(qw + i * (BW * 4));
             uint32_t p[4];
-            dequant_word_paired(w, s2, p);
+            if constexpr (ASYM)
+              dequant_word_paired_z(w, s2, zlo, zhi, p);
+            else
+              dequant_word_paired(w, s2, p);
 #pragma unroll
             for (int j = 0; j < 4; ++j) cells[4 * i + j] = p[j];
           }
@@ -517,15 +537,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int WPS, int BT>
-cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, int M, int K, int group_shift,
-                     int splits, int x3d, const DecodeShape& d, cudaStream_t stream,
-                     const DeviceInfo& dev) {
+template <int WPS, int BT, bool ASYM>
+cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtensorMap& qz_map,
+                     int M, int K, int group_shift, int splits, int x3d, const DecodeShape& d,
+                     cudaStream_t stream, const DeviceInfo& dev) {
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
   const int di = dev.device & 63;
   std::call_once(once[di], [&] {
-    attr_err[di] = cudaFuncSetAttribute(decode_kernel<WPS, BT>,
+    attr_err[di] = cudaFuncSetAttribute(decode_kernel<WPS, BT, ASYM>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         1024 + kRingBudget + 256);
   });
@@ -549,8 +569,9 @@ cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, int M, int K
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT>, x_map, ls, M, K, group_shift, d.stages,
-                            d.stage_bytes, d.scale_rows, x3d, dev.error_word);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT, ASYM>, x_map, ls, qz_map, M, K,
+                            group_shift, d.stages, d.stage_bytes, d.scale_rows, x3d,
+                            dev.error_word);
 }
 
 // One linear of a launch, as the host sees it.
@@ -563,10 +584,15 @@ struct LinearArgs {
 
 // Tensor maps and launch for a token tile of BT over `count` linears that
 // share X (count = 1 for a plain call).
+// qzeros: packed zero points of the (single) linear for asymmetric weights,
+// or nullptr.
 template <int BT>
-cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count, int64_t M, int64_t K,
-                      int group_shift, int splits, cudaStream_t stream, const DeviceInfo& dev) {
-  const DecodeShape d = decode_shape<BT>(group_shift);
+cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count, const int32_t* qzeros,
+                      int64_t M, int64_t K, int group_shift, int splits, cudaStream_t stream,
+                      const DeviceInfo& dev) {
+  const bool asym = qzeros != nullptr;
+  if (asym && count != 1) return cudaErrorInvalidValue;
+  const DecodeShape d = decode_shape<BT>(group_shift, asym);
   if (d.stages < GROUPS || d.smem_bytes > 1024 + kRingBudget + 256) return cudaErrorInvalidValue;
   if (count < 1 || count > kMaxLinears) return cudaErrorInvalidValue;
   const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
@@ -608,20 +634,42 @@ cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count, int64
   if (!x3d && !tensor_map_2d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K,
                              (uint64_t)M, (uint64_t)K * 2, 64, BT, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  CUtensorMap qz_map = ls.qw[0];  // read only for asymmetric weights
+  if (asym) {
+    const uint64_t N = (uint64_t)lin[0].n;
+    if (!tensor_map_2d(&qz_map, qzeros, CU_TENSOR_MAP_DATA_TYPE_INT32, N / 8, (uint64_t)n_groups,
+                       N / 2, BW / 8, (uint32_t)d.scale_rows, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  }
   if (splits <= 0) splits = decode_pick_splits_blocks(ls.blk0[count], K, dev);
   const int iM = (int)M, iK = (int)K;
+  if (asym) {
+    if (group_shift == 4)
+      return launch_t<2, BT, true>(x_map, ls, qz_map, iM, iK, group_shift, splits, x3d, d, stream,
+                                   dev);
+    if (group_shift == 5)
+      return launch_t<4, BT, true>(x_map, ls, qz_map, iM, iK, group_shift, splits, x3d, d, stream,
+                                   dev);
+    return launch_t<WPT, BT, true>(x_map, ls, qz_map, iM, iK, group_shift, splits, x3d, d, stream,
+                                   dev);
+  }
   if (group_shift == 4)
-    return launch_t<2, BT>(x_map, ls, iM, iK, group_shift, splits, x3d, d, stream, dev);
+    return launch_t<2, BT, false>(x_map, ls, qz_map, iM, iK, group_shift, splits, x3d, d, stream,
+                                  dev);
   if (group_shift == 5)
-    return launch_t<4, BT>(x_map, ls, iM, iK, group_shift, splits, x3d, d, stream, dev);
-  return launch_t<WPT, BT>(x_map, ls, iM, iK, group_shift, splits, x3d, d, stream, dev);
+    return launch_t<4, BT, false>(x_map, ls, qz_map, iM, iK, group_shift, splits, x3d, d, stream,
+                                  dev);
+  return launch_t<WPT, BT, false>(x_map, ls, qz_map, iM, iK, group_shift, splits, x3d, d, stream,
+                                  dev);
 }
 
-cudaError_t launch_set(const uint16_t* x, const LinearArgs* lin, int count, int64_t M, int64_t K,
-                       int group_shift, int splits, cudaStream_t stream, const DeviceInfo& dev) {
+cudaError_t launch_set(const uint16_t* x, const LinearArgs* lin, int count,
+                       const int32_t* qzeros, int64_t M, int64_t K, int group_shift, int splits,
+                       cudaStream_t stream, const DeviceInfo& dev) {
   // token tile: 16 tokens up to M = 16, else 32
-  if (M <= 16) return launch_bt<16>(x, lin, count, M, K, group_shift, splits, stream, dev);
-  return launch_bt<32>(x, lin, count, M, K, group_shift, splits, stream, dev);
+  if (M <= 16)
+    return launch_bt<16>(x, lin, count, qzeros, M, K, group_shift, splits, stream, dev);
+  return launch_bt<32>(x, lin, count, qzeros, M, K, group_shift, splits, stream, dev);
 }
 
 }  // namespace
@@ -655,7 +703,15 @@ cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint1
                           uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
                           int splits, cudaStream_t stream, const DeviceInfo& dev) {
   const LinearArgs one{qweight, scales, y, N};
-  return launch_set(x, &one, 1, M, K, group_shift, splits, stream, dev);
+  return launch_set(x, &one, 1, nullptr, M, K, group_shift, splits, stream, dev);
+}
+
+cudaError_t launch_decode_asym(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                               const int32_t* qzeros, uint16_t* y, int64_t M, int64_t K,
+                               int64_t N, int group_shift, cudaStream_t stream,
+                               const DeviceInfo& dev) {
+  const LinearArgs one{qweight, scales, y, N};
+  return launch_set(x, &one, 1, qzeros, M, K, group_shift, 0, stream, dev);
 }
 
 cudaError_t launch_decode_grouped(const uint16_t* x, const int32_t* const* qweights,
@@ -665,7 +721,7 @@ cudaError_t launch_decode_grouped(const uint16_t* x, const int32_t* const* qweig
   if (count < 1 || count > kMaxLinears) return cudaErrorInvalidValue;
   LinearArgs lin[kMaxLinears];
   for (int i = 0; i < count; ++i) lin[i] = LinearArgs{qweights[i], scales[i], ys[i], ns[i]};
-  return launch_set(x, lin, count, M, K, group_shift, 0, stream, dev);
+  return launch_set(x, lin, count, nullptr, M, K, group_shift, 0, stream, dev);
 }
 
 }  // namespace gptq

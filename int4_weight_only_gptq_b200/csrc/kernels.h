@@ -39,6 +39,12 @@ int decode_pick_splits_blocks(int64_t column_blocks, int64_t K, const DeviceInfo
 cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                           uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
                           int splits, cudaStream_t stream, const DeviceInfo& dev);
+// Decode with asymmetric zero points: qzeros [n_groups, N/8] int32, eight
+// 4-bit zeros per word along N (N % 32 == 0).
+cudaError_t launch_decode_asym(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                               const int32_t* qzeros, uint16_t* y, int64_t M, int64_t K,
+                               int64_t N, int group_shift, cudaStream_t stream,
+                               const DeviceInfo& dev);
 // Decode of `count` linears that share X (1..GPTQ_MAX_GROUPED), one launch;
 // the split is picked from the total number of column blocks.
 cudaError_t launch_decode_grouped(const uint16_t* x, const int32_t* const* qweights,

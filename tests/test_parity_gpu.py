@@ -503,7 +503,9 @@ def run_asym(p, qzeros):
 
 
 @pytest.mark.parametrize("M,K,N,G", [
-    (1, 512, 256, 128), (7, 1024, 160, 32), (16, 2048, 288, -1),
+    # decode kernel (M <= 32): 16- and 32-token tiles, groups of 16 and 32
+    (1, 512, 256, 128), (5, 512, 256, 16), (7, 1024, 160, 32), (16, 2048, 288, -1),
+    (24, 1040, 224, 128), (32, 6144, 96, 64),
     (33, 528, 128, 16),                 # 128-token pair tile, ragged K and last group
     (130, 1040, 416, 64),               # 256-token pair tile, odd number of column tiles
     (300, 96, 224, 32),                 # a single k stage
@@ -520,15 +522,17 @@ def test_asym_parity(M, K, N, G):
     assert err <= TOL
 
 
-def test_asym_with_every_zero_eight_equals_the_symmetric_layer_bitwise():
-    """Above 32 tokens the symmetric call runs the same pair kernel; with all
-    zeros 8 the dequantised values are identical, hence Y too."""
-    p = W.make_problem(200, 2048, 416, 128, seed=31)
+@pytest.mark.parametrize("M,G", [(1, 128), (16, 32), (200, 128)])
+def test_asym_with_every_zero_eight_equals_the_symmetric_layer_bitwise(M, G):
+    """The symmetric call runs the same kernel (decode up to 32 tokens, the
+    pair kernel above); with all zeros 8 the dequantised values are identical,
+    hence Y too."""
+    p = W.make_problem(M, 2048, 416, G, seed=31)
     qz = np.full((p.scales.shape[0], p.N // 8), 0x88888888, dtype=np.uint32).view(np.int32)
     assert np.array_equal(run_asym(p, qz).view(np.uint16), run(p).view(np.uint16))
 
 
-@pytest.mark.parametrize("M", [1, 40, 300])
+@pytest.mark.parametrize("M", [1, 20, 40, 300])
 def test_asym_integer_exact_inputs_bitwise(M):
     rng = np.random.default_rng(M)
     p = W.make_problem(M, 2048, 160, 64, seed=M)
