@@ -1,31 +1,36 @@
-// Prefill kernel: Y[M, N] = X[M, K] . dequant(qweight, scales) for any M,
-// on the 5th-generation tensor cores (tcgen05) with TMEM accumulators.
+// Single-CTA prefill kernel: Y[M, N] = X[M, K] . dequant(qweight, scales) on
+// the 5th-generation tensor cores (tcgen05) with TMEM accumulators, and the
+// prefill dispatcher.
 //
 // Operation: GPTQ-Pro README, "Runtime contract" and "Ampere kernel
 // architecture" (tensor-core prefill with FP32 accumulation that reads the
 // native int32 qweight; predicated tails; FP16 output).  The Ampere design
-// (cp.async staging, mma.sync) is prior art only.  On sm_100a:
+// (cp.async staging, mma.sync) is prior art only.
+//
+// Above 32 tokens the dispatcher below sends every call to the persistent
+// CTA-pair kernel (prefill_pair.cu).  This kernel takes the prefill path at
+// M <= 32, which only a caller that forces the prefill kernel reaches (the
+// automatic choice there is the decode kernel); it runs 64-token tiles (the
+// template also builds 128 and 256):
 //
 // * The product is computed transposed, Y^T = W^T . X^T, so that the weights
 //   are the MMA's A operand (M = 128 weight columns per CTA) and the tokens are
-//   its N dimension (256 per CTA).  A comes from tensor memory: dequantisation
-//   warps unpack each int32 word (eight consecutive k of one column) into four
-//   32-bit TMEM cells of that column's lane, so dequantised weights never
-//   touch shared memory.
-// * One TMA producer thread streams, per 64-k stage, the X tile [256 tokens x
-//   64 k] (FP16, 128-byte swizzle: the B operand), the qweight tile [8 packed
-//   rows x 128 columns] and the scale rows of the stage; out-of-range rows and
-//   columns read as zero.  The dequantisation warps read their column's words
-//   and scales from shared memory at fixed offsets.
+//   its N dimension.  A comes from tensor memory: dequantisation warps unpack
+//   each int32 word (eight consecutive k of one column) into four 32-bit TMEM
+//   cells of that column's lane, so dequantised weights never touch shared
+//   memory.
+// * Producer threads stream, per 64-k stage, the X tile [BT tokens x 64 k]
+//   (FP16, 128-byte swizzle: the B operand), the qweight tile [8 packed rows x
+//   128 columns] and the scale rows of the stage; out-of-range rows and
+//   columns read as zero.
 // * One thread issues tcgen05.mma (kind::f16, FP32 accumulate) into a
-//   128 x 256 FP32 accumulator in TMEM; tcgen05.commit releases each stage.
+//   128 x BT FP32 accumulator in TMEM; tcgen05.commit releases each stage.
 // * The dequantisation warps then read the accumulator back (tcgen05.ld),
 //   round to FP16 and store Y.
 // * Every wait is bounded in time; on expiry the kernel records
 //   GPTQ_ERR_TIMEOUT in the device error word, drains its own copies and MMAs,
 //   frees TMEM and exits.  Nothing traps.
 //
-// Bytes per CTA tile: 128 x K / 2 (qweight) + scales + 256 x K x 2 (X, mostly from L2).
 // FLOPs per call: 2 M K N.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -42,7 +47,7 @@ namespace gptq {
 namespace {
 
 constexpr int BW = 128;  // weight columns per CTA (MMA M; one TMEM lane each)
-constexpr int BT_MAX = 256;  // tokens per CTA (MMA N): 64, 128 or 256, by M
+constexpr int BT_MAX = 256;  // tokens per CTA (MMA N): 64 in use, up to 256
 constexpr int BK = 64;   // k per pipeline stage (four k16 MMAs)
 constexpr int XS = 4;        // X ring stages (BT x 64 k each)
 constexpr int WS = 8;        // weight-tile ring stages (qweight + scales of 64 k)
