@@ -1,4 +1,4 @@
-"""B200-native (sm_100a) symmetric INT4 GPTQ W4A16 linear layer.
+"""B200-native (sm_100a) INT4 GPTQ W4A16 linear layer.
 
     Y[M, N] = X[M, K] . dequant(qweight[K/8, N], scales[n_groups, N])
 
@@ -9,9 +9,10 @@ and fails loudly if it is missing.
 """
 __version__ = "0.1.0"
 
-_BINDING_NAMES = {"gemm", "gemm_grouped", "gemm_asym", "gemm_lora", "gemm_lora_noalloc", "dequant", "select", "device_error", "version",
-                  "load", "GptqError", "KERNEL_AUTO", "KERNEL_DECODE", "KERNEL_PREFILL",
-                  "DECODE_MAX_M", "MAX_GROUPED", "MAX_LORA_RANK", "LORA_SCRATCH_BYTES", "GROUP_SIZES"}
+_BINDING_NAMES = {"gemm", "gemm_grouped", "gemm_asym", "gemm_lora", "gemm_lora_noalloc",
+                  "dequant", "select", "device_error", "version", "load", "GptqError",
+                  "KERNEL_AUTO", "KERNEL_DECODE", "KERNEL_PREFILL", "DECODE_MAX_M",
+                  "MAX_GROUPED", "MAX_LORA_RANK", "LORA_SCRATCH_BYTES", "GROUP_SIZES"}
 
 
 def __getattr__(name):
