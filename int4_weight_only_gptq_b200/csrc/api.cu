@@ -181,8 +181,11 @@ int lora_impl(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_lora_down(x, lora_a, t_work, M, K, rank, s, *dev);
   if (e == cudaSuccess)
-    e = launch_prefill_pair_lora(x, qweight, scales, y, M, K, N, group_shift_of(group), t_work,
-                                 lora_b, rank, s, *dev);
+    e = M <= GPTQ_DECODE_MAX_M
+            ? launch_decode_lora(x, qweight, scales, y, M, K, N, group_shift_of(group), t_work,
+                                 lora_b, rank, s, *dev)
+            : launch_prefill_pair_lora(x, qweight, scales, y, M, K, N, group_shift_of(group),
+                                       t_work, lora_b, rank, s, *dev);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return GPTQ_ERR_CUDA;

@@ -74,6 +74,10 @@ constexpr int DQ_WARPS = GROUPS * GROUP_WARPS;
 constexpr int THREADS = (2 + DQ_WARPS) * 32;
 constexpr int X_ATOMS = BKS / 64;
 constexpr int QW_STAGE_BYTES = PRS * BW * 4;
+// A LoRA stage's lora_b tile: 128 rows x 64 ranks (128-byte rows, 128-byte
+// swizzle) per half, two halves in the qweight area.
+constexpr int LORA_HALF_BYTES = BW * 64 * 2;
+static_assert(2 * LORA_HALF_BYTES <= QW_STAGE_BYTES, "a LoRA stage fits the qweight area");
 constexpr int S_ROW_BYTES = BW * 2;
 constexpr int Z_ROW_BYTES = BW / 8 * 4;  // one row of packed zero points (asymmetric weights)
 constexpr int kMaxStages = 8;
@@ -203,11 +207,21 @@ __device__ __forceinline__ void permute_x_chunk(uint8_t* p) {
 // ASYM: asymmetric weights (one linear): qz_map describes the packed zero
 // points [n_groups, N/8]; each stage holds their rows after the scales and
 // every column's zero replaces the 8 of the symmetric layer.
+// lora_rank > 0: a LoRA adapter (one linear; GPTQ-Pro README, "Runtime
+// contract": adapters on the linear path).  t_map describes T = fp16(X .
+// lora_a^T) [M, rank] and b_map lora_b [N, rank].  The last CTA of each
+// column block's split runs rank/128 more stages after its K stages: lora_b's
+// 128 rows x 128 ranks go to the qweight area (two 64-rank boxes, 128-byte
+// swizzle), T's rows to the X area (two 64-rank atoms); one fill per stage
+// copies lora_b into the A slot in the paired k order (T is permuted like X),
+// and the MMAs add T . lora_b^T to the same accumulators.
 template <int WPS, int BT, bool ASYM>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ LinearSet ls,
-                  const __grid_constant__ CUtensorMap qz_map, int M, int K, int group_shift,
-                  int stages, int stage_bytes, int scale_rows, int x3d, int* err) {
+                  const __grid_constant__ CUtensorMap qz_map,
+                  const __grid_constant__ CUtensorMap t_map,
+                  const __grid_constant__ CUtensorMap b_map, int M, int K, int group_shift,
+                  int stages, int stage_bytes, int scale_rows, int x3d, int lora_rank, int* err) {
   constexpr int X_ATOM_BYTES = TokGeo<BT>::X_ATOM_BYTES;
   constexpr int X_STAGE_BYTES = TokGeo<BT>::X_STAGE_BYTES;
   constexpr int QW_OFF = TokGeo<BT>::QW_OFF;
@@ -234,6 +248,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int st_begin = (int)((int64_t)blockIdx.y * NS / splits);
   const int st_end = (int)((int64_t)(blockIdx.y + 1) * NS / splits);
   const int n_st = st_end - st_begin;
+  // LoRA stages of this CTA (the last of the column block's split), then all
+  const int n_lora = (lora_rank > 0 && (int)blockIdx.y == splits - 1) ? (lora_rank + 127) / 128 : 0;
+  const int n_tot = n_st + n_lora;
   const int gs = min(group_shift, 30);        // group -1 (shift 62): row 0 throughout
   const int z_off = S_OFF + scale_rows * S_ROW_BYTES;  // zero-point rows (ASYM)
 
@@ -255,6 +272,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     prefetch_tensormap(qw_map);
     prefetch_tensormap(s_map);
     if (ASYM) prefetch_tensormap(&qz_map);
+    if (n_lora > 0) {
+      prefetch_tensormap(&t_map);
+      prefetch_tensormap(&b_map);
+    }
     // L2 prefetch of the first stages' weight tiles: safe before the wait
     const int pf = min(n_st, 2);
     for (int t = 0; t < pf; ++t) tma_prefetch_l2_2d(qw_map, n0, (st_begin + t) * PRS);
@@ -275,7 +296,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       int issued = 0;
       int s = 0;
       uint32_t ph = 0;
-      for (int t = 0; t < n_st; ++t) {
+      for (int t = 0; t < n_tot; ++t) {
         if (!mbar_wait_bounded(&bar->empty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
           record_timeout(err, bar);
           break;
@@ -287,6 +308,24 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         uint8_t* st = smem + s * stage_bytes;
+        if (t >= n_st) {
+          // LoRA stage: ranks 128 l .. 128 l + 127, as two 64-rank halves
+          // (a half wholly past the rank is neither loaded nor multiplied)
+          const int r0 = 128 * (t - n_st);
+          const uint32_t halves = r0 + 64 < lora_rank ? 2u : 1u;
+          mbar_arrive_expect_tx(&bar->full[s], halves * (LORA_HALF_BYTES + X_ATOM_BYTES));
+          for (uint32_t h = 0; h < halves; ++h) {
+            tma_load_2d(st + QW_OFF + h * LORA_HALF_BYTES, &b_map, r0 + 64 * (int)h, n0,
+                        &bar->full[s]);
+            tma_load_2d(st + h * X_ATOM_BYTES, &t_map, r0 + 64 * (int)h, 0, &bar->full[s]);
+          }
+          ++issued;
+          if (++s == stages) {
+            s = 0;
+            ph ^= 1u;
+          }
+          continue;
+        }
         const int k0 = (st_begin + t) * BKS;
         mbar_arrive_expect_tx(&bar->full[s],
                               X_STAGE_BYTES + QW_STAGE_BYTES +
@@ -327,9 +366,37 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool ok = true;
     int s = 0, a = 0;
     uint32_t ph = 0, aph = 0;
-    for (int t = 0; t < n_st && ok; ++t) {
+    for (int t = 0; t < n_tot && ok; ++t) {
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar->full[s], ph, abort_flag, kWaitLimitNs));
       const uint64_t x_desc = smem_desc_sw128(smem_u32(smem + s * stage_bytes));
+      if (t >= n_st) {
+        // LoRA stage: one fill, one k16 step per 16 ranks of the stage
+        if (ok)
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait_bounded(&bar->afull[a], aph, abort_flag, kWaitLimitNs));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a_base = tmem + A_COL0 + a * A_SLOT_COLS;
+        const int nk = min(128, lora_rank - 128 * (t - n_st)) / 16;
+        if (elect_one()) {
+          for (int kk = 0; kk < nk; ++kk)
+            mma_f16_ts(tmem + D_COL + (kk % NACC) * BT, a_base + 8 * kk,
+                       x_desc + (uint64_t)(((kk >> 2) * X_ATOM_BYTES + (kk & 3) * 32) >> 4),
+                       idesc, 1u);
+          mma_commit(&bar->aempty[a]);
+          mma_commit(&bar->empty[s]);
+        }
+        __syncwarp();
+        if (++a == A_SLOTS) {
+          a = 0;
+          aph ^= 1u;
+        }
+        if (++s == stages) {
+          s = 0;
+          ph ^= 1u;
+        }
+        continue;
+      }
 #pragma unroll
       for (int hf = 0; hf < HALVES; ++hf) {
         if (ok)
@@ -394,7 +461,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ring slot and phase of stage t, advanced incrementally (GROUPS <= stages)
     int s = grp % stages;
     uint32_t ph = (uint32_t)(grp / stages) & 1u;
-    for (int t = grp; t < n_st && ok; t += GROUPS, s += GROUPS) {
+    for (int t = grp; t < n_tot && ok; t += GROUPS, s += GROUPS) {
       if (s >= stages) {
         s -= stages;
         ph ^= 1u;
@@ -407,6 +474,54 @@ __global__ void __launch_bounds__(THREADS, 1)
       // does not matter); rows >= M are zero and stay so
       for (int j = gid; j < x_chunks; j += GROUP_WARPS * 32)
         permute_x_chunk(st + ((j & 63) >> 3) * X_ATOM_BYTES + (j >> 6) * 128 + (j & 7) * 16);
+
+      if (t >= n_st) {
+        // LoRA stage: one fill.  Row rho (eight ranks) of this slice's chunks
+        // comes from lora_b row `col` in the swizzled qweight area and is
+        // paired (k, k+4) like X and the dequantised weights.
+        const int f = HALVES * n_st + (t - n_st);
+        const int a = f % A_SLOTS;
+        const uint32_t aph = (uint32_t)(f / A_SLOTS) & 1u;
+#pragma unroll
+        for (int c = 0; c < CHUNKS; ++c) {
+          const int row0 = WPT * (CHUNKS * hs + c);
+          const bool mine = row0 < 128 / 8;  // the stage holds 128 ranks: 16 rows
+          uint32_t cells[4 * WPT];
+          if (mine) {
+#pragma unroll
+            for (int i = 0; i < WPT; ++i) {
+              const int rho = row0 + i;
+              const uint4 v = *reinterpret_cast<const uint4*>(
+                  st + QW_OFF + (rho >> 3) * LORA_HALF_BYTES + col * 128 +
+                  (((rho & 7) ^ (col & 7)) << 4));
+              cells[4 * i] = prmt(v.x, v.z, 0x5410);
+              cells[4 * i + 1] = prmt(v.x, v.z, 0x7632);
+              cells[4 * i + 2] = prmt(v.y, v.w, 0x5410);
+              cells[4 * i + 3] = prmt(v.y, v.w, 0x7632);
+            }
+          }
+          if (c == CHUNKS - 1) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->empty[s]);  // lora_b tile of the stage read
+          }
+          if (c == 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar->aempty[a], aph ^ 1u, abort_flag,
+                                                           kWaitLimitNs));
+            if (!ok) break;
+            tc_fence_after();
+          }
+          if (mine)
+            tmem_st_32x32b_x32(tmem + lane_addr + A_COL0 + a * A_SLOT_COLS +
+                                   4 * WPT * (CHUNKS * hs + c),
+                               cells);
+        }
+        if (!ok) break;
+        tmem_wait_st();
+        if (x_writer) fence_proxy_async_smem();  // the permuted T rows, for the MMAs
+        tc_fence_before();
+        mbar_arrive(&bar->afull[a]);
+        continue;
+      }
 
 #pragma unroll
       for (int hf = 0; hf < HALVES; ++hf) {
@@ -539,7 +654,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 template <int WPS, int BT, bool ASYM>
 cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtensorMap& qz_map,
-                     int M, int K, int group_shift, int splits, int x3d, const DecodeShape& d,
+                     const CUtensorMap& t_map, const CUtensorMap& b_map, int lora_rank, int M,
+                     int K, int group_shift, int splits, int x3d, const DecodeShape& d,
                      cudaStream_t stream, const DeviceInfo& dev) {
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
@@ -569,9 +685,9 @@ cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtens
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT, ASYM>, x_map, ls, qz_map, M, K,
-                            group_shift, d.stages, d.stage_bytes, d.scale_rows, x3d,
-                            dev.error_word);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT, ASYM>, x_map, ls, qz_map, t_map, b_map,
+                            M, K, group_shift, d.stages, d.stage_bytes, d.scale_rows, x3d,
+                            lora_rank, dev.error_word);
 }
 
 // One linear of a launch, as the host sees it.
@@ -584,14 +700,22 @@ struct LinearArgs {
 
 // Tensor maps and launch for a token tile of BT over `count` linears that
 // share X (count = 1 for a plain call).
-// qzeros: packed zero points of the (single) linear for asymmetric weights,
-// or nullptr.
+// The extras of a single linear: packed zero points for asymmetric weights,
+// and a LoRA adapter (t = fp16(x . lora_a^T) [M, rank], lora_b [N, rank]).
+struct LinearExtras {
+  const int32_t* qzeros = nullptr;
+  const uint16_t* t = nullptr;
+  const uint16_t* lora_b = nullptr;
+  int64_t rank = 0;
+};
+
 template <int BT>
-cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count, const int32_t* qzeros,
-                      int64_t M, int64_t K, int group_shift, int splits, cudaStream_t stream,
-                      const DeviceInfo& dev) {
+cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count,
+                      const LinearExtras& ex, int64_t M, int64_t K, int group_shift, int splits,
+                      cudaStream_t stream, const DeviceInfo& dev) {
+  const int32_t* qzeros = ex.qzeros;
   const bool asym = qzeros != nullptr;
-  if (asym && count != 1) return cudaErrorInvalidValue;
+  if ((asym || ex.rank > 0) && count != 1) return cudaErrorInvalidValue;
   const DecodeShape d = decode_shape<BT>(group_shift, asym);
   if (d.stages < GROUPS || d.smem_bytes > 1024 + kRingBudget + 256) return cudaErrorInvalidValue;
   if (count < 1 || count > kMaxLinears) return cudaErrorInvalidValue;
@@ -641,35 +765,46 @@ cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count, const
                        N / 2, BW / 8, (uint32_t)d.scale_rows, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
+  // LoRA: T [M, rank] as 64-rank atoms of BT rows (the X layout), lora_b
+  // [N, rank] as 64-rank halves of 128 rows; both with the 128-byte swizzle
+  CUtensorMap t_map = x_map, b_map = x_map;  // read only with an adapter
+  const int lora_rank = (int)ex.rank;
+  if (lora_rank > 0) {
+    const uint64_t N = (uint64_t)lin[0].n;
+    if (!tensor_map_2d(&t_map, ex.t, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)lora_rank,
+                       (uint64_t)M, (uint64_t)lora_rank * 2, 64, BT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !tensor_map_2d(&b_map, ex.lora_b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)lora_rank, N,
+                       (uint64_t)lora_rank * 2, 64, BW, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
   if (splits <= 0) splits = decode_pick_splits_blocks(ls.blk0[count], K, dev);
   const int iM = (int)M, iK = (int)K;
   if (asym) {
     if (group_shift == 4)
-      return launch_t<2, BT, true>(x_map, ls, qz_map, iM, iK, group_shift, splits, x3d, d, stream,
-                                   dev);
+      return launch_t<2, BT, true>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
+                                   group_shift, splits, x3d, d, stream, dev);
     if (group_shift == 5)
-      return launch_t<4, BT, true>(x_map, ls, qz_map, iM, iK, group_shift, splits, x3d, d, stream,
-                                   dev);
-    return launch_t<WPT, BT, true>(x_map, ls, qz_map, iM, iK, group_shift, splits, x3d, d, stream,
-                                   dev);
+      return launch_t<4, BT, true>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
+                                   group_shift, splits, x3d, d, stream, dev);
+    return launch_t<WPT, BT, true>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
+                                   group_shift, splits, x3d, d, stream, dev);
   }
   if (group_shift == 4)
-    return launch_t<2, BT, false>(x_map, ls, qz_map, iM, iK, group_shift, splits, x3d, d, stream,
-                                  dev);
+    return launch_t<2, BT, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
+                                  splits, x3d, d, stream, dev);
   if (group_shift == 5)
-    return launch_t<4, BT, false>(x_map, ls, qz_map, iM, iK, group_shift, splits, x3d, d, stream,
-                                  dev);
-  return launch_t<WPT, BT, false>(x_map, ls, qz_map, iM, iK, group_shift, splits, x3d, d, stream,
-                                  dev);
+    return launch_t<4, BT, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
+                                  splits, x3d, d, stream, dev);
+  return launch_t<WPT, BT, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
+                                  splits, x3d, d, stream, dev);
 }
 
 cudaError_t launch_set(const uint16_t* x, const LinearArgs* lin, int count,
-                       const int32_t* qzeros, int64_t M, int64_t K, int group_shift, int splits,
+                       const LinearExtras& ex, int64_t M, int64_t K, int group_shift, int splits,
                        cudaStream_t stream, const DeviceInfo& dev) {
   // token tile: 16 tokens up to M = 16, else 32
-  if (M <= 16)
-    return launch_bt<16>(x, lin, count, qzeros, M, K, group_shift, splits, stream, dev);
-  return launch_bt<32>(x, lin, count, qzeros, M, K, group_shift, splits, stream, dev);
+  if (M <= 16) return launch_bt<16>(x, lin, count, ex, M, K, group_shift, splits, stream, dev);
+  return launch_bt<32>(x, lin, count, ex, M, K, group_shift, splits, stream, dev);
 }
 
 }  // namespace
@@ -703,7 +838,7 @@ cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint1
                           uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
                           int splits, cudaStream_t stream, const DeviceInfo& dev) {
   const LinearArgs one{qweight, scales, y, N};
-  return launch_set(x, &one, 1, nullptr, M, K, group_shift, splits, stream, dev);
+  return launch_set(x, &one, 1, LinearExtras{}, M, K, group_shift, splits, stream, dev);
 }
 
 cudaError_t launch_decode_asym(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
@@ -711,7 +846,21 @@ cudaError_t launch_decode_asym(const uint16_t* x, const int32_t* qweight, const 
                                int64_t N, int group_shift, cudaStream_t stream,
                                const DeviceInfo& dev) {
   const LinearArgs one{qweight, scales, y, N};
-  return launch_set(x, &one, 1, qzeros, M, K, group_shift, 0, stream, dev);
+  LinearExtras ex;
+  ex.qzeros = qzeros;
+  return launch_set(x, &one, 1, ex, M, K, group_shift, 0, stream, dev);
+}
+
+cudaError_t launch_decode_lora(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                               uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
+                               const uint16_t* t, const uint16_t* lora_b, int64_t rank,
+                               cudaStream_t stream, const DeviceInfo& dev) {
+  const LinearArgs one{qweight, scales, y, N};
+  LinearExtras ex;
+  ex.t = t;
+  ex.lora_b = lora_b;
+  ex.rank = rank;
+  return launch_set(x, &one, 1, ex, M, K, group_shift, 0, stream, dev);
 }
 
 cudaError_t launch_decode_grouped(const uint16_t* x, const int32_t* const* qweights,
@@ -721,7 +870,7 @@ cudaError_t launch_decode_grouped(const uint16_t* x, const int32_t* const* qweig
   if (count < 1 || count > kMaxLinears) return cudaErrorInvalidValue;
   LinearArgs lin[kMaxLinears];
   for (int i = 0; i < count; ++i) lin[i] = LinearArgs{qweights[i], scales[i], ys[i], ns[i]};
-  return launch_set(x, lin, count, nullptr, M, K, group_shift, 0, stream, dev);
+  return launch_set(x, lin, count, LinearExtras{}, M, K, group_shift, 0, stream, dev);
 }
 
 }  // namespace gptq

@@ -45,6 +45,13 @@ cudaError_t launch_decode_asym(const uint16_t* x, const int32_t* qweight, const 
                                const int32_t* qzeros, uint16_t* y, int64_t M, int64_t K,
                                int64_t N, int group_shift, cudaStream_t stream,
                                const DeviceInfo& dev);
+// Decode with a LoRA adapter: t = fp16(x . lora_a^T) [M, rank] (from
+// launch_lora_down), lora_b [N, rank]; rank/128 extra stages in the last
+// split of each column block.
+cudaError_t launch_decode_lora(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                               uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
+                               const uint16_t* t, const uint16_t* lora_b, int64_t rank,
+                               cudaStream_t stream, const DeviceInfo& dev);
 // Decode of `count` linears that share X (1..GPTQ_MAX_GROUPED), one launch;
 // the split is picked from the total number of column blocks.
 cudaError_t launch_decode_grouped(const uint16_t* x, const int32_t* const* qweights,
