@@ -144,33 +144,48 @@ __global__ void __launch_bounds__(THREADS)
   }
 }
 
-// Up to 8 tokens: one warp per rank j, its lanes over 8-k chunks of the
-// CTA's k range (16-byte loads of lora_a and of each X row), per-token FP32
-// sums reduced across the warp by shuffles; the CTAs of a cluster split K
-// and rank 0 adds their sums in rank order.  No shared-memory staging and no
-// barrier per chunk: at these sizes the product is a few loads per lane.
-constexpr int SMALL_M = 8;
+// Up to 32 tokens: one warp per rank j.  The CTA's k range goes in pieces
+// of 256: the piece's X rows are staged in shared memory once (16-byte
+// loads by all threads), then lane l of each warp takes k chunk l of the
+// piece (eight values: one 16-byte load of lora_a, one 16-byte shared load
+// per token) into per-token FP32 sums, reduced across the warp by shuffles;
+// the CTAs of a cluster split K and rank 0 adds their sums in rank order.
+// Two barriers per 256 k, against two per 64 k in the tiled form.
+constexpr int SMALL_M = 32;
 constexpr int SMALL_WARPS = 8;  // ranks per CTA
+constexpr int PIECE = 256;      // k per staged piece: one 8-k chunk per lane
 
 template <int MB>  // token bound: M <= MB
 __global__ void __launch_bounds__(SMALL_WARPS * 32)
     lora_down_small_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a,
                            uint16_t* __restrict__ t, int M, int K, int r, int splits) {
+  __shared__ __align__(16) uint16_t xs[MB][PIECE];
   __shared__ float part[SMALL_WARPS][MB];
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x * SMALL_WARPS + warp;
   const int split = splits > 1 ? (int)cluster_ctarank() : 0;
-  const int chunks = K / 8;  // K is a multiple of 16
-  const int per = (chunks + splits - 1) / splits;
-  const int c_begin = split * per, c_end = min(chunks, c_begin + per);
+  const int pieces = (K + PIECE - 1) / PIECE;
+  const int per = (pieces + splits - 1) / splits;
+  const int p_begin = split * per, p_end = min(pieces, p_begin + per);
 
   float acc[MB];
 #pragma unroll
   for (int m = 0; m < MB; ++m) acc[m] = 0.0f;
-  if (j < r) {
-    for (int c = c_begin + lane; c < c_end; c += 32) {
-      const uint4 av = __ldg(reinterpret_cast<const uint4*>(a + (int64_t)j * K + 8 * c));
+  for (int pc = p_begin; pc < p_end; ++pc) {
+    const int k0 = pc * PIECE;
+    // stage the piece's X rows (zero outside M and K)
+    for (int i = threadIdx.x; i < MB * (PIECE / 8); i += SMALL_WARPS * 32) {
+      const int m = i / (PIECE / 8), c = i % (PIECE / 8);
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (m < M && k0 + 8 * c < K)
+        v = __ldg(reinterpret_cast<const uint4*>(x + (int64_t)m * K + k0 + 8 * c));
+      *reinterpret_cast<uint4*>(&xs[m][8 * c]) = v;
+    }
+    __syncthreads();
+    const int k = k0 + 8 * lane;
+    if (j < r && k < K) {
+      const uint4 av = __ldg(reinterpret_cast<const uint4*>(a + (int64_t)j * K + k));
       const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&av.x));
       const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&av.y));
       const float2 a2 = __half22float2(*reinterpret_cast<const __half2*>(&av.z));
@@ -178,24 +193,25 @@ __global__ void __launch_bounds__(SMALL_WARPS * 32)
 #pragma unroll
       for (int m = 0; m < MB; ++m) {
         if (m < M) {
-          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (int64_t)m * K + 8 * c));
+          const uint4 xv = *reinterpret_cast<const uint4*>(&xs[m][8 * lane]);
           const float2 x0 = __half22float2(*reinterpret_cast<const __half2*>(&xv.x));
           const float2 x1 = __half22float2(*reinterpret_cast<const __half2*>(&xv.y));
           const float2 x2 = __half22float2(*reinterpret_cast<const __half2*>(&xv.z));
           const float2 x3 = __half22float2(*reinterpret_cast<const __half2*>(&xv.w));
-          float s = acc[m];
-          s = fmaf(x0.x, a0.x, s);
-          s = fmaf(x0.y, a0.y, s);
-          s = fmaf(x1.x, a1.x, s);
-          s = fmaf(x1.y, a1.y, s);
-          s = fmaf(x2.x, a2.x, s);
-          s = fmaf(x2.y, a2.y, s);
-          s = fmaf(x3.x, a3.x, s);
-          s = fmaf(x3.y, a3.y, s);
-          acc[m] = s;
+          float sm = acc[m];
+          sm = fmaf(x0.x, a0.x, sm);
+          sm = fmaf(x0.y, a0.y, sm);
+          sm = fmaf(x1.x, a1.x, sm);
+          sm = fmaf(x1.y, a1.y, sm);
+          sm = fmaf(x2.x, a2.x, sm);
+          sm = fmaf(x2.y, a2.y, sm);
+          sm = fmaf(x3.x, a3.x, sm);
+          sm = fmaf(x3.y, a3.y, sm);
+          acc[m] = sm;
         }
       }
     }
+    __syncthreads();  // the piece is used before the next one is staged
   }
   // sums over the warp's lanes (fixed shuffle order), lane 0 keeps them
 #pragma unroll
@@ -231,7 +247,7 @@ cudaError_t launch_small(const uint16_t* x, const uint16_t* lora_a, uint16_t* t,
   const unsigned gr = (unsigned)((r + SMALL_WARPS - 1) / SMALL_WARPS);
   // split K over a cluster until the CTAs cover the SMs (at most 16)
   int splits = (int)std::min<int64_t>(kMaxSplits, std::max<int64_t>(1, dev.num_sms / gr));
-  splits = std::min<int>(splits, (int)std::max<int64_t>(1, K / 256));
+  splits = std::min<int>(splits, (int)std::max<int64_t>(1, (K + PIECE - 1) / PIECE));
   if (splits > 8) {
     static std::once_flag once[64];
     static cudaError_t attr_err[64];
@@ -261,9 +277,9 @@ cudaError_t launch_small(const uint16_t* x, const uint16_t* lora_a, uint16_t* t,
 
 cudaError_t launch_lora_down(const uint16_t* x, const uint16_t* lora_a, uint16_t* t, int64_t M,
                              int64_t K, int64_t r, cudaStream_t stream, const DeviceInfo& dev) {
-  // up to 8 tokens the per-lane form wins (measured: M = 1 rank 32, 5.5 us
-  // against 14 us); from 16 tokens on, X rows are better shared through
-  // shared memory by the tiled form
+  // up to 32 tokens the per-lane form (measured at M = 1, rank 32: 5.5 us
+  // against 14 us for the tiled form, which stalls on barriers there)
+  if (M <= 8) return launch_small<8>(x, lora_a, t, M, K, r, stream, dev);
   if (M <= SMALL_M) return launch_small<SMALL_M>(x, lora_a, t, M, K, r, stream, dev);
   const unsigned gm = (unsigned)((M + MT - 1) / MT), gr = (unsigned)((r + RT - 1) / RT);
   const int64_t tiles = (int64_t)gm * gr;
