@@ -2,17 +2,16 @@
 //
 // GPTQ-Pro README, "Runtime contract": adapters are LoRA on the linear path;
 // the adapter's own output is FP16 (its dtype), summed here in FP32.  T then
-// enters the prefill pair kernel as extra K of the layer's product
-// (prefill_pair.cu), where T . lora_b^T is added to the FP32 accumulator.
+// enters the decode kernel (up to 32 tokens) or the prefill pair kernel as
+// extra K of the layer's product, where T . lora_b^T is added to the FP32
+// accumulator.
 //
-// This product is at most rank/N of the layer's work (well under 1 % for the
-// usual ranks), so it runs on the FP32 cores: one CTA computes 32 tokens x 32
-// ranks, streaming 64-k chunks of X and lora_a through shared memory (as
-// FP32, with three chunks in flight in registers: at small M this product is
-// a few chunks per CTA, and memory latency, not arithmetic, sets its time).  When there are fewer tiles than twice the SMs, the CTAs of a
-// thread-block cluster (up to 16) split K and the partial sums are added in a
-// fixed order (rank 0, 1, ...) through distributed shared memory, so T is the
-// same on every call.
+// Two forms, both deterministic (fixed summation orders, no global scratch):
+// up to 32 tokens a per-lane form on the FP32 cores (one warp per rank; the
+// product is a few loads per lane there), above that the tensor cores
+// (tcgen05.mma with both operands from shared memory).  Either splits K over
+// a thread-block cluster when its tiles cannot fill the SMs and adds the
+// partial sums in rank order through distributed shared memory.
 
 #include <cuda_runtime.h>
 
@@ -21,128 +20,14 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc05.cuh"
+#include "tmap.h"
 
 namespace gptq {
 
 namespace {
 
-constexpr int MT = 32;           // tokens per CTA
-constexpr int RT = 32;           // ranks per CTA (one per lane)
-constexpr int KC = 64;           // k per shared-memory chunk
-constexpr int THREADS = 256;     // warp w: tokens 4w .. 4w+3; lane: one rank
-constexpr int TOK_PER_WARP = MT / (THREADS / 32);
-constexpr int A_ROW = KC + 4;    // padded FP32 row: 16-byte loads by 8 lanes hit 32 banks
-constexpr int WORDS = MT * KC / 2 / THREADS;  // 32-bit words of each chunk per thread
 constexpr int kMaxSplits = 16;
-constexpr int PF = 3;  // chunks in flight per thread
-static_assert(RT * KC / 2 / THREADS == WORDS, "X and lora_a chunks have the same size");
-
-// This thread's words of chunk c: X rows m0.., lora_a rows j0.. (zero outside
-// M, r and K).
-__device__ __forceinline__ void load_chunk(const uint16_t* __restrict__ x,
-                                           const uint16_t* __restrict__ a, int M, int K, int r,
-                                           int m0, int j0, int c, uint32_t (&xv)[WORDS],
-                                           uint32_t (&av)[WORDS]) {
-  const int k0 = c * KC;
-#pragma unroll
-  for (int u = 0; u < WORDS; ++u) {
-    const int i = threadIdx.x + u * THREADS;
-    const int row = i / (KC / 2), k = k0 + 2 * (i % (KC / 2));
-    const int m = m0 + row, j = j0 + row;
-    xv[u] = (m < M && k < K) ? __ldg(reinterpret_cast<const unsigned int*>(x + (int64_t)m * K + k))
-                             : 0u;
-    av[u] = (j < r && k < K) ? __ldg(reinterpret_cast<const unsigned int*>(a + (int64_t)j * K + k))
-                             : 0u;
-  }
-}
-
-__global__ void __launch_bounds__(THREADS)
-    lora_down_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a,
-                     uint16_t* __restrict__ t, int M, int K, int r, int splits) {
-  __shared__ __align__(16) float xs[MT][KC];     // X chunk in FP32
-  __shared__ __align__(16) float as[RT][A_ROW];  // lora_a chunk in FP32 (padded rows)
-  __shared__ float part[THREADS][TOK_PER_WARP];
-
-  // The layer launch that reads T may start now: it waits for this grid's
-  // completion before its first read of T, and every CTA of this grid is
-  // resident once all have passed this point, so the early start cannot keep
-  // any of them from an SM.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * MT, j0 = blockIdx.y * RT;
-  const int split = splits > 1 ? (int)cluster_ctarank() : 0;  // the cluster spans z
-  // this CTA's k range, whole chunks
-  const int chunks = (K + KC - 1) / KC;
-  const int per = (chunks + splits - 1) / splits;
-  const int c_begin = split * per, c_end = min(chunks, c_begin + per);
-
-  float acc[TOK_PER_WARP] = {};
-  // PF chunks in flight in registers: ring slot u holds chunk c_begin + u
-  // (mod PF); a slot is refilled as soon as its chunk is in shared memory
-  uint32_t xv[PF][WORDS], av[PF][WORDS];
-#pragma unroll
-  for (int u = 0; u < PF; ++u)
-    if (c_begin + u < c_end) load_chunk(x, a, M, K, r, m0, j0, c_begin + u, xv[u], av[u]);
-  for (int c0 = c_begin; c0 < c_end; c0 += PF) {
-#pragma unroll
-    for (int u = 0; u < PF; ++u) {
-      const int c = c0 + u;
-      if (c >= c_end) break;
-      // store chunk c (FP32), refill its slot with chunk c + PF, compute
-#pragma unroll
-      for (int w = 0; w < WORDS; ++w) {
-        const int i = threadIdx.x + w * THREADS;
-        const int row = i / (KC / 2), col2 = i % (KC / 2);
-        *reinterpret_cast<float2*>(&xs[row][2 * col2]) =
-            __half22float2(*reinterpret_cast<const __half2*>(&xv[u][w]));
-        *reinterpret_cast<float2*>(&as[row][2 * col2]) =
-            __half22float2(*reinterpret_cast<const __half2*>(&av[u][w]));
-      }
-      __syncthreads();
-      if (c + PF < c_end) load_chunk(x, a, M, K, r, m0, j0, c + PF, xv[u], av[u]);
-#pragma unroll 4
-      for (int k = 0; k < KC; k += 4) {
-        const float4 a4 = *reinterpret_cast<const float4*>(&as[lane][k]);
-#pragma unroll
-        for (int q = 0; q < TOK_PER_WARP; ++q) {
-          const float4 x4 = *reinterpret_cast<const float4*>(&xs[TOK_PER_WARP * warp + q][k]);
-          acc[q] = fmaf(x4.x, a4.x, acc[q]);
-          acc[q] = fmaf(x4.y, a4.y, acc[q]);
-          acc[q] = fmaf(x4.z, a4.z, acc[q]);
-          acc[q] = fmaf(x4.w, a4.w, acc[q]);
-        }
-      }
-      __syncthreads();
-    }
-  }
-
-  // partial sums of this CTA, then (split-K) the fixed-order sum over the
-  // cluster's CTAs in rank 0
-#pragma unroll
-  for (int q = 0; q < TOK_PER_WARP; ++q) part[threadIdx.x][q] = acc[q];
-  if (splits > 1) {
-    cluster_sync_all();  // every CTA's partial sums are in its shared memory
-    if (split == 0) {
-      const uint32_t mine = smem_u32(&part[threadIdx.x][0]);
-#pragma unroll
-      for (int q = 0; q < TOK_PER_WARP; ++q) acc[q] = 0.0f;
-      for (int s = 0; s < splits; ++s) {
-        const uint32_t addr = map_to_rank(mine, (uint32_t)s);
-#pragma unroll
-        for (int q = 0; q < TOK_PER_WARP; ++q) acc[q] += ld_dsmem_f32(addr + 4u * q);
-      }
-    }
-    cluster_sync_all();  // no CTA leaves while rank 0 reads its shared memory
-  }
-  if (split == 0) {
-    const int j = j0 + lane;
-#pragma unroll
-    for (int q = 0; q < TOK_PER_WARP; ++q) {
-      const int m = m0 + TOK_PER_WARP * warp + q;
-      if (m < M && j < r) t[(int64_t)m * r + j] = __half_as_ushort(__float2half_rn(acc[q]));
-    }
-  }
-}
 
 // Up to 32 tokens: one warp per rank j.  The CTA's k range goes in pieces
 // of 256: the piece's X rows are staged in shared memory once (16-byte
@@ -273,35 +158,259 @@ cudaError_t launch_small(const uint16_t* x, const uint16_t* lora_a, uint16_t* t,
                             (int)r, splits);
 }
 
-}  // namespace
+// Above 32 tokens: the tensor cores.  T^T [r, M] = lora_a . X^T with both
+// operands K-major FP16 tiles in shared memory (128-byte swizzle, by TMA):
+// one CTA computes 128 ranks x 128 tokens into an FP32 accumulator in TMEM
+// (tcgen05.mma, A and B from shared memory), 64 k per stage, four stages.
+// When the tiles cannot fill the SMs, the CTAs of a cluster split K: each
+// writes its tile to shared memory, and rank s adds rows s*128/S .. of every
+// rank's tile in rank order (distributed shared memory) and stores them.
+// One lane of a converged warp (the lowest active one) returns true.
+__device__ __forceinline__ bool elect_one_lane() {
+  uint32_t p = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(p));
+  return p != 0;
+}
 
-cudaError_t launch_lora_down(const uint16_t* x, const uint16_t* lora_a, uint16_t* t, int64_t M,
-                             int64_t K, int64_t r, cudaStream_t stream, const DeviceInfo& dev) {
-  // up to 32 tokens the per-lane form (measured at M = 1, rank 32: 5.5 us
-  // against 14 us for the tiled form, which stalls on barriers there)
-  if (M <= 8) return launch_small<8>(x, lora_a, t, M, K, r, stream, dev);
-  if (M <= SMALL_M) return launch_small<SMALL_M>(x, lora_a, t, M, K, r, stream, dev);
-  const unsigned gm = (unsigned)((M + MT - 1) / MT), gr = (unsigned)((r + RT - 1) / RT);
-  const int64_t tiles = (int64_t)gm * gr;
-  const int chunks = (int)((K + KC - 1) / KC);
-  // split K over a cluster when the tiles alone cannot fill the SMs twice
-  int splits = (int)std::min<int64_t>(kMaxSplits, std::max<int64_t>(1, 2 * dev.num_sms / tiles));
-  splits = std::min(splits, chunks);
-  if (splits > 8) {
-    // clusters above the portable size of 8 have to be allowed per kernel
-    static std::once_flag once[64];
-    static cudaError_t attr_err[64];
-    const int d = dev.device & 63;
-    std::call_once(once[d], [&] {
-      attr_err[d] = cudaFuncSetAttribute(lora_down_kernel,
-                                         cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    });
-    if (attr_err[d] != cudaSuccess) splits = 8;
+constexpr int TC_R = 128;    // ranks per CTA (MMA M; ranks past r read as zero)
+constexpr int TC_T = 128;    // tokens per CTA (MMA N)
+constexpr int TC_BK = 64;    // k per stage
+constexpr int TC_STAGES = 4;
+constexpr int TC_A_BYTES = TC_R * TC_BK * 2;
+constexpr int TC_B_BYTES = TC_T * TC_BK * 2;
+constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES;
+constexpr int TC_THREADS = 192;  // warp 0: copies, warp 1: MMAs and TMEM, warps 2..5: read-out
+constexpr int TC_RED_ROW = TC_T + 4;  // FP32 reduction rows, padded (16-byte stores, no conflicts)
+constexpr int kTcMaxSplits = 8;
+constexpr uint64_t kTcWaitNs = 4000000000ull;
+constexpr uint64_t kTcDrainNs = 200000000ull;
+static_assert(TC_R * TC_RED_ROW * 4 <= TC_STAGES * TC_STAGE_BYTES, "reduction tile fits the ring");
+
+struct TcBars {
+  uint64_t full[TC_STAGES];
+  uint64_t empty[TC_STAGES];
+  uint64_t dfull;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    lora_down_tc_kernel(const __grid_constant__ CUtensorMap a_map,
+                        const __grid_constant__ CUtensorMap x_map, uint16_t* __restrict__ t,
+                        int M, int K, int r, int splits, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  TcBars* bar = reinterpret_cast<TcBars*>(smem + TC_STAGES * TC_STAGE_BYTES);
+  volatile int* abort_flag = &bar->abort_flag;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = splits > 1 ? (int)cluster_ctarank() : 0;
+  const int t0 = blockIdx.x * TC_T, j0 = blockIdx.y * TC_R;
+  const int KB = (K + TC_BK - 1) / TC_BK;
+  // balanced split of the k stages: every CTA gets at least one (splits <=
+  // KB), so every accumulator is written by its first MMA before it is read
+  const int kb0 = (int)((int64_t)split * KB / splits);
+  const int kb1 = (int)((int64_t)(split + 1) * KB / splits);
+  const int n = kb1 - kb0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < TC_STAGES; ++s) {
+      mbar_init(&bar->full[s], 1);
+      mbar_init(&bar->empty[s], 1);
+    }
+    mbar_init(&bar->dfull, 1);
+    bar->abort_flag = 0;
+    fence_mbarrier_init();
   }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&a_map);
+    prefetch_tensormap(&x_map);
+  }
+  __syncwarp();
+  if (warp == 1) {
+    tmem_alloc(&bar->tmem_base, TC_T);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0, issued = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < n; ++i) {
+        if (!mbar_wait_bounded(&bar->empty[s], ph ^ 1u, abort_flag, kTcWaitNs)) {
+          atomicExch(err, kDeviceErrTimeout);
+          *abort_flag = 1;
+          break;
+        }
+        uint8_t* st = smem + s * TC_STAGE_BYTES;
+        const int k0 = (kb0 + i) * TC_BK;
+        mbar_arrive_expect_tx(&bar->full[s], TC_STAGE_BYTES);
+        tma_load_2d(st, &a_map, k0, j0, &bar->full[s]);
+        tma_load_2d(st + TC_A_BYTES, &x_map, k0, t0, &bar->full[s]);
+        ++issued;
+        if (++s == TC_STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (*abort_flag) {
+        int never = 0;
+        for (int j = issued - 1; j >= 0 && j >= issued - TC_STAGES; --j)
+          mbar_wait_bounded(&bar->full[j % TC_STAGES], (uint32_t)(j / TC_STAGES) & 1u, &never,
+                            kTcDrainNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    const uint32_t idesc = idesc_f16_f32(TC_R, TC_T);
+    bool ok = true;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int i = 0; i < n && ok; ++i) {
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_bounded(&bar->full[s], ph, abort_flag, kTcWaitNs));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t st = smem_u32(smem + s * TC_STAGE_BYTES);
+      const uint64_t a_desc = smem_desc_sw128(st), b_desc = smem_desc_sw128(st + TC_A_BYTES);
+      if (elect_one_lane()) {
+#pragma unroll
+        for (int kk = 0; kk < TC_BK / 16; ++kk)
+          mma_f16_ss(tmem, a_desc + (uint64_t)((kk * 32) >> 4), b_desc + (uint64_t)((kk * 32) >> 4),
+                     idesc, (i | kk) != 0 ? 1u : 0u);
+        mma_commit(&bar->empty[s]);
+      }
+      __syncwarp();
+      if (++s == TC_STAGES) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+    if (!ok && lane == 0) {
+      atomicExch(err, kDeviceErrTimeout);
+      *abort_flag = 1;
+    }
+    if (elect_one_lane()) mma_commit(&bar->dfull);
+    __syncwarp();
+  }
+
+  // read-out: warps 2..5, TMEM lane quarter warp % 4 (ranks j0 + 32q + lane)
+  const bool reader = warp >= 2;
+  const int q = warp & 3;
+  const int j = j0 + 32 * q + lane;
+  float* red = reinterpret_cast<float*>(smem);  // the ring is free once dfull completes
+  bool ok = true;
+  if (reader) {
+    ok = __all_sync(0xffffffffu, mbar_wait_bounded<true>(&bar->dfull, 0, abort_flag, kTcWaitNs));
+    if (!ok && lane == 0) {
+      atomicExch(err, kDeviceErrTimeout);
+      *abort_flag = 1;
+    }
+  }
+  if (reader && ok) {
+    tc_fence_after();
+#pragma unroll 1
+    for (int c = 0; c < TC_T / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + 32 * c, v);
+      tmem_wait_ld();
+      if (splits == 1) {
+        if (j < r) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int tok = t0 + 32 * c + i;
+            if (tok < M)
+              t[(int64_t)tok * r + j] = __half_as_ushort(__float2half_rn(__uint_as_float(v[i])));
+          }
+        }
+      } else {
+        float* row = red + (32 * q + lane) * TC_RED_ROW + 32 * c;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(row + i) =
+              make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                          __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+      }
+    }
+  }
+  if (splits > 1) {
+    cluster_sync_all();  // every CTA's partial tile is in its shared memory
+    if (reader) {
+      // rank `split` adds rows split*RS .. of all ranks' tiles: thread i of
+      // the 128 readers takes row split*RS + i / (128/RS), 128/(128/RS)
+      // consecutive tokens of it
+      const int RS = TC_R / splits;                 // rows per rank
+      const int tpr = (TC_THREADS - 64) / RS;       // threads per row
+      const int tid = threadIdx.x - 64;
+      const int row = split * RS + tid / tpr;
+      const int tw = TC_T / tpr;                    // tokens per thread
+      const int tk0 = (tid % tpr) * tw;
+      const int jr = j0 + row;
+      for (int c = 0; c < tw; c += 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const uint32_t addr = smem_u32(red + row * TC_RED_ROW + tk0 + c);
+        for (int sp = 0; sp < splits; ++sp) {
+          const uint32_t ra = map_to_rank(addr, (uint32_t)sp);
+          acc.x += ld_dsmem_f32(ra);
+          acc.y += ld_dsmem_f32(ra + 4);
+          acc.z += ld_dsmem_f32(ra + 8);
+          acc.w += ld_dsmem_f32(ra + 12);
+        }
+        const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int tok = t0 + tk0 + c + u;
+          if (jr < r && tok < M)
+            t[(int64_t)tok * r + jr] = __half_as_ushort(__float2half_rn(vals[u]));
+        }
+      }
+    }
+    cluster_sync_all();  // no CTA leaves while another reads its shared memory
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TC_T);
+  }
+}
+
+cudaError_t launch_tc(const uint16_t* x, const uint16_t* lora_a, uint16_t* t, int64_t M,
+                      int64_t K, int64_t r, cudaStream_t stream, const DeviceInfo& dev) {
+  CUtensorMap a_map, x_map;
+  if (!tensor_map_2d(&a_map, lora_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)r,
+                     (uint64_t)K * 2, TC_BK, TC_R, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tensor_map_2d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M,
+                     (uint64_t)K * 2, TC_BK, TC_T, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  const unsigned gm = (unsigned)((M + TC_T - 1) / TC_T), gr = (unsigned)((r + TC_R - 1) / TC_R);
+  const int64_t tiles = (int64_t)gm * gr;
+  const int64_t kb = (K + TC_BK - 1) / TC_BK;
+  // a power-of-two K split (the reduction shares the 128 rows evenly) while
+  // the tiles cannot fill the SMs
+  int splits = 1;
+  while (splits * 2 <= kTcMaxSplits && tiles * splits * 2 <= dev.num_sms && splits * 2 <= kb)
+    splits *= 2;
+  constexpr size_t smem = 1024 + (size_t)TC_STAGES * TC_STAGE_BYTES + 256;
+  static std::once_flag once[64];
+  static cudaError_t attr_err[64];
+  const int d = dev.device & 63;
+  std::call_once(once[d], [&] {
+    attr_err[d] = cudaFuncSetAttribute(lora_down_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  });
+  if (attr_err[d] != cudaSuccess) return attr_err[d];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(gm, gr, (unsigned)splits);
-  cfg.blockDim = dim3(THREADS, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.blockDim = dim3(TC_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -310,7 +419,20 @@ cudaError_t launch_lora_down(const uint16_t* x, const uint16_t* lora_a, uint16_t
   attr[0].val.clusterDim.z = (unsigned)splits;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, lora_down_kernel, x, lora_a, t, (int)M, (int)K, (int)r, splits);
+  return cudaLaunchKernelEx(&cfg, lora_down_tc_kernel, a_map, x_map, t, (int)M, (int)K, (int)r,
+                            splits, dev.error_word);
+}
+
+}  // namespace
+
+cudaError_t launch_lora_down(const uint16_t* x, const uint16_t* lora_a, uint16_t* t, int64_t M,
+                             int64_t K, int64_t r, cudaStream_t stream, const DeviceInfo& dev) {
+  // up to 32 tokens the per-lane form on the FP32 cores (at M = 1, rank 32:
+  // 5.5 us, against 14 us for an FP32 form with shared-memory tiles, which
+  // stalled on barriers there); above, the tensor cores
+  if (M <= 8) return launch_small<8>(x, lora_a, t, M, K, r, stream, dev);
+  if (M <= SMALL_M) return launch_small<SMALL_M>(x, lora_a, t, M, K, r, stream, dev);
+  return launch_tc(x, lora_a, t, M, K, r, stream, dev);
 }
 
 }  // namespace gptq
