@@ -778,6 +778,13 @@ cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count,
       return cudaErrorInvalidValue;
   }
   if (splits <= 0) splits = decode_pick_splits_blocks(ls.blk0[count], K, dev);
+  // with an adapter, the last split's CTA (which runs the LoRA stages after
+  // its K stages) must own at least one K stage: the first MMAs of its K
+  // stages are what initialise its accumulators
+  if (lora_rank > 0) {
+    const int ns = (int)(((K >> 3) + PRS - 1) / PRS);
+    if (splits > ns) splits = ns;
+  }
   const int iM = (int)M, iK = (int)K;
   if (asym) {
     if (group_shift == 4)
