@@ -173,20 +173,6 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32
                : "memory");
 }
 
-// One lane of a converged warp (the lowest active one) returns true.
-__device__ __forceinline__ bool elect_one() {
-  uint32_t p = 0;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}"
-      : "=r"(p));
-  return p != 0;
-}
-
-__device__ __forceinline__ void record_timeout(int* err, DecodeBars* b) {
-  atomicExch(err, kDeviceErrTimeout);
-  *reinterpret_cast<volatile int*>(&b->abort_flag) = 1;
-}
-
 // One 16-byte chunk of an X row (eight consecutive k) rewritten in place from
 // natural order (x0 .. x7) to the paired order of the unpacked weights:
 // (x0, x4), (x1, x5), (x2, x6), (x3, x7).

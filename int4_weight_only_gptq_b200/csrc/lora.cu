@@ -165,15 +165,6 @@ cudaError_t launch_small(const uint16_t* x, const uint16_t* lora_a, uint16_t* t,
 // When the tiles cannot fill the SMs, the CTAs of a cluster split K: each
 // writes its tile to shared memory, and rank s adds rows s*128/S .. of every
 // rank's tile in rank order (distributed shared memory) and stores them.
-// One lane of a converged warp (the lowest active one) returns true.
-__device__ __forceinline__ bool elect_one_lane() {
-  uint32_t p = 0;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}"
-      : "=r"(p));
-  return p != 0;
-}
-
 constexpr int TC_R = 128;    // ranks per CTA (MMA M; ranks past r read as zero)
 constexpr int TC_T = 128;    // tokens per CTA (MMA N)
 constexpr int TC_BK = 64;    // k per stage
@@ -245,8 +236,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t ph = 0;
       for (int i = 0; i < n; ++i) {
         if (!mbar_wait_bounded(&bar->empty[s], ph ^ 1u, abort_flag, kTcWaitNs)) {
-          atomicExch(err, kDeviceErrTimeout);
-          *abort_flag = 1;
+          record_timeout(err, bar);
           break;
         }
         uint8_t* st = smem + s * TC_STAGE_BYTES;
@@ -280,7 +270,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_after();
       const uint32_t st = smem_u32(smem + s * TC_STAGE_BYTES);
       const uint64_t a_desc = smem_desc_sw128(st), b_desc = smem_desc_sw128(st + TC_A_BYTES);
-      if (elect_one_lane()) {
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < TC_BK / 16; ++kk)
           mma_f16_ss(tmem, a_desc + (uint64_t)((kk * 32) >> 4), b_desc + (uint64_t)((kk * 32) >> 4),
@@ -294,10 +284,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
     }
     if (!ok && lane == 0) {
-      atomicExch(err, kDeviceErrTimeout);
-      *abort_flag = 1;
+      record_timeout(err, bar);
     }
-    if (elect_one_lane()) mma_commit(&bar->dfull);
+    if (elect_one()) mma_commit(&bar->dfull);
     __syncwarp();
   }
 
@@ -310,8 +299,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   if (reader) {
     ok = __all_sync(0xffffffffu, mbar_wait_bounded<true>(&bar->dfull, 0, abort_flag, kTcWaitNs));
     if (!ok && lane == 0) {
-      atomicExch(err, kDeviceErrTimeout);
-      *abort_flag = 1;
+      record_timeout(err, bar);
     }
   }
   if (reader && ok) {

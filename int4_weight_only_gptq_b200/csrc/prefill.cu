@@ -93,20 +93,6 @@ struct Barriers {
 };
 static_assert(sizeof(Barriers) <= 512, "barrier area");
 
-__device__ __forceinline__ void record_timeout(int* err, Barriers* b) {
-  atomicExch(err, kDeviceErrTimeout);
-  *reinterpret_cast<volatile int*>(&b->abort_flag) = 1;
-}
-
-// One lane of a converged warp (the lowest active one) returns true.
-__device__ __forceinline__ bool elect_one() {
-  uint32_t p = 0;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}"
-      : "=r"(p));
-  return p != 0;
-}
-
 // scale_rows: scale rows one 64-k stage touches (1, or 64/group for groups
 // below 64); stages start on 64-k boundaries, so they align with groups.
 //

@@ -144,20 +144,6 @@ struct PairBarriers {
 };
 static_assert(sizeof(PairBarriers) <= 512, "barrier area");
 
-__device__ __forceinline__ void record_timeout(int* err, PairBarriers* b) {
-  atomicExch(err, kDeviceErrTimeout);
-  *reinterpret_cast<volatile int*>(&b->abort_flag) = 1;
-}
-
-// One lane of a converged warp (the lowest active one) returns true.
-__device__ __forceinline__ bool elect_one() {
-  uint32_t p = 0;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}"
-      : "=r"(p));
-  return p != 0;
-}
-
 // The tiles of one cluster: tile = cluster + i * clusters for i = 0, 1, ...;
 // column pair fastest.
 struct TileWalk {

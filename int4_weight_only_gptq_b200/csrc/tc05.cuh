@@ -6,8 +6,26 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "kernels.h"
 
 namespace gptq {
+
+// One lane of a converged warp (the lowest active one) returns true.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(p));
+  return p != 0;
+}
+
+// Records a wait that gave up: the timeout code in the device error word, and
+// the CTA's abort flag, so that its other roles stop waiting.
+template <class Bars>
+__device__ __forceinline__ void record_timeout(int* err, Bars* b) {
+  atomicExch(err, kDeviceErrTimeout);
+  *reinterpret_cast<volatile int*>(&b->abort_flag) = 1;
+}
 
 // ---- time-bounded mbarrier wait ----------------------------------------------
 
