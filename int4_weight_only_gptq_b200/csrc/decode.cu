@@ -37,8 +37,12 @@
 // * Programmatic dependent launch: before waiting for the previous kernel in
 //   the stream, the producer only prefetches its first weight tiles into L2 (a
 //   prefetch cannot observe stale data); every copy into shared memory and
-//   every store of Y happens after the wait.  Once it has issued its last
-//   copy, the producer lets the next kernel in the stream begin its prologue.
+//   every store of Y happens after the wait.  With a LoRA adapter the previous
+//   launch is the one computing T, which is launched without this attribute
+//   (it starts after all earlier work completed): then only the first read of
+//   T waits, and the K stages overlap that launch.  Once it has issued its
+//   last copy, the producer lets the next kernel in the stream begin its
+//   prologue.
 // * Every wait is bounded in time; on expiry the kernel records
 //   GPTQ_ERR_TIMEOUT in the device error word, drains its own copies and MMAs,
 //   frees TMEM and exits.  Nothing traps.
@@ -274,7 +278,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
-  grid_dependency_wait();
+  // Without an adapter the previous kernel in the stream may still be running
+  // and may write X: every thread waits for it here.  With one, the previous
+  // launch computes T and itself started only after all earlier work had
+  // completed, so X, the weights and Y are safe now and only the producer's
+  // first read of T waits for that launch (below).
+  if (lora_rank == 0) grid_dependency_wait();
 
   if (warp == 0) {
     // ---------------- TMA producer (one lane) ----------------
@@ -282,6 +291,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       int issued = 0;
       int s = 0;
       uint32_t ph = 0;
+      bool t_waited = false;
       for (int t = 0; t < n_tot; ++t) {
         if (!mbar_wait_bounded(&bar->empty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
           record_timeout(err, bar);
@@ -297,6 +307,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (t >= n_st) {
           // LoRA stage: ranks 128 l .. 128 l + 127, as two 64-rank halves
           // (a half wholly past the rank is neither loaded nor multiplied)
+          if (t == n_st) {
+            grid_dependency_wait();  // T is complete and visible
+            t_waited = true;
+          }
           const int r0 = 128 * (t - n_st);
           const uint32_t halves = r0 + 64 < lora_rank ? 2u : 1u;
           mbar_arrive_expect_tx(&bar->full[s], halves * (LORA_HALF_BYTES + X_ATOM_BYTES));
@@ -339,6 +353,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           mbar_wait_bounded(&bar->full[j % stages], (uint32_t)(j / stages) & 1u, &never,
                             kDrainLimitNs);
       }
+      // a CTA with adapter stages completes only after the launch computing T
+      // (so this grid's completion implies T's, also when it gave up early)
+      if (n_lora > 0 && !t_waited) grid_dependency_wait();
       // all of this CTA's copies are issued: the next kernel in the stream may
       // start its prologue (it waits for this grid before touching its inputs)
       allow_dependent_launch();
@@ -825,6 +842,10 @@ int decode_pick_splits_blocks(int64_t nblk, int64_t K, const DeviceInfo& dev) {
 int decode_pick_splits(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev) {
   (void)M;
   return decode_pick_splits_blocks((N + BW - 1) / BW, K, dev);
+}
+
+int64_t decode_ctas(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev) {
+  return (N + BW - 1) / BW * decode_pick_splits(M, K, N, dev);
 }
 
 cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,

@@ -84,7 +84,12 @@ cudaError_t launch_prefill_pair_asym(const uint16_t* x, const int32_t* qweight,
                                      int64_t M, int64_t K, int64_t N, int group_shift,
                                      cudaStream_t stream, const DeviceInfo& dev);
 // t [M, r] = fp16(x . lora_a^T), lora_a [r, K] (the adapter's down-projection).
+// free_sms: SMs that the layer's launch after it leaves unused (0 if none or
+// unknown); up to 32 tokens the launch stays on them when it can.
 cudaError_t launch_lora_down(const uint16_t* x, const uint16_t* lora_a, uint16_t* t, int64_t M,
-                             int64_t K, int64_t r, cudaStream_t stream, const DeviceInfo& dev);
+                             int64_t K, int64_t r, int free_sms, cudaStream_t stream,
+                             const DeviceInfo& dev);
+// CTAs of one decode launch of this shape (column blocks x K split).
+int64_t decode_ctas(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev);
 
 }  // namespace gptq

@@ -12,6 +12,12 @@
 // (tcgen05.mma with both operands from shared memory).  Either splits K over
 // a thread-block cluster when its tiles cannot fill the SMs and adds the
 // partial sums in rank order through distributed shared memory.
+//
+// Stream order: both forms are launched WITHOUT programmatic stream
+// serialisation, so they start only after every earlier kernel in the stream
+// has completed, and each lets its dependent start at once.  The layer's
+// launch that follows relies on this: it reads X and the weights without
+// waiting and waits for this grid only before its first read of T.
 
 #include <cuda_runtime.h>
 
@@ -29,21 +35,114 @@ namespace {
 
 constexpr int kMaxSplits = 16;
 
-// Up to 32 tokens: one warp per rank j.  The CTA's k range goes in pieces
-// of 256: the piece's X rows are staged in shared memory once (16-byte
-// loads by all threads), then lane l of each warp takes k chunk l of the
-// piece (eight values: one 16-byte load of lora_a, one 16-byte shared load
-// per token) into per-token FP32 sums, reduced across the warp by shuffles;
-// the CTAs of a cluster split K and rank 0 adds their sums in rank order.
-// Two barriers per 256 k, against two per 64 k in the tiled form.
+// Up to 32 tokens: one warp per rank j, lane l taking 8-k chunk l of every
+// 256-k piece of the CTA's k range (one 16-byte load of lora_a, one 16-byte
+// load of X per token) into per-token FP32 sums, reduced across the warp by
+// shuffles; the CTAs of a cluster split K and rank 0 adds their sums in rank
+// order.  Two forms of the loop:
+//  * up to 8 tokens (lanes form) X is read straight through L1 and the loop
+//    has no barriers, so the loads of successive pieces overlap and a CTA
+//    gets through its range in a few memory latencies even when only a few
+//    CTAs run (launch_small);
+//  * up to 32 tokens (staged form) each piece's X rows are staged in shared
+//    memory once by all threads, two barriers per piece.
 constexpr int SMALL_M = 32;
+constexpr int LANES_M = 8;
 constexpr int SMALL_WARPS = 8;  // ranks per CTA
-constexpr int PIECE = 256;      // k per staged piece: one 8-k chunk per lane
+constexpr int PIECE = 256;      // k per piece: one 8-k chunk per lane
 
-template <int MB>  // token bound: M <= MB
+// The common end of both forms: sums over the warp's lanes (fixed shuffle
+// order), then over the cluster's CTAs in rank order in rank 0, then T.
+template <int MB>
+__device__ __forceinline__ void small_finish(float (&acc)[MB], float (*part)[MB], uint16_t* t,
+                                             int M, int r, int split, int splits) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int m = 0; m < MB; ++m) {
+    float v = acc[m];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+    if (lane == 0) part[warp][m] = v;
+  }
+  __syncthreads();
+  // thread (w, m)
+  const int w = threadIdx.x / MB, m = threadIdx.x % MB;
+  const bool mine = threadIdx.x < SMALL_WARPS * MB;
+  float sum = 0.0f;
+  if (splits > 1) {
+    cluster_sync_all();
+    if (split == 0 && mine) {
+      const uint32_t addr = smem_u32(&part[w][m]);
+      for (int sp = 0; sp < splits; ++sp) sum += ld_dsmem_f32(map_to_rank(addr, (uint32_t)sp));
+    }
+    cluster_sync_all();  // no CTA leaves while rank 0 reads its shared memory
+  } else if (mine) {
+    sum = part[w][m];
+  }
+  const int jj = blockIdx.x * SMALL_WARPS + w;
+  if (split == 0 && mine && m < M && jj < r)
+    t[(int64_t)m * r + jj] = __half_as_ushort(__float2half_rn(sum));
+}
+
+__device__ __forceinline__ void fma8(float& sm, const uint4 xv, const float2 a0, const float2 a1,
+                                     const float2 a2, const float2 a3) {
+  const float2 x0 = __half22float2(*reinterpret_cast<const __half2*>(&xv.x));
+  const float2 x1 = __half22float2(*reinterpret_cast<const __half2*>(&xv.y));
+  const float2 x2 = __half22float2(*reinterpret_cast<const __half2*>(&xv.z));
+  const float2 x3 = __half22float2(*reinterpret_cast<const __half2*>(&xv.w));
+  sm = fmaf(x0.x, a0.x, sm);
+  sm = fmaf(x0.y, a0.y, sm);
+  sm = fmaf(x1.x, a1.x, sm);
+  sm = fmaf(x1.y, a1.y, sm);
+  sm = fmaf(x2.x, a2.x, sm);
+  sm = fmaf(x2.y, a2.y, sm);
+  sm = fmaf(x3.x, a3.x, sm);
+  sm = fmaf(x3.y, a3.y, sm);
+}
+
+// Lanes form, M <= LANES_M.
 __global__ void __launch_bounds__(SMALL_WARPS * 32)
-    lora_down_small_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a,
+    lora_down_lanes_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a,
                            uint16_t* __restrict__ t, int M, int K, int r, int splits) {
+  __shared__ float part[SMALL_WARPS][LANES_M];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x * SMALL_WARPS + warp;
+  const int split = splits > 1 ? (int)cluster_ctarank() : 0;
+  const int pieces = (K + PIECE - 1) / PIECE;
+  // balanced: every split gets at least one piece (splits <= pieces)
+  const int p_begin = split * pieces / splits, p_end = (split + 1) * pieces / splits;
+
+  float acc[LANES_M];
+#pragma unroll
+  for (int m = 0; m < LANES_M; ++m) acc[m] = 0.0f;
+  if (j < r) {
+    const uint16_t* __restrict__ arow = a + (int64_t)j * K;
+#pragma unroll 4
+    for (int pc = p_begin; pc < p_end; ++pc) {
+      const int k = pc * PIECE + 8 * lane;
+      if (k < K) {  // K % 8 == 0: the chunk is whole
+        const uint4 av = __ldg(reinterpret_cast<const uint4*>(arow + k));
+        const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&av.x));
+        const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&av.y));
+        const float2 a2 = __half22float2(*reinterpret_cast<const __half2*>(&av.z));
+        const float2 a3 = __half22float2(*reinterpret_cast<const __half2*>(&av.w));
+#pragma unroll
+        for (int m = 0; m < LANES_M; ++m)
+          if (m < M)
+            fma8(acc[m], __ldg(reinterpret_cast<const uint4*>(x + (int64_t)m * K + k)), a0, a1,
+                 a2, a3);
+      }
+    }
+  }
+  small_finish<LANES_M>(acc, part, t, M, r, split, splits);
+}
+
+// Staged form, M <= SMALL_M.
+__global__ void __launch_bounds__(SMALL_WARPS * 32)
+    lora_down_staged_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a,
+                            uint16_t* __restrict__ t, int M, int K, int r, int splits) {
+  constexpr int MB = SMALL_M;
   __shared__ __align__(16) uint16_t xs[MB][PIECE];
   __shared__ float part[SMALL_WARPS][MB];
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -76,72 +175,35 @@ __global__ void __launch_bounds__(SMALL_WARPS * 32)
       const float2 a2 = __half22float2(*reinterpret_cast<const __half2*>(&av.z));
       const float2 a3 = __half22float2(*reinterpret_cast<const __half2*>(&av.w));
 #pragma unroll
-      for (int m = 0; m < MB; ++m) {
-        if (m < M) {
-          const uint4 xv = *reinterpret_cast<const uint4*>(&xs[m][8 * lane]);
-          const float2 x0 = __half22float2(*reinterpret_cast<const __half2*>(&xv.x));
-          const float2 x1 = __half22float2(*reinterpret_cast<const __half2*>(&xv.y));
-          const float2 x2 = __half22float2(*reinterpret_cast<const __half2*>(&xv.z));
-          const float2 x3 = __half22float2(*reinterpret_cast<const __half2*>(&xv.w));
-          float sm = acc[m];
-          sm = fmaf(x0.x, a0.x, sm);
-          sm = fmaf(x0.y, a0.y, sm);
-          sm = fmaf(x1.x, a1.x, sm);
-          sm = fmaf(x1.y, a1.y, sm);
-          sm = fmaf(x2.x, a2.x, sm);
-          sm = fmaf(x2.y, a2.y, sm);
-          sm = fmaf(x3.x, a3.x, sm);
-          sm = fmaf(x3.y, a3.y, sm);
-          acc[m] = sm;
-        }
-      }
+      for (int m = 0; m < MB; ++m)
+        if (m < M) fma8(acc[m], *reinterpret_cast<const uint4*>(&xs[m][8 * lane]), a0, a1, a2, a3);
     }
     __syncthreads();  // the piece is used before the next one is staged
   }
-  // sums over the warp's lanes (fixed shuffle order), lane 0 keeps them
-#pragma unroll
-  for (int m = 0; m < MB; ++m) {
-    float v = acc[m];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
-    if (lane == 0) part[warp][m] = v;
-  }
-  __syncthreads();
-  // then over the cluster's CTAs in rank order, in rank 0; thread (w, m)
-  const int w = threadIdx.x / MB, m = threadIdx.x % MB;
-  const bool mine = threadIdx.x < SMALL_WARPS * MB;
-  float sum = 0.0f;
-  if (splits > 1) {
-    cluster_sync_all();
-    if (split == 0 && mine) {
-      const uint32_t addr = smem_u32(&part[w][m]);
-      for (int sp = 0; sp < splits; ++sp) sum += ld_dsmem_f32(map_to_rank(addr, (uint32_t)sp));
-    }
-    cluster_sync_all();  // no CTA leaves while rank 0 reads its shared memory
-  } else if (mine) {
-    sum = part[w][m];
-  }
-  const int jj = blockIdx.x * SMALL_WARPS + w;
-  if (split == 0 && mine && m < M && jj < r)
-    t[(int64_t)m * r + jj] = __half_as_ushort(__float2half_rn(sum));
+  small_finish<MB>(acc, part, t, M, r, split, splits);
 }
 
-template <int MB>
-cudaError_t launch_small(const uint16_t* x, const uint16_t* lora_a, uint16_t* t, int64_t M,
-                         int64_t K, int64_t r, cudaStream_t stream, const DeviceInfo& dev) {
+// lanes: the lanes form (up to 8 tokens) on the free SMs when there are
+// enough (the layer's launch after it then starts everywhere at once and its
+// K stages overlap this one), else, like the staged form, split K over a
+// cluster (at most 16) until the CTAs cover the SMs.
+cudaError_t launch_small(bool lanes, const uint16_t* x, const uint16_t* lora_a, uint16_t* t,
+                         int64_t M, int64_t K, int64_t r, int free_sms, cudaStream_t stream,
+                         const DeviceInfo& dev) {
   const unsigned gr = (unsigned)((r + SMALL_WARPS - 1) / SMALL_WARPS);
-  // split K over a cluster until the CTAs cover the SMs (at most 16)
-  int splits = (int)std::min<int64_t>(kMaxSplits, std::max<int64_t>(1, dev.num_sms / gr));
+  int splits = lanes && free_sms >= (int)gr ? free_sms / (int)gr : dev.num_sms / (int)gr;
+  splits = std::max(1, std::min(kMaxSplits, splits));
   splits = std::min<int>(splits, (int)std::max<int64_t>(1, (K + PIECE - 1) / PIECE));
+  const void* fn = lanes ? (const void*)lora_down_lanes_kernel : (const void*)lora_down_staged_kernel;
   if (splits > 8) {
-    static std::once_flag once[64];
-    static cudaError_t attr_err[64];
+    static std::once_flag once[2][64];
+    static cudaError_t attr_err[2][64];
     const int d = dev.device & 63;
-    std::call_once(once[d], [&] {
-      attr_err[d] = cudaFuncSetAttribute(lora_down_small_kernel<MB>,
-                                         cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    std::call_once(once[lanes][d], [&] {
+      attr_err[lanes][d] =
+          cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     });
-    if (attr_err[d] != cudaSuccess) splits = 8;
+    if (attr_err[lanes][d] != cudaSuccess) splits = 8;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(gr, 1, (unsigned)splits);
@@ -154,8 +216,10 @@ cudaError_t launch_small(const uint16_t* x, const uint16_t* lora_a, uint16_t* t,
   attr[0].val.clusterDim.z = (unsigned)splits;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, lora_down_small_kernel<MB>, x, lora_a, t, (int)M, (int)K,
-                            (int)r, splits);
+  return lanes ? cudaLaunchKernelEx(&cfg, lora_down_lanes_kernel, x, lora_a, t, (int)M, (int)K,
+                                    (int)r, splits)
+               : cudaLaunchKernelEx(&cfg, lora_down_staged_kernel, x, lora_a, t, (int)M, (int)K,
+                                    (int)r, splits);
 }
 
 // Above 32 tokens: the tensor cores.  T^T [r, M] = lora_a . X^T with both
@@ -414,12 +478,13 @@ cudaError_t launch_tc(const uint16_t* x, const uint16_t* lora_a, uint16_t* t, in
 }  // namespace
 
 cudaError_t launch_lora_down(const uint16_t* x, const uint16_t* lora_a, uint16_t* t, int64_t M,
-                             int64_t K, int64_t r, cudaStream_t stream, const DeviceInfo& dev) {
+                             int64_t K, int64_t r, int free_sms, cudaStream_t stream,
+                             const DeviceInfo& dev) {
   // up to 32 tokens the per-lane form on the FP32 cores (at M = 1, rank 32:
   // 5.5 us, against 14 us for an FP32 form with shared-memory tiles, which
   // stalled on barriers there); above, the tensor cores
-  if (M <= 8) return launch_small<8>(x, lora_a, t, M, K, r, stream, dev);
-  if (M <= SMALL_M) return launch_small<SMALL_M>(x, lora_a, t, M, K, r, stream, dev);
+  if (M <= LANES_M) return launch_small(true, x, lora_a, t, M, K, r, free_sms, stream, dev);
+  if (M <= SMALL_M) return launch_small(false, x, lora_a, t, M, K, r, free_sms, stream, dev);
   return launch_tc(x, lora_a, t, M, K, r, stream, dev);
 }
 
