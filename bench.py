@@ -115,18 +115,49 @@ def tensor_peak(burst, sustained, src, elapsed_ms, reasons):
     return burst, f"{src} burst bf16 figure (timed region {elapsed_ms:.0f} ms); FP16 dense has the same nominal rate"
 
 
-def traffic_record(kernel_file: str, key: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (matching hash); else None."""
+def _code_only(text: str) -> str:
+    """C/C++ source without its comments, blank space collapsed (string and
+    character literals kept whole)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
+def kernel_source_digest() -> str:
+    """Hash of the code of the CUDA sources (comments and blank space do not
+    count): ncu counters stay attached to the kernels across edits of their
+    comments and are dropped by any change of code."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "traffic.txt")
     src = os.path.join(ROOT, "int4_weight_only_gptq_b200", "csrc")
     h = hashlib.sha256()
     for name in sorted(os.listdir(src)):
         if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(src, name), "rb") as f:
-                h.update(f.read())
-    digest = h.hexdigest()[:16]
+            with open(os.path.join(src, name), encoding="utf-8") as f:
+                h.update(name.encode() + b"\0" + _code_only(f.read()).encode())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel_file: str, key: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel code (matching digest); else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    digest = kernel_source_digest()
     try:
         with open(path) as f:
             for line in f:

@@ -6,14 +6,14 @@
 // extra K of the layer's product, where T . lora_b^T is added to the FP32
 // accumulator.
 //
-// Two forms, both deterministic (fixed summation orders, no global scratch):
-// up to 32 tokens a per-lane form on the FP32 cores (one warp per rank; the
-// product is a few loads per lane there), above that the tensor cores
-// (tcgen05.mma with both operands from shared memory).  Either splits K over
-// a thread-block cluster when its tiles cannot fill the SMs and adds the
-// partial sums in rank order through distributed shared memory.
+// Deterministic forms (fixed summation orders, no global scratch): up to 32
+// tokens per-lane forms on the FP32 cores (one warp per rank; the product is
+// a few loads per lane there), above that the tensor cores (tcgen05.mma with
+// both operands from shared memory).  Each splits K over a thread-block
+// cluster and adds the partial sums in rank order through distributed shared
+// memory.
 //
-// Stream order: both forms are launched WITHOUT programmatic stream
+// Stream order: every form is launched WITHOUT programmatic stream
 // serialisation, so they start only after every earlier kernel in the stream
 // has completed, and each lets its dependent start at once.  The layer's
 // launch that follows relies on this: it reads X and the weights without
@@ -480,9 +480,9 @@ cudaError_t launch_tc(const uint16_t* x, const uint16_t* lora_a, uint16_t* t, in
 cudaError_t launch_lora_down(const uint16_t* x, const uint16_t* lora_a, uint16_t* t, int64_t M,
                              int64_t K, int64_t r, int free_sms, cudaStream_t stream,
                              const DeviceInfo& dev) {
-  // up to 32 tokens the per-lane form on the FP32 cores (at M = 1, rank 32:
-  // 5.5 us, against 14 us for an FP32 form with shared-memory tiles, which
-  // stalled on barriers there); above, the tensor cores
+  // up to 32 tokens the per-lane forms on the FP32 cores (an FP32 form with
+  // shared-memory tiles took 14 us at M = 1, rank 32, stalled on barriers);
+  // above, the tensor cores
   if (M <= LANES_M) return launch_small(true, x, lora_a, t, M, K, r, free_sms, stream, dev);
   if (M <= SMALL_M) return launch_small(false, x, lora_a, t, M, K, r, free_sms, stream, dev);
   return launch_tc(x, lora_a, t, M, K, r, stream, dev);
