@@ -177,7 +177,9 @@ GPTQ_API int gptq_w4a16_gemm_asym(const uint16_t* x, const int32_t* qweight,
  * T is summed in FP32 and rounded to FP16; T . lora_b^T is added to the
  * layer's FP32 accumulator (the adapter's rank is extra K of the same
  * tensor-core product) and Y is rounded once.  Two launches on `stream`: T,
- * then the layer; every M runs on the prefill path.  Other arguments, checks
+ * then the layer, which follows M as in gptq_w4a16_gemm (decode up to
+ * GPTQ_DECODE_MAX_M, prefill above) and may start while T is computed (it
+ * waits for T only before reading it).  Other arguments, checks
  * and errors as gptq_w4a16_gemm, plus GPTQ_ERR_NULL for a NULL lora_a, lora_b
  * or t_work (when M > 0), GPTQ_ERR_SHAPE for a rank out of range, and
  * GPTQ_ERR_ALIAS when t_work or y overlaps any other buffer.
