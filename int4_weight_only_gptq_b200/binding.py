@@ -154,12 +154,13 @@ def gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, group: in
             raise ValueError(f"out has shape {tuple(out.shape)}, expected {(M, N)}")
     s = _stream_handle(stream, dev)
     args = (_ptr(x), _ptr(qweight), _ptr(scales), M, K, N, group, _ptr(out), s)
-    if decode_splits:
-        _check(lib.gptq_w4a16_gemm_decode_splits(*args, decode_splits))
-    elif kernel == KERNEL_AUTO:
-        _check(lib.gptq_w4a16_gemm(*args))
-    else:
-        _check(lib.gptq_w4a16_gemm_kernel(*args, kernel))
+    with torch.cuda.device(dev):  # the library works on the current device
+        if decode_splits:
+            _check(lib.gptq_w4a16_gemm_decode_splits(*args, decode_splits))
+        elif kernel == KERNEL_AUTO:
+            _check(lib.gptq_w4a16_gemm(*args))
+        else:
+            _check(lib.gptq_w4a16_gemm_kernel(*args, kernel))
     return out
 
 
@@ -196,8 +197,9 @@ def gemm_grouped(x: torch.Tensor, qweights, scales, group: int, outs=None,
     sa = (ctypes.c_void_p * count)(*[_ptr(t) for t in scales])
     na = (ctypes.c_int64 * count)(*Ns)
     ya = (ctypes.c_void_p * count)(*[_ptr(o) for o in outs])
-    _check(lib.gptq_w4a16_gemm_grouped(_ptr(x), qa, sa, na, count, M, K, group, ya,
-                                       _stream_handle(stream, dev)))
+    with torch.cuda.device(dev):
+        _check(lib.gptq_w4a16_gemm_grouped(_ptr(x), qa, sa, na, count, M, K, group, ya,
+                                           _stream_handle(stream, dev)))
     return outs
 
 
@@ -221,8 +223,9 @@ def gemm_asym(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
         out = torch.empty((M, N), dtype=torch.float16, device=dev)
     else:
         _require(out, "out", lambda d: d == torch.float16, dev)
-    _check(lib.gptq_w4a16_gemm_asym(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(qzeros), M, K,
-                                    N, group, _ptr(out), _stream_handle(stream, dev)))
+    with torch.cuda.device(dev):
+        _check(lib.gptq_w4a16_gemm_asym(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(qzeros), M,
+                                        K, N, group, _ptr(out), _stream_handle(stream, dev)))
     return out
 
 
@@ -260,9 +263,10 @@ def gemm_lora(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, grou
         _require(out, "out", lambda d: d == torch.float16, dev)
         if tuple(out.shape) != (M, N):
             raise ValueError(f"out has shape {tuple(out.shape)}, expected {(M, N)}")
-    _check(lib.gptq_w4a16_gemm_lora(_ptr(x), _ptr(qweight), _ptr(scales), M, K, N, group,
-                                    _ptr(lora_a), _ptr(lora_b), rank, _ptr(t_work), _ptr(out),
-                                    _stream_handle(stream, dev)))
+    with torch.cuda.device(dev):
+        _check(lib.gptq_w4a16_gemm_lora(_ptr(x), _ptr(qweight), _ptr(scales), M, K, N, group,
+                                        _ptr(lora_a), _ptr(lora_b), rank, _ptr(t_work),
+                                        _ptr(out), _stream_handle(stream, dev)))
     return out
 
 
@@ -286,9 +290,10 @@ def gemm_lora_noalloc(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tens
         out = torch.empty((M, N), dtype=torch.float16, device=dev)
     else:
         _require(out, "out", lambda d: d == torch.float16, dev)
-    _check(lib.gptq_w4a16_gemm_lora_noalloc(_ptr(x), _ptr(qweight), _ptr(scales), M, K, N,
-                                            group, _ptr(lora_a), _ptr(lora_b), rank, _ptr(out),
-                                            _stream_handle(stream, dev)))
+    with torch.cuda.device(dev):
+        _check(lib.gptq_w4a16_gemm_lora_noalloc(_ptr(x), _ptr(qweight), _ptr(scales), M, K, N,
+                                                group, _ptr(lora_a), _ptr(lora_b), rank,
+                                                _ptr(out), _stream_handle(stream, dev)))
     return out
 
 
@@ -304,8 +309,9 @@ def dequant(qweight: torch.Tensor, scales: torch.Tensor, group: int,
         out = torch.empty((K, N), dtype=torch.float16, device=dev)
     else:
         _require(out, "out", lambda d: d == torch.float16, dev)
-    _check(lib.gptq_dequant(_ptr(qweight), _ptr(scales), K, N, group, _ptr(out),
-                            _stream_handle(stream, dev)))
+    with torch.cuda.device(dev):
+        _check(lib.gptq_dequant(_ptr(qweight), _ptr(scales), K, N, group, _ptr(out),
+                                _stream_handle(stream, dev)))
     return out
 
 
