@@ -24,3 +24,23 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+# The parity tests print one "[parity] ..." line per compared case (the measured
+# max |y - y_ref| / (1 + |y_ref|)); pytest captures the output of passing tests,
+# so the lines are collected here and repeated in the session summary.
+_PARITY_LINES = []
+
+
+def pytest_runtest_logreport(report):
+    if report.when == "call" and report.passed:
+        for line in report.capstdout.splitlines():
+            if line.startswith("[parity]"):
+                _PARITY_LINES.append(line)
+
+
+def pytest_terminal_summary(terminalreporter):
+    if _PARITY_LINES:
+        terminalreporter.write_sep("-", "measured parity errors, max |y - y_ref| / (1 + |y_ref|)")
+        for line in _PARITY_LINES:
+            terminalreporter.write_line(line)
