@@ -483,7 +483,12 @@ def run_ours(args):
         if rank == 0:
             out["sweep"] = sweep
     if rank == 0:
-        out["cpu_baseline"] = cpu_baseline(p, bytes_per_step, bound)
+        cb = cpu_baseline(p, bytes_per_step, bound,
+                          y_gpu=yh.view(torch.int16).numpy().view(np.float16))
+        parity = cb.pop("parity", None)
+        out["cpu_baseline"] = cb
+        if parity is not None:
+            out["parity"] = parity
         print(json.dumps(out), flush=True)
     if world > 1:
         dist.barrier()
@@ -567,18 +572,32 @@ def run_sweep(lib, torch, l2, hbm, tf):
 
 # ---- CPU oracle ----------------------------------------------------------
 
-def cpu_baseline(p, bytes_per_step, bound="hbm", budget_s: float = 10.0):
+def parity_on_rows(y_gpu, ref, rows):
+    """The required error measure on the sampled rows (every column):
+    max |y - y_ref| / (1 + |y_ref|), y the layer's FP16 output, y_ref the
+    binary64 oracle."""
+    y = np.asarray(y_gpu, dtype=np.float64)[rows]
+    ref = np.asarray(ref, dtype=np.float64)
+    if y.shape != ref.shape:
+        raise ValueError(f"shapes {y.shape} and {ref.shape}")
+    err = float(np.max(np.abs(y - ref) / (1.0 + np.abs(ref)))) if y.size else 0.0
+    return {"max_rel_err": err, "bound": 1e-2, "within": bool(err <= 1e-2 and np.all(np.isfinite(y))),
+            "rows": [int(r) for r in rows], "cols": "all", "against": "binary64 oracle"}
+
+
+def cpu_baseline(p, bytes_per_step, bound="hbm", budget_s: float = 10.0, y_gpu=None):
     """The oracle as it stands (OpenMP over output columns) on a bounded
     sample of the same workload, repeated for about budget_s: every row when
     M <= 16, else four rows (first, last, two inside), scaled to the metric's
-    unit by the share of the work they are."""
+    unit by the share of the work they are.  With y_gpu (the layer's output
+    for the same inputs) the oracle's rows also give the parity error."""
     import oracle
     oracle.build()
     threads = oracle.get_threads()
     rows = list(range(p.M)) if p.M <= 16 else sorted({0, p.M // 3, 2 * p.M // 3, p.M - 1})
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle.gemm_rows(p.x, p.qweight, p.scales, p.group, rows)
+        ref = oracle.gemm_rows(p.x, p.qweight, p.scales, p.group, rows)
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s or n >= 1000:
@@ -590,9 +609,15 @@ def cpu_baseline(p, bytes_per_step, bound="hbm", budget_s: float = 10.0):
     else:
         value, unit = p.flops * share / per / 1e12, "TFLOP/s"
     what = "whole call(s) of the workload" if share == 1 else f"calls on {len(rows)} of {p.M} rows"
-    return {"value": round(value, 6), "unit": unit, "cores": threads, "kind": "oracle",
-            "sample": f"{n} {what} ({el:.1f} s, {threads} OpenMP threads over output columns)",
-            "s_per_call": round(per, 4)}
+    out = {"value": round(value, 6), "unit": unit, "cores": threads, "kind": "oracle",
+           "sample": f"{n} {what} ({el:.1f} s, {threads} OpenMP threads over output columns)",
+           "s_per_call": round(per, 4)}
+    if y_gpu is not None:
+        try:
+            out["parity"] = parity_on_rows(y_gpu, ref, rows)
+        except Exception as e:  # the timing stands; the comparison reports why it failed
+            out["parity"] = {"error": f"{type(e).__name__}: {e}"}
+    return out
 
 
 def run_reference(args):

@@ -68,3 +68,46 @@ def test_reference_arm_prints_the_contract_line():
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
     assert "workload" in d["config"]
+
+
+def test_parity_on_rows_measures_the_required_error():
+    import numpy as np
+    ref = np.array([[1.0, -3.0, 0.0], [10.0, 0.5, -0.25]])
+    y = np.zeros((4, 3), dtype=np.float16)
+    y[1] = ref[0]
+    y[3] = ref[1]
+    y[3, 0] = 10.5  # off by 0.5 where |y_ref| = 10: 0.5 / 11
+    out = bench.parity_on_rows(y, ref, [1, 3])
+    assert abs(out["max_rel_err"] - 0.5 / 11) < 1e-12
+    assert out["within"] is False and out["rows"] == [1, 3] and out["bound"] == 1e-2
+    y[3, 0] = 10.0
+    out = bench.parity_on_rows(y, ref, [1, 3])
+    assert out["max_rel_err"] == 0.0 and out["within"] is True
+
+
+def test_parity_on_rows_flags_non_finite_and_shape_errors():
+    import numpy as np
+    import pytest
+    ref = np.zeros((1, 2))
+    y = np.array([[np.inf, 0.0]], dtype=np.float16)
+    assert bench.parity_on_rows(y, ref, [0])["within"] is False
+    with pytest.raises(ValueError):
+        bench.parity_on_rows(np.zeros((2, 3)), ref, [0])
+
+
+def test_cpu_baseline_reports_parity_of_a_given_output():
+    """The CPU leg compares the output it is handed with its own oracle rows:
+    the oracle's FP16-rounded result is within the bound, a perturbed one is
+    caught."""
+    import numpy as np
+    import oracle
+    from int4_weight_only_gptq_b200 import workloads as W
+    p = W.tiny(4)
+    y = oracle.gemm(p.x, p.qweight, p.scales, p.group).astype(np.float16)
+    cb = bench.cpu_baseline(p, p.algorithmic_bytes, "hbm", budget_s=0.01, y_gpu=y)
+    assert cb["parity"]["within"] and cb["parity"]["max_rel_err"] < 1e-3
+    assert cb["parity"]["rows"] == [0, 1, 2, 3]
+    y[2, 5] = np.float16(float(y[2, 5]) + 1.0)
+    cb = bench.cpu_baseline(p, p.algorithmic_bytes, "hbm", budget_s=0.01, y_gpu=y)
+    assert cb["parity"]["max_rel_err"] > 0.1 and not cb["parity"]["within"]
+    assert "parity" not in bench.cpu_baseline(p, p.algorithmic_bytes, "hbm", budget_s=0.01)
