@@ -11,24 +11,28 @@
 // * The product is computed transposed, Y^T = W^T . X^T: a CTA owns 128 weight
 //   columns (the MMA's M, one TMEM lane each) and a range of K; the tokens are
 //   the MMA's N = BT, 16 or 32 (rows at or beyond M read as zero).
-// * One TMA producer thread streams, per 256-k stage, the qweight tile [32
-//   packed rows x 128 columns], the scale rows of the stage and the X tile
-//   [16 tokens x 256 k] (FP16, 128-byte swizzle: the B operand) into a ring of
-//   up to eight stages in shared memory.
-// * Sixteen dequantisation warps (four k-slices x four TMEM lane quarters)
-//   each turn eight words of their column into 32 TMEM cells of an A slot.  A
-//   word's codes come out paired (k, k+4) from the magic-number unpack; rather
-//   than shuffling every weight back to natural order, the same warps permute
-//   the (few) X rows of the stage in place to the paired order, so A and B
-//   agree on the order of k inside every 8-k block.
+// * One TMA producer thread streams, per 512-k stage, the qweight tile [64
+//   packed rows x 128 columns] (32 KB), the scale rows of the stage and the X
+//   tile [BT tokens x 512 k] (FP16, 128-byte swizzle: the B operand; one 3-D
+//   box when K is a multiple of 64) into a ring of stages in shared memory
+//   (three or four fit in the 224 KB budget).
+// * Sixteen dequantisation warps in two groups of eight take alternate stages
+//   (so one group's waits overlap the other's arithmetic); in a group, two
+//   k-slices x four TMEM lane quarters each turn eight words of their column
+//   at a time into 32 TMEM cells of an A slot (256 k per slot, three slots).
+//   A word's codes come out paired (k, k+4) from the magic-number unpack;
+//   rather than shuffling every weight back to natural order, the same warps
+//   permute the (few) X rows of the stage in place to the paired order, so A
+//   and B agree on the order of k inside every 8-k block.
 // * Each weight is dequantised exactly as defined, fp16((q - 8) * s): 1024 + q
 //   by a LOP3 into the FP16 mantissa of 1024, minus 1032 (exact), times the
 //   group scale (one rounding).  Keeping the definition's per-weight rounding
 //   matters: on inputs with large activation outliers, skipping it (scaling
 //   FP32 partial sums per group instead) moves Y by up to ~1e-2 relative.
-// * One thread issues tcgen05.mma (kind::f16, A from TMEM, B from shared
-//   memory, FP32 accumulate in TMEM); tcgen05.commit releases the ring slot and
-//   the A slot of each stage.  With only 16 tokens an MMA is short, and MMAs
+// * One elected lane of a converged MMA warp issues tcgen05.mma (kind::f16,
+//   A from TMEM, B from shared memory, FP32 accumulate in TMEM);
+//   tcgen05.commit releases the A slot of each fill and the ring slot of each
+//   stage.  With only 16 tokens an MMA is short, and MMAs
 //   into one accumulator run one after another, so the k16 steps go round-robin
 //   to NACC independent accumulators, summed in a fixed order at the end.
 // * Split-K: the `splits` CTAs of a thread-block cluster take consecutive K
