@@ -24,6 +24,12 @@ contract), read with GPTQ's packed qzeros [n_groups, N/8] (eight codes per
 int32 along N, lowest nibble = lowest n), each zero taken as stored:
     z[g,n] = (uint32(qzeros[g, n//8]) >> 4*(n%8)) & 0xF
     W[k,n] = fp16_RNE((q[k,n] - z[k//G, n]) * scales[k//G, n])
+
+With act order (GPTQ-Pro README, "Runtime contract": desc_act=False only there,
+act-order checkpoints outside that fork's contract; GPTQModel wiki, "Defaults
+and compatibility decisions": desc_act), read with GPTQ's group index per input
+channel g_idx [K] int32, qweight keeping the channels in their own order:
+    W[k,n] = fp16_RNE((q[k,n] - 8) * scales[g_idx[k], n])
 """
 from __future__ import annotations
 
@@ -86,6 +92,11 @@ def _load():
             lib.oracle_gemm_asym_rows.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32,
                                                   _i64, _p, _p]
             lib.oracle_lora_up_add.argtypes = [_p, _p, _i64, _i64, _i64, _p, _p]
+            lib.oracle_dequant_gidx.argtypes = [_p, _p, _p, _i64, _i64, _i64, _p]
+            lib.oracle_dequant_gidx.restype = ctypes.c_int
+            lib.oracle_gemm_gidx_rows.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i64,
+                                                  _i64, _p, _p]
+            lib.oracle_gemm_gidx_rows.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -311,3 +322,53 @@ def gemm_asym_rows(x, qweight, scales, qzeros, group, ms) -> np.ndarray:
 def gemm_asym(x, qweight, scales, qzeros, group) -> np.ndarray:
     """Y = x . W_asym in binary64, float64 [M, N]."""
     return gemm_asym_rows(x, qweight, scales, qzeros, group, np.arange(np.asarray(x).shape[0]))
+
+
+def _gidx(g_idx, K, n_groups):
+    g = np.asarray(g_idx)
+    if not np.issubdtype(g.dtype, np.integer):
+        raise TypeError(f"g_idx must be integer, got {g.dtype}")
+    if g.shape != (K,):
+        raise ValueError(f"g_idx must have shape ({K},)")
+    if g.size and (g.min() < 0 or g.max() >= n_groups):
+        raise ValueError("g_idx entry outside 0 .. n_groups - 1")
+    return np.ascontiguousarray(g, dtype=np.int32)
+
+
+def dequant_gidx(qweight, scales, g_idx) -> np.ndarray:
+    """W = fp16((q - 8) * scales[g_idx[k]]) as float16 [K, N] (act order)."""
+    qw = _c(qweight, np.int32)
+    s = _bits16(scales)
+    K, N = qw.shape[0] * 8, qw.shape[1]
+    if s.shape[1] != N:
+        raise ValueError("scales do not match N")
+    g = _gidx(g_idx, K, s.shape[0])
+    w = np.empty((K, N), dtype=np.uint16)
+    if _load().oracle_dequant_gidx(_ptr(qw), _ptr(s), _ptr(g), K, N, s.shape[0], _ptr(w)):
+        raise ValueError("g_idx entry out of range")
+    return w.view(np.float16)
+
+
+def gemm_gidx_rows(x, qweight, scales, g_idx, ms) -> np.ndarray:
+    """Rows ms of Y = x . W_act_order in binary64, float64 [len(ms), N]."""
+    xb = _bits16(x)
+    qw = _c(qweight, np.int32)
+    s = _bits16(scales)
+    M, K = xb.shape
+    N = qw.shape[1]
+    if qw.shape[0] * 8 != K or s.shape[1] != N:
+        raise ValueError("qweight or scales do not match x")
+    g = _gidx(g_idx, K, s.shape[0])
+    ms = _c(np.asarray(ms, dtype=np.int64), np.int64)
+    if ms.size and (ms.min() < 0 or ms.max() >= M):
+        raise IndexError("row index out of range")
+    out = np.empty((ms.size, N), dtype=np.float64)
+    if _load().oracle_gemm_gidx_rows(_ptr(xb), _ptr(qw), _ptr(s), _ptr(g), M, K, N,
+                                     s.shape[0], ms.size, _ptr(ms), _ptr(out)):
+        raise ValueError("g_idx entry out of range")
+    return out
+
+
+def gemm_gidx(x, qweight, scales, g_idx) -> np.ndarray:
+    """Y = x . W_act_order in binary64, float64 [M, N]."""
+    return gemm_gidx_rows(x, qweight, scales, g_idx, np.arange(np.asarray(x).shape[0]))

@@ -329,3 +329,64 @@ void oracle_gemm_asym_rows(const uint16_t* x, const int32_t* qweight, const uint
         }
     }
 }
+
+/* ---- act-order weights (per-channel group index) -------------------------
+ *
+ * GPTQ-Pro README, "Runtime contract" (desc_act=False only; act-order
+ * checkpoints lie outside that fork's contract) and GPTQModel wiki
+ * "Installation and Quickstart", "Defaults and compatibility decisions"
+ * (desc_act is activation ordering).  With act order the quantiser visits the
+ * input channels in a permuted order, so a group is no longer a run of
+ * consecutive k.  The pages give no storage for it; read with GPTQ's group
+ * index per input channel, qweight keeping the channels in their own order:
+ *     g_idx [K] int32,  0 <= g_idx[k] < n_groups
+ *     W[k,n] = fp16_RNE((q[k,n] - 8) * scales[g_idx[k], n])
+ * With g_idx[k] = floor(k / G) this is the layer above.
+ */
+
+static int gidx_valid(const int32_t* g_idx, int64_t K, int64_t n_groups)
+{
+    for (int64_t k = 0; k < K; ++k)
+        if (g_idx[k] < 0 || g_idx[k] >= n_groups) return 0;
+    return 1;
+}
+
+static uint16_t dequant_gidx_at(const int32_t* qweight, const uint16_t* scales,
+                                const int32_t* g_idx, int64_t N, int64_t k, int64_t n)
+{
+    double q = (double)code_at(qweight, N, k, n);
+    double s = oracle_half_to_double(scales[(int64_t)g_idx[k] * N + n]);
+    return oracle_double_to_half((q - 8.0) * s);   /* exact product, one rounding */
+}
+
+/* W (FP16 bits) [K, N]; returns 1, writing nothing, if an index is out of range. */
+int oracle_dequant_gidx(const int32_t* qweight, const uint16_t* scales, const int32_t* g_idx,
+                        int64_t K, int64_t N, int64_t n_groups, uint16_t* w)
+{
+    if (!gidx_valid(g_idx, K, n_groups)) return 1;
+    #pragma omp parallel for schedule(static)
+    for (int64_t k = 0; k < K; ++k)
+        for (int64_t n = 0; n < N; ++n)
+            w[k * N + n] = dequant_gidx_at(qweight, scales, g_idx, N, k, n);
+    return 0;
+}
+
+/* Y rows ms[0..count) of the act-order layer, binary64 [count, N], k
+ * ascending; returns 1, writing nothing, if an index is out of range. */
+int oracle_gemm_gidx_rows(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                          const int32_t* g_idx, int64_t M, int64_t K, int64_t N,
+                          int64_t n_groups, int64_t count, const int64_t* ms, double* out)
+{
+    (void)M;
+    if (!gidx_valid(g_idx, K, n_groups)) return 1;
+    #pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t i = 0; i < count; ++i) out[i * N + n] = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double w = oracle_half_to_double(dequant_gidx_at(qweight, scales, g_idx, N, k, n));
+            for (int64_t i = 0; i < count; ++i)
+                out[i * N + n] += oracle_half_to_double(x[ms[i] * K + k]) * w;
+        }
+    }
+    return 0;
+}

@@ -396,3 +396,110 @@ def test_gemm_asym_against_numpy_einsum(M, K, N, G):
     w = ((codes - z[g]) * s[g].astype(np.float64)).astype(np.float16).astype(np.float64)
     ref = np.einsum("mk,kn->mn", x.astype(np.float64), w)
     assert np.allclose(oracle.gemm_asym(x, qw, s, qz, G), ref, rtol=1e-12, atol=1e-12)
+
+
+# ---- act order (per-channel group index) --------------------------------------
+
+def _np_codes(qw):
+    """Codes [K, N] from qweight by numpy shifts (independent of the oracle)."""
+    u = np.asarray(qw).view(np.uint32)
+    K = u.shape[0] * 8
+    k = np.arange(K)
+    return ((u[k // 8] >> (4 * (k % 8))[:, None].astype(np.uint32)) & 0xF).astype(np.int64)
+
+
+def _np_pack(codes):
+    """Codes [K, N] -> qweight [K/8, N] by numpy (independent of the oracle)."""
+    c = np.asarray(codes, dtype=np.uint32)
+    words = np.zeros((c.shape[0] // 8, c.shape[1]), dtype=np.uint32)
+    for j in range(8):
+        words |= (c[j::8] & 0xF) << (4 * j)
+    return words.view(np.int32)
+
+
+def _np_dequant_gidx(qw, s, g_idx):
+    """(q - 8) * s[g_idx[k]] is exact in float32; numpy rounds it to float16."""
+    q = _np_codes(qw).astype(np.float32)
+    return ((q - 8.0) * np.asarray(s)[np.asarray(g_idx)].astype(np.float32)).astype(np.float16)
+
+
+def _gidx_problem(M, K, N, ng, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    qw = _np_pack(rng.integers(0, 16, size=(K, N)))
+    s = rng.uniform(1e-3, 2e-2, size=(ng, N)).astype(np.float16)
+    g = rng.integers(0, ng, size=K).astype(np.int32)
+    return x, qw, s, g
+
+
+@pytest.mark.parametrize("K,G", [(128, 16), (512, 128), (528, 128), (96, -1)])
+def test_gidx_with_consecutive_groups_is_the_plain_layer(K, G):
+    rng = np.random.default_rng(K)
+    N = 24
+    qw = _np_pack(rng.integers(0, 16, size=(K, N)))
+    ng = oracle.num_groups(K, G)
+    s = rng.uniform(1e-3, 2e-2, size=(ng, N)).astype(np.float16)
+    x = rng.standard_normal((3, K)).astype(np.float16)
+    g = np.arange(K) // (K if G == -1 else G)
+    assert np.array_equal(oracle.dequant_gidx(qw, s, g).view(np.uint16),
+                          oracle.dequant(qw, s, G).view(np.uint16))
+    assert np.array_equal(oracle.gemm_gidx(x, qw, s, g), oracle.gemm(x, qw, s, G))
+
+
+def test_gidx_dequant_against_numpy_float16():
+    """Every code, scattered group indices, ordinary and extreme scales."""
+    rng = np.random.default_rng(5)
+    K, N, ng = 256, 64, 7
+    svals = np.concatenate([rng.uniform(1e-4, 8.0, (ng, N - 2)),
+                            np.full((ng, 1), 2.0 ** -14), np.full((ng, 1), 65504.0)], axis=1)
+    s = svals.astype(np.float16)
+    qw = _np_pack(np.tile((np.arange(K) % 16)[:, None], (1, N)))
+    g = rng.integers(0, ng, size=K)
+    assert np.array_equal(oracle.dequant_gidx(qw, s, g).view(np.uint16),
+                          _np_dequant_gidx(qw, s, g).view(np.uint16))
+
+
+def test_gemm_gidx_against_numpy_einsum():
+    for M, K, N, ng in ((1, 16, 8, 1), (3, 64, 24, 5), (2, 160, 40, 9)):
+        x, qw, s, g = _gidx_problem(M, K, N, ng, seed=M + K)
+        w = _np_dequant_gidx(qw, s, g).astype(np.float64)
+        ref = np.einsum("mk,kn->mn", x.astype(np.float64), w)
+        assert np.allclose(oracle.gemm_gidx(x, qw, s, g), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_gidx_channel_permutation_leaves_y_unchanged():
+    """Permuting the input channels of x, the qweight rows and g_idx together
+    is the same layer (only the order of the sum over k changes)."""
+    x, qw, s, g = _gidx_problem(4, 128, 32, 6, seed=9)
+    perm = np.random.default_rng(9).permutation(128)
+    qw_p = _np_pack(_np_codes(qw)[perm])
+    y = oracle.gemm_gidx(x, qw, s, g)
+    y_p = oracle.gemm_gidx(np.ascontiguousarray(x[:, perm]), qw_p, s, g[perm])
+    assert np.allclose(y_p, y, rtol=1e-12, atol=1e-12)
+    w_p = oracle.dequant_gidx(qw_p, s, g[perm])
+    assert np.array_equal(w_p.view(np.uint16), oracle.dequant_gidx(qw, s, g)[perm].view(np.uint16))
+
+
+def test_gidx_one_entry_moves_one_weight_row():
+    x, qw, s, g = _gidx_problem(2, 64, 16, 4, seed=11)
+    w0 = oracle.dequant_gidx(qw, s, g)
+    g1 = g.copy()
+    g1[37] = (g[37] + 1) % 4
+    w1 = oracle.dequant_gidx(qw, s, g1)
+    rows = set(np.argwhere(w0.view(np.uint16) != w1.view(np.uint16))[:, 0])
+    assert rows == {37}
+
+
+def test_gidx_rejects_bad_indices():
+    x, qw, s, g = _gidx_problem(1, 32, 8, 3, seed=12)
+    for bad in (-1, 3):
+        gb = g.copy()
+        gb[5] = bad
+        with pytest.raises(ValueError):
+            oracle.dequant_gidx(qw, s, gb)
+        with pytest.raises(ValueError):
+            oracle.gemm_gidx(x, qw, s, gb)
+    with pytest.raises(ValueError):
+        oracle.dequant_gidx(qw, s, g[:-1])
+    with pytest.raises(TypeError):
+        oracle.dequant_gidx(qw, s, g.astype(np.float64))
