@@ -252,30 +252,73 @@ def copies_for(p, l2_bytes: int) -> int:
     return max(1, math.ceil(2 * l2_bytes / per) + 1)
 
 
-def time_gemm(lib, torch, p, steps, warmup, kernel=0, stream=None, l2_bytes=0):
-    """Device time per call (ms) of back-to-back calls through the C ABI."""
-    copies = copies_for(p, l2_bytes) if l2_bytes else 1
-    sets = to_device(p, torch, copies)
-    stream = stream or torch.cuda.current_stream()
-    sh = ctypes.c_void_p(stream.cuda_stream)
-    fn = lib.gptq_w4a16_gemm if kernel == 0 else lib.gptq_w4a16_gemm_kernel
-    argv = []
-    for (x, qw, s, y) in sets:
-        a = (ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(qw.data_ptr()),
-             ctypes.c_void_p(s.data_ptr()), p.M, p.K, p.N, p.group, ctypes.c_void_p(y.data_ptr()), sh)
-        argv.append(a if kernel == 0 else a + (kernel,))
+def time_loop(torch, fn, make_argv, steps, warmup, graph=True):
+    """Device time per call (ms) of `steps` back-to-back calls fn(*argv[i % n]),
+    argv = make_argv(stream handle), after `warmup` untimed calls.
+
+    graph=True: the `steps` calls are captured once in a CUDA graph (each call
+    still validates, dispatches and launches through the C ABI while it is
+    captured) and the graph is replayed once untimed and once timed, so the
+    device runs the calls back to back without waiting for the host.  Else an
+    eager loop of calls.  Returns (ms per call, host us per call of the eager
+    enqueue loop or None)."""
+    stream = torch.cuda.current_stream()
+    argv = make_argv(ctypes.c_void_p(stream.cuda_stream))
+    n = len(argv)
     for i in range(warmup):
-        st = fn(*argv[i % copies])
+        st = fn(*argv[i % n])
         if st:
-            raise RuntimeError(f"gemm status {st}")
+            raise RuntimeError(f"status {st}")
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        with torch.cuda.graph(g, stream=cap):
+            av = make_argv(ctypes.c_void_p(cap.cuda_stream))
+            for i in range(steps):
+                st = fn(*av[i % n])
+                if st:
+                    raise RuntimeError(f"status {st} while capturing")
+        g.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        del g
+        return ms, None
     e0.record(stream)
+    t0 = time.perf_counter()
     for i in range(steps):
-        fn(*argv[i % copies])
+        fn(*argv[i % n])
+    host_us = (time.perf_counter() - t0) * 1e6 / steps
     e1.record(stream)
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / steps, copies
+    return e0.elapsed_time(e1) / steps, host_us
+
+
+def gemm_argv(p, sets, kernel=0):
+    def make(sh):
+        out = []
+        for (x, qw, s, y) in sets:
+            a = (ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(qw.data_ptr()),
+                 ctypes.c_void_p(s.data_ptr()), p.M, p.K, p.N, p.group,
+                 ctypes.c_void_p(y.data_ptr()), sh)
+            out.append(a if kernel == 0 else a + (kernel,))
+        return out
+    return make
+
+
+def time_gemm(lib, torch, p, steps, warmup, kernel=0, l2_bytes=0, graph=True):
+    """Device time per call (ms) of back-to-back calls through the C ABI,
+    rotating enough copies of the inputs that each call reads from HBM."""
+    copies = copies_for(p, l2_bytes) if l2_bytes else 1
+    sets = to_device(p, torch, copies)
+    fn = lib.gptq_w4a16_gemm if kernel == 0 else lib.gptq_w4a16_gemm_kernel
+    ms, _ = time_loop(torch, fn, gemm_argv(p, sets, kernel), steps, warmup, graph)
+    return ms, copies
 
 
 def time_grouped(lib, torch, ps, steps, warmup, l2_bytes):
@@ -283,8 +326,7 @@ def time_grouped(lib, torch, ps, steps, warmup, l2_bytes):
     X), rotating enough weight copies that they do not stay in L2."""
     total = sum(p.algorithmic_bytes for p in ps)
     copies = max(1, -(-2 * l2_bytes // total) + 1)
-    sh = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    keep, argv = [], []
+    keep, per_copy = [], []
     M, K, count = ps[0].M, ps[0].K, len(ps)
     x = torch.from_numpy(ps[0].x.view(np.int16)).view(torch.float16).cuda()
     for c in range(copies):
@@ -296,20 +338,13 @@ def time_grouped(lib, torch, ps, steps, warmup, l2_bytes):
         sa = (ctypes.c_void_p * count)(*[ctypes.c_void_p(t.data_ptr()) for t in ss])
         na = (ctypes.c_int64 * count)(*[p.N for p in ps])
         ya = (ctypes.c_void_p * count)(*[ctypes.c_void_p(t.data_ptr()) for t in ys])
-        argv.append((ctypes.c_void_p(x.data_ptr()), qa, sa, na, count, M, K, ps[0].group, ya, sh))
-    fn = lib.gptq_w4a16_gemm_grouped
-    for i in range(warmup):
-        st = fn(*argv[i % copies])
-        if st:
-            raise RuntimeError(f"grouped gemm status {st}")
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(steps):
-        fn(*argv[i % copies])
-    e1.record()
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / steps
+        per_copy.append((qa, sa, na, ya))
+
+    def make(sh):
+        return [(ctypes.c_void_p(x.data_ptr()), qa, sa, na, count, M, K, ps[0].group, ya, sh)
+                for (qa, sa, na, ya) in per_copy]
+    ms, _ = time_loop(torch, lib.gptq_w4a16_gemm_grouped, make, steps, warmup)
+    return ms
 
 
 def time_asym(lib, torch, p, qzeros, steps, warmup, l2_bytes):
@@ -318,23 +353,13 @@ def time_asym(lib, torch, p, qzeros, steps, warmup, l2_bytes):
     copies = copies_for(p, l2_bytes) if l2_bytes else 1
     sets = to_device(p, torch, copies)
     zs = [torch.from_numpy(qzeros).cuda() for _ in range(copies)]
-    sh = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     v = ctypes.c_void_p
-    argv = [(v(x.data_ptr()), v(qw.data_ptr()), v(s.data_ptr()), v(z.data_ptr()), p.M, p.K, p.N,
-             p.group, v(y.data_ptr()), sh) for (x, qw, s, y), z in zip(sets, zs)]
-    fn = lib.gptq_w4a16_gemm_asym
-    for i in range(warmup):
-        st = fn(*argv[i % copies])
-        if st:
-            raise RuntimeError(f"asym gemm status {st}")
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(steps):
-        fn(*argv[i % copies])
-    e1.record()
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / steps
+
+    def make(sh):
+        return [(v(x.data_ptr()), v(qw.data_ptr()), v(s.data_ptr()), v(z.data_ptr()), p.M, p.K,
+                 p.N, p.group, v(y.data_ptr()), sh) for (x, qw, s, y), z in zip(sets, zs)]
+    ms, _ = time_loop(torch, lib.gptq_w4a16_gemm_asym, make, steps, warmup)
+    return ms
 
 
 def time_lora(lib, torch, p, ad, steps, warmup, l2_bytes):
@@ -346,24 +371,28 @@ def time_lora(lib, torch, p, ad, steps, warmup, l2_bytes):
     a = torch.from_numpy(ad.lora_a.view(np.int16)).view(torch.float16).cuda()
     b = torch.from_numpy(ad.lora_b.view(np.int16)).view(torch.float16).cuda()
     t = torch.empty((p.M, ad.rank), dtype=torch.float16, device="cuda")
-    sh = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     v = ctypes.c_void_p
-    argv = [(v(x.data_ptr()), v(qw.data_ptr()), v(s.data_ptr()), p.M, p.K, p.N, p.group,
-             v(a.data_ptr()), v(b.data_ptr()), ad.rank, v(t.data_ptr()), v(y.data_ptr()), sh)
-            for (x, qw, s, y) in sets]
-    fn = lib.gptq_w4a16_gemm_lora
-    for i in range(warmup):
-        st = fn(*argv[i % copies])
-        if st:
-            raise RuntimeError(f"lora gemm status {st}")
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(steps):
-        fn(*argv[i % copies])
-    e1.record()
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / steps
+
+    def make(sh):
+        return [(v(x.data_ptr()), v(qw.data_ptr()), v(s.data_ptr()), p.M, p.K, p.N, p.group,
+                 v(a.data_ptr()), v(b.data_ptr()), ad.rank, v(t.data_ptr()), v(y.data_ptr()), sh)
+                for (x, qw, s, y) in sets]
+    ms, _ = time_loop(torch, lib.gptq_w4a16_gemm_lora, make, steps, warmup)
+    return ms
+
+
+def hbm_entry(p, ms, hbm, extra_bytes=0):
+    gbs = (p.algorithmic_bytes + extra_bytes) / (ms * 1e-3) / 1e9
+    return {"M": p.M, "K": p.K, "N": p.N, "group": p.group, "ms": round(ms, 5),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
+                         "unit": "GB/s", "frac": round(gbs / hbm, 3)}}
+
+
+def tensor_entry(p, ms, peak, extra_flops=0):
+    tfl = (p.flops + extra_flops) / (ms * 1e-3) / 1e12
+    return {"M": p.M, "K": p.K, "N": p.N, "group": p.group, "ms": round(ms, 4),
+            "roofline": {"bound": "tensor", "achieved": round(tfl, 1), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(tfl / peak, 3)}}
 
 
 def run_ours(args):
@@ -386,16 +415,27 @@ def run_ours(args):
     # the tensor-bound ones move more than the L2 per call anyway
     copies = copies_for(p, l2) if bound == "hbm" else 1
     sets = to_device(p, torch, copies)
-    stream = torch.cuda.current_stream()
-    sh = ctypes.c_void_p(stream.cuda_stream)
-    argv = [(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(qw.data_ptr()),
-             ctypes.c_void_p(s.data_ptr()), p.M, p.K, p.N, p.group,
-             ctypes.c_void_p(y.data_ptr()), sh) for (x, qw, s, y) in sets]
     fn = lib.gptq_w4a16_gemm
-    for i in range(max(3, args.warmup)):
+    make_argv = gemm_argv(p, sets)
+    stream = torch.cuda.current_stream()
+    argv = make_argv(ctypes.c_void_p(stream.cuda_stream))
+    warm = max(3, args.warmup)
+    for i in range(warm):
         st = fn(*argv[i % copies])
         if st:
             raise RuntimeError(f"gptq_w4a16_gemm returned {st}: {binding.status_string(st)}")
+    torch.cuda.synchronize()
+    # the timed steps, captured once as a CUDA graph of `steps` library calls
+    # (each call validates, dispatches and launches while it is captured)
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    with torch.cuda.graph(graph, stream=cap):
+        av = make_argv(ctypes.c_void_p(cap.cuda_stream))
+        for i in range(args.steps):
+            st = fn(*av[i % copies])
+            if st:
+                raise RuntimeError(f"gptq_w4a16_gemm returned {st} while captured")
+    graph.replay()  # untimed: the graph's first replay
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -403,13 +443,16 @@ def run_ours(args):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank, str(getattr(props, "uuid", "")) or None) as clk:
         e0.record(stream)
-        for i in range(args.steps):
-            fn(*argv[i % copies])
+        graph.replay()
         e1.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     elapsed_ms = max_over_ranks(e0.elapsed_time(e1), "cuda")
+    del graph
+    # the same steps as an eager loop of calls (host enqueue between calls)
+    eager_ms, host_us = time_loop(torch, fn, make_argv, args.steps, 0, graph=False)
+    eager_ms = max_over_ranks(eager_ms, "cuda")
     if binding.device_error() != 0:
         raise RuntimeError("a kernel reported a bounded-wait timeout")
     ms, value, per_gpu = aggregate(bytes_per_step, args.steps, elapsed_ms, world)
@@ -420,7 +463,6 @@ def run_ours(args):
     # end to end through the public API with host buffers: pinned X in, Y out
     xh = torch.from_numpy(p.x.view(np.int16)).view(torch.float16).pin_memory()
     yh = torch.empty((p.M, p.N), dtype=torch.float16).pin_memory()
-    xd, qw, s, yd = sets[0]
     e2 = []
     for rep in range(2):
         torch.cuda.synchronize()
@@ -449,39 +491,47 @@ def run_ours(args):
             peak_src = ("measured (MEASURED_PEAKS.json hbm_gbs)" if src == "measured"
                         else "fallback 6.65 TB/s")
             e2e_val = bytes_per_step * world / (e2e_ms * 1e-3) / 1e9
+            eager_val = bytes_per_step / (eager_ms * 1e-3) / 1e9
         else:
             metric = "W4A16 GEMM prefill TFLOP/s (2*M*K*N)"
             unit, punit = "TFLOP/s", "TFLOP/s"
             peak, peak_src = tensor_peak(tf_burst, tf_sust, src, elapsed_ms,
                                          clocks.get("reasons") if clocks else None)
             e2e_val = p.flops * world / (e2e_ms * 1e-3) / 1e12
+            eager_val = p.flops / (eager_ms * 1e-3) / 1e12
         out = {
             "metric": metric,
             "value": round(value, 1), "unit": unit, "n_gpus": world, "steps": args.steps,
-            "warmup": max(3, args.warmup), "ms_per_step": round(ms, 6),
+            "warmup": warm, "ms_per_step": round(ms, 6),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp16 x int4 -> fp32 acc -> fp16", "data": "synthetic (seeded, PCG64 seed 0)",
             "config": {"workload": desc, "M": p.M, "K": p.K, "N": p.N, "group": p.group,
                        "bytes_per_step": bytes_per_step,
                        "l2": f"rotating {copies} input copies ({copies * bytes_per_step / 1e6:.0f} MB > 2x L2 {l2 / 1e6:.0f} MB)",
+                       "timing": "the steps captured once as a CUDA graph of library calls, replayed once untimed and once timed (CUDA events on the replay stream)",
                        "parallelism": f"replicas x{world} (no exchange)",
                        "kernel": {1: "decode", 2: "prefill"}.get(kernel_id, kernel_id),
                        "split_k_ctas": split},
             "roofline": {"bound": bound, "achieved": round(per_gpu, 1), "peak": peak,
                          "unit": punit, "frac": round(per_gpu / peak, 4),
                          "peak_source": peak_src, "traffic": traffic},
+            "eager": {"value": round(eager_val, 1), "unit": unit, "ms_per_step": round(eager_ms, 6),
+                      "host_us_per_call": round(host_us, 2),
+                      "note": "the same steps as a Python loop of C-ABI calls (no graph)"},
             "e2e": {"value": round(e2e_val, 1),
                     "unit": unit, "ms_per_step": round(e2e_ms, 6),
                     "h2d_bytes_per_step": int(p.M * p.K * 2),
                     "d2h_bytes_per_step": int(p.M * p.N * 2),
-                    "note": "pinned host X -> device, gptq_w4a16_gemm, device Y -> pinned host; weights resident"},
+                    "note": "eager loop: pinned host X -> device, gptq_w4a16_gemm, device Y -> pinned host; weights resident"},
             "gpu_launches": args.steps,
             "clocks": clocks,
         }
     if not args.no_sweep and world == 1:
         sweep = run_sweep(lib, torch, l2, hbm, tf_burst)
         if rank == 0:
-            out["sweep"] = sweep
+            # the long sweep on its own line first; the contract line stays short
+            print(json.dumps({"sweep": sweep}), flush=True)
+            out.update(headline_keys(sweep))
     if rank == 0:
         cb = cpu_baseline(p, bytes_per_step, bound,
                           y_gpu=yh.view(torch.int16).numpy().view(np.float16))
@@ -495,24 +545,33 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def headline_keys(sweep):
+    """The other halves of the metric, compact, for the contract line: prefill
+    at M = 2048 and 8192 (tensor roofline), the down-projection decode at
+    M = 16 and the mid-M up-projection at M = 64 (HBM roofline)."""
+    pick = lambda names: {n.split("_")[-1]: sweep[n] for n in names if n in sweep}
+    return {"prefill": pick(["prefill_M2048", "prefill_M8192"]),
+            "decode_down": pick(["decode_down_M1", "decode_down_M16"]),
+            "midm": pick(["midm_up_M48", "midm_up_M64"])}
+
+
 def run_sweep(lib, torch, l2, hbm, tf):
-    """The other workloads, one line each: decode GB/s, prefill TFLOP/s."""
+    """The other workloads: decode GB/s, prefill TFLOP/s, each with its
+    roofline fraction (HBM: measured copy bandwidth; tensor: measured burst)."""
     res = {}
 
     def hbm_case(name, p, steps=300):
         ms, copies = time_gemm(lib, torch, p, steps, 20, l2_bytes=l2)
-        gbs = p.algorithmic_bytes / (ms * 1e-3) / 1e9
-        res[name] = {"ms": round(ms, 5), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
+        res[name] = hbm_entry(p, ms, hbm)
 
     def tc_case(name, p, steps=30):
         ms, _ = time_gemm(lib, torch, p, steps, 5)
-        tfl = p.flops / (ms * 1e-3) / 1e12
-        res[name] = {"ms": round(ms, 4), "TFLOP/s": round(tfl, 1), "frac_tensor": round(tfl / tf, 3)}
+        res[name] = tensor_entry(p, ms, tf)
 
     for M in (1, 2, 4, 8, 16, 32):
         hbm_case(f"decode_down_M{M}", W.decode_down(M))
-    # between the kernels: decode up to M = 32, prefill (64-token tile) above
-    for M in (24, 32, 48, 64):
+    # between the kernels: decode up to M = 32, pair prefill above
+    for M in (24, 32, 48, 64, 96, 128):
         hbm_case(f"midm_up_M{M}", W.make_problem(M, 5120, 17408, 128, seed=0), steps=100)
     for M in (512, 2048, 8192):
         tc_case(f"prefill_M{M}", W.prefill(M))
@@ -525,8 +584,7 @@ def run_sweep(lib, torch, l2, hbm, tf):
             hbm_case(f"layer_{name}_M{M}", W.layer_linear(name, M))
         tc_case(f"layer_{name}_M4096", W.layer_linear(name, 4096))
     for M in (1, 16, 4096):
-        key = "ms"
-        total = sum(res[f"layer_{n}_M{M}"][key] * c for n, _, _, c in W.LAYER_LINEARS)
+        total = sum(res[f"layer_{n}_M{M}"]["ms"] * c for n, _, _, c in W.LAYER_LINEARS)
         res[f"layer_total_M{M}_ms"] = round(total, 4)
     # shared-input linears in one call (q/k/v: 3 x 5120->5120; gate+up: 2 x 5120->17408)
     for name, count, N in (("qkv", 3, 5120), ("gate_up", 2, 17408)):
@@ -585,12 +643,27 @@ def parity_on_rows(y_gpu, ref, rows):
             "rows": [int(r) for r in rows], "cols": "all", "against": "binary64 oracle"}
 
 
-def cpu_baseline(p, bytes_per_step, bound="hbm", budget_s: float = 10.0, y_gpu=None):
-    """The oracle as it stands (OpenMP over output columns) on a bounded
-    sample of the same workload, repeated for about budget_s: every row when
-    M <= 16, else four rows (first, last, two inside), scaled to the metric's
-    unit by the share of the work they are.  With y_gpu (the layer's output
-    for the same inputs) the oracle's rows also give the parity error."""
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
+def cpu_baseline(p, bytes_per_step, bound="hbm", budget_s: float = 8.0, y_gpu=None):
+    """The oracle as it stands on a bounded sample of the same workload, in two
+    variants: OpenMP over output columns on every host thread (the line's
+    value), and one thread.  Every row when M <= 16, else four rows (first,
+    last, two inside); the single-thread variant takes a column slice of those
+    rows.  Each is repeated for about budget_s and scaled to the metric's unit
+    by the share of the work it did.  With y_gpu (the layer's output for the
+    same inputs) the oracle's rows also give the parity error."""
     import oracle
     oracle.build()
     threads = oracle.get_threads()
@@ -604,14 +677,39 @@ def cpu_baseline(p, bytes_per_step, bound="hbm", budget_s: float = 10.0, y_gpu=N
             break
     per = el / n
     share = len(rows) / p.M
-    if bound == "hbm":
-        value, unit = bytes_per_step * share / per / 1e9, "GB/s"
-    else:
-        value, unit = p.flops * share / per / 1e12, "TFLOP/s"
+
+    def rate(share_of_work, seconds):
+        if bound == "hbm":
+            return bytes_per_step * share_of_work / seconds / 1e9, "GB/s"
+        return p.flops * share_of_work / seconds / 1e12, "TFLOP/s"
+
+    value, unit = rate(share, per)
     what = "whole call(s) of the workload" if share == 1 else f"calls on {len(rows)} of {p.M} rows"
     out = {"value": round(value, 6), "unit": unit, "cores": threads, "kind": "oracle",
            "sample": f"{n} {what} ({el:.1f} s, {threads} OpenMP threads over output columns)",
-           "s_per_call": round(per, 4)}
+           "s_per_call": round(per, 4), "cpu_model": cpu_model(),
+           "host_threads": os.cpu_count()}
+    # one thread: a slice of the columns of the same rows
+    n_cols = min(p.N, 1088)
+    cols = np.arange(n_cols, dtype=np.int64)
+    ms_ = np.repeat(np.asarray(rows, dtype=np.int64), n_cols)
+    ns_ = np.tile(cols, len(rows))
+    try:
+        oracle.set_threads(1)
+        n1, t1 = 0, time.perf_counter()
+        while True:
+            oracle.gemm_entries(p.x, p.qweight, p.scales, p.group, ms_, ns_)
+            n1 += 1
+            el1 = time.perf_counter() - t1
+            if el1 >= budget_s or n1 >= 1000:
+                break
+    finally:
+        oracle.set_threads(threads)
+    share1 = len(rows) * n_cols / (p.M * p.N)
+    v1, _ = rate(share1, el1 / n1)
+    out["single_thread"] = {"value": round(v1, 6), "unit": unit, "cores": 1,
+                            "sample": f"{n1} calls on {len(rows)} row(s) x {n_cols} of {p.N} "
+                                      f"columns ({el1:.1f} s, one thread)"}
     if y_gpu is not None:
         try:
             out["parity"] = parity_on_rows(y_gpu, ref, rows)
@@ -658,7 +756,7 @@ def run_reference(args):
         "data": "synthetic (seeded, PCG64 seed 0)",
         "config": {"workload": desc, "M": p.M, "K": p.K, "N": p.N, "group": p.group},
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": threads,
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle", "sample": sample, "cpu_model": cpu_model()},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }), flush=True)

@@ -131,6 +131,50 @@ def _require(t: torch.Tensor, name: str, dtype_ok, device):
         raise TypeError(f"{name} has dtype {t.dtype}")
 
 
+def n_groups(K: int, group: int) -> int:
+    """Scale rows of a layer: one for group -1 or a group of K or more, else
+    ceil(K / group) (a ragged last group when group does not divide K)."""
+    return 1 if group == -1 or group >= K else -(-K // group)
+
+
+def layer_shapes(x, qweight, scales, group: int) -> tuple[int, int, int]:
+    """(M, K, N) of a layer call, after checking that x [M, K], qweight
+    [K/8, N] and scales [n_groups(K, group), N] agree.  The C ABI sees only
+    pointers and the sizes it is given, and builds its tensor maps from them,
+    so a tensor smaller than those sizes would be read past its end: the
+    shapes are checked here, before the library is called.  An unsupported
+    group is left to the library (GPTQ_ERR_GROUP)."""
+    if x.dim() != 2 or qweight.dim() != 2 or scales.dim() != 2:
+        raise ValueError("x, qweight and scales must be 2-D")
+    M, K = (int(v) for v in x.shape)
+    N = int(qweight.shape[1])
+    if int(qweight.shape[0]) * 8 != K:
+        raise ValueError(f"qweight rows {qweight.shape[0]} do not match K={K}")
+    if group in GROUP_SIZES and K > 0:
+        want = (n_groups(K, group), N)
+        if tuple(scales.shape) != want:
+            raise ValueError(f"scales has shape {tuple(scales.shape)}, expected {want} "
+                             f"for K={K}, group={group}")
+    return M, K, N
+
+
+def adapter_shapes(lora_a, lora_b, K: int, N: int) -> int:
+    """The adapter's rank, after checking lora_a [rank, K] and lora_b [N, rank]."""
+    if lora_a.dim() != 2 or lora_b.dim() != 2:
+        raise ValueError("lora_a and lora_b must be 2-D")
+    rank = int(lora_a.shape[0])
+    if int(lora_a.shape[1]) != K:
+        raise ValueError(f"lora_a has shape {tuple(lora_a.shape)}, expected ({rank}, {K})")
+    if tuple(lora_b.shape) != (N, rank):
+        raise ValueError(f"lora_b has shape {tuple(lora_b.shape)}, expected {(N, rank)}")
+    return rank
+
+
+def _check_shape(t, name: str, shape: tuple):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
 def gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, group: int,
          out: torch.Tensor | None = None, stream=None, kernel: int = KERNEL_AUTO,
          decode_splits: int = 0) -> torch.Tensor:
@@ -140,18 +184,12 @@ def gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, group: in
     _require(qweight, "qweight", lambda d: d == torch.int32, None)
     _require(scales, "scales", lambda d: d == torch.float16, dev)
     _require(x, "x", lambda d: d == torch.float16, dev)
-    if x.dim() != 2 or qweight.dim() != 2 or scales.dim() != 2:
-        raise ValueError("x, qweight and scales must be 2-D")
-    M, K = x.shape
-    N = qweight.shape[1]
-    if qweight.shape[0] * 8 != K:
-        raise ValueError(f"qweight rows {qweight.shape[0]} do not match K={K}")
+    M, K, N = layer_shapes(x, qweight, scales, group)
     if out is None:
         out = torch.empty((M, N), dtype=torch.float16, device=dev)
     else:
         _require(out, "out", lambda d: d == torch.float16, dev)
-        if tuple(out.shape) != (M, N):
-            raise ValueError(f"out has shape {tuple(out.shape)}, expected {(M, N)}")
+        _check_shape(out, "out", (M, N))
     s = _stream_handle(stream, dev)
     args = (_ptr(x), _ptr(qweight), _ptr(scales), M, K, N, group, _ptr(out), s)
     with torch.cuda.device(dev):  # the library works on the current device
@@ -182,7 +220,8 @@ def gemm_grouped(x: torch.Tensor, qweights, scales, group: int, outs=None,
         _require(sc, f"scales[{i}]", lambda d: d == torch.float16, dev)
         if qw.dim() != 2 or qw.shape[0] * 8 != K:
             raise ValueError(f"qweights[{i}] does not match K={K}")
-        Ns.append(qw.shape[1])
+        layer_shapes(x, qw, sc, group)
+        Ns.append(int(qw.shape[1]))
     if outs is None:
         outs = [torch.empty((M, n), dtype=torch.float16, device=dev) for n in Ns]
     else:
@@ -214,15 +253,15 @@ def gemm_asym(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
     _require(scales, "scales", lambda d: d == torch.float16, dev)
     _require(qzeros, "qzeros", lambda d: d == torch.int32, dev)
     _require(x, "x", lambda d: d == torch.float16, dev)
-    M, K = x.shape
-    N = qweight.shape[1]
-    if tuple(qzeros.shape) != (scales.shape[0], N // 8):
+    M, K, N = layer_shapes(x, qweight, scales, group)
+    if qzeros.dim() != 2 or tuple(qzeros.shape) != (scales.shape[0], N // 8):
         raise ValueError(f"qzeros has shape {tuple(qzeros.shape)}, expected "
                          f"{(scales.shape[0], N // 8)}")
     if out is None:
         out = torch.empty((M, N), dtype=torch.float16, device=dev)
     else:
         _require(out, "out", lambda d: d == torch.float16, dev)
+        _check_shape(out, "out", (M, N))
     with torch.cuda.device(dev):
         _check(lib.gptq_w4a16_gemm_asym(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(qzeros), M,
                                         K, N, group, _ptr(out), _stream_handle(stream, dev)))
@@ -242,27 +281,18 @@ def gemm_lora(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, grou
     _require(x, "x", lambda d: d == torch.float16, dev)
     _require(lora_a, "lora_a", lambda d: d == torch.float16, dev)
     _require(lora_b, "lora_b", lambda d: d == torch.float16, dev)
-    if x.dim() != 2 or lora_a.dim() != 2 or lora_b.dim() != 2:
-        raise ValueError("x, lora_a and lora_b must be 2-D")
-    M, K = x.shape
-    N = qweight.shape[1]
-    rank = lora_a.shape[0]
-    if qweight.shape[0] * 8 != K or lora_a.shape[1] != K:
-        raise ValueError(f"qweight or lora_a do not match K={K}")
-    if tuple(lora_b.shape) != (N, rank):
-        raise ValueError(f"lora_b has shape {tuple(lora_b.shape)}, expected {(N, rank)}")
+    M, K, N = layer_shapes(x, qweight, scales, group)
+    rank = adapter_shapes(lora_a, lora_b, K, N)
     if t_work is None:
         t_work = torch.empty((M, rank), dtype=torch.float16, device=dev)
     else:
         _require(t_work, "t_work", lambda d: d == torch.float16, dev)
-        if tuple(t_work.shape) != (M, rank):
-            raise ValueError(f"t_work has shape {tuple(t_work.shape)}, expected {(M, rank)}")
+        _check_shape(t_work, "t_work", (M, rank))
     if out is None:
         out = torch.empty((M, N), dtype=torch.float16, device=dev)
     else:
         _require(out, "out", lambda d: d == torch.float16, dev)
-        if tuple(out.shape) != (M, N):
-            raise ValueError(f"out has shape {tuple(out.shape)}, expected {(M, N)}")
+        _check_shape(out, "out", (M, N))
     with torch.cuda.device(dev):
         _check(lib.gptq_w4a16_gemm_lora(_ptr(x), _ptr(qweight), _ptr(scales), M, K, N, group,
                                         _ptr(lora_a), _ptr(lora_b), rank, _ptr(t_work),
@@ -283,13 +313,13 @@ def gemm_lora_noalloc(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tens
     _require(x, "x", lambda d: d == torch.float16, dev)
     _require(lora_a, "lora_a", lambda d: d == torch.float16, dev)
     _require(lora_b, "lora_b", lambda d: d == torch.float16, dev)
-    M, K = x.shape
-    N = qweight.shape[1]
-    rank = lora_a.shape[0]
+    M, K, N = layer_shapes(x, qweight, scales, group)
+    rank = adapter_shapes(lora_a, lora_b, K, N)
     if out is None:
         out = torch.empty((M, N), dtype=torch.float16, device=dev)
     else:
         _require(out, "out", lambda d: d == torch.float16, dev)
+        _check_shape(out, "out", (M, N))
     with torch.cuda.device(dev):
         _check(lib.gptq_w4a16_gemm_lora_noalloc(_ptr(x), _ptr(qweight), _ptr(scales), M, K, N,
                                                 group, _ptr(lora_a), _ptr(lora_b), rank,
@@ -304,11 +334,17 @@ def dequant(qweight: torch.Tensor, scales: torch.Tensor, group: int,
     dev = qweight.device
     _require(qweight, "qweight", lambda d: d == torch.int32, None)
     _require(scales, "scales", lambda d: d == torch.float16, dev)
-    K, N = qweight.shape[0] * 8, qweight.shape[1]
+    if qweight.dim() != 2 or scales.dim() != 2:
+        raise ValueError("qweight and scales must be 2-D")
+    K, N = int(qweight.shape[0]) * 8, int(qweight.shape[1])
+    if group in GROUP_SIZES and tuple(scales.shape) != (n_groups(K, group), N):
+        raise ValueError(f"scales has shape {tuple(scales.shape)}, expected "
+                         f"{(n_groups(K, group), N)} for K={K}, group={group}")
     if out is None:
         out = torch.empty((K, N), dtype=torch.float16, device=dev)
     else:
         _require(out, "out", lambda d: d == torch.float16, dev)
+        _check_shape(out, "out", (K, N))
     with torch.cuda.device(dev):
         _check(lib.gptq_dequant(_ptr(qweight), _ptr(scales), K, N, group, _ptr(out),
                                 _stream_handle(stream, dev)))

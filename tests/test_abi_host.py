@@ -227,3 +227,52 @@ def test_asym_empty_m_and_no_device(lib):
     assert call_asym(lib, M=0, x=0, y=0, qz=0) == 1
     if not torch.cuda.is_available():
         assert call_asym(lib) == 5
+
+
+# ---- binding: shape checks before the library is called ----------------------
+# The C ABI sees pointers and the sizes it is given; a tensor smaller than those
+# sizes would be read or written past its end, so the binding checks shapes.
+# The checks are pure shape logic and run here on CPU tensors.
+
+def _t(*shape, dtype=None):
+    import torch
+    return torch.zeros(shape, dtype=dtype or torch.float16)
+
+
+def test_n_groups():
+    assert binding.n_groups(512, 128) == 4
+    assert binding.n_groups(528, 128) == 5       # ragged last group
+    assert binding.n_groups(512, -1) == 1
+    assert binding.n_groups(512, 1024) == 1      # a group of K or more is one group
+    assert binding.n_groups(512, 512) == 1
+
+
+def test_layer_shapes_accept_and_reject():
+    import torch
+    i32 = torch.int32
+    assert binding.layer_shapes(_t(3, 512), _t(64, 256, dtype=i32), _t(4, 256), 128) == (3, 512, 256)
+    assert binding.layer_shapes(_t(3, 528), _t(66, 256, dtype=i32), _t(5, 256), 128) == (3, 528, 256)
+    assert binding.layer_shapes(_t(1, 512), _t(64, 256, dtype=i32), _t(1, 256), -1) == (1, 512, 256)
+    bad = [
+        (_t(3, 512), _t(63, 256, dtype=i32), _t(4, 256), 128),     # qweight rows != K/8
+        (_t(3, 512), _t(64, 256, dtype=i32), _t(2, 256), 128),     # scales for group 256
+        (_t(3, 512), _t(64, 256, dtype=i32), _t(4, 248), 128),     # scales narrower than N
+        (_t(3, 512), _t(64, 256, dtype=i32), _t(4, 256), -1),      # group -1 has one row
+        (_t(512), _t(64, 256, dtype=i32), _t(4, 256), 128),        # x not 2-D
+        (_t(3, 512), _t(64, 256, dtype=i32), _t(1024), 128),       # scales not 2-D
+    ]
+    for args in bad:
+        with pytest.raises(ValueError):
+            binding.layer_shapes(*args)
+    # an unsupported group is the library's to report (GPTQ_ERR_GROUP)
+    assert binding.layer_shapes(_t(3, 512), _t(64, 256, dtype=i32), _t(7, 256), 100) == (3, 512, 256)
+
+
+def test_adapter_shapes_accept_and_reject():
+    assert binding.adapter_shapes(_t(32, 512), _t(256, 32), 512, 256) == 32
+    for a, b in ((_t(32, 520), _t(256, 32)),     # lora_a does not match K
+                 (_t(32, 512), _t(248, 32)),     # lora_b rows != N
+                 (_t(32, 512), _t(256, 48)),     # lora_b rank != lora_a rank
+                 (_t(32 * 512), _t(256, 32))):   # lora_a not 2-D
+        with pytest.raises(ValueError):
+            binding.adapter_shapes(a, b, 512, 256)

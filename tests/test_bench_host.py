@@ -111,3 +111,28 @@ def test_cpu_baseline_reports_parity_of_a_given_output():
     cb = bench.cpu_baseline(p, p.algorithmic_bytes, "hbm", budget_s=0.01, y_gpu=y)
     assert cb["parity"]["max_rel_err"] > 0.1 and not cb["parity"]["within"]
     assert "parity" not in bench.cpu_baseline(p, p.algorithmic_bytes, "hbm", budget_s=0.01)
+
+
+def test_headline_keys_pick_the_metric_halves_from_the_sweep():
+    sweep = {"prefill_M2048": {"ms": 0.25}, "prefill_M8192": {"ms": 0.95},
+             "decode_down_M1": {"ms": 0.017}, "decode_down_M16": {"ms": 0.018},
+             "midm_up_M64": {"ms": 0.02}, "square_g128_M1": {"ms": 0.01}}
+    h = bench.headline_keys(sweep)
+    assert set(h) == {"prefill", "decode_down", "midm"}
+    assert h["prefill"] == {"M2048": {"ms": 0.25}, "M8192": {"ms": 0.95}}
+    assert h["decode_down"]["M16"] == {"ms": 0.018}
+    assert h["midm"] == {"M64": {"ms": 0.02}}
+
+
+def test_roofline_entries():
+    from int4_weight_only_gptq_b200 import workloads as W
+    p = W.decode_up()
+    e = bench.hbm_entry(p, p.algorithmic_bytes / 6523.3e9 * 1e3, 6523.3)
+    assert abs(e["roofline"]["frac"] - 1.0) < 1e-3 and e["roofline"]["unit"] == "GB/s"
+    q = W.make_problem(2048, 5120, 17408, 128, seed=0)
+    t = bench.tensor_entry(q, q.flops / 1637.3e12 * 1e3, 1637.3)
+    assert abs(t["roofline"]["frac"] - 1.0) < 1e-3 and t["roofline"]["unit"] == "TFLOP/s"
+
+
+def test_cpu_model_is_named():
+    assert isinstance(bench.cpu_model(), str) and bench.cpu_model()

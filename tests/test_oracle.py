@@ -505,3 +505,45 @@ def test_gidx_rejects_bad_indices():
         oracle.dequant_gidx(qw, s, g[:-1])
     with pytest.raises(TypeError):
         oracle.dequant_gidx(qw, s, g.astype(np.float64))
+
+
+# ---- thread-count independence ------------------------------------------------
+# OpenMP threads only split independent outputs; each output's sum runs
+# sequentially in k.  So the result must not depend on the thread count: one
+# thread and every core give bitwise-identical outputs.
+
+def test_results_do_not_depend_on_thread_count():
+    import os
+    rng = np.random.default_rng(7)
+    M, K, N, G, r = 5, 528, 264, 128, 48
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    qw = rng.integers(-2**31, 2**31, size=(K // 8, N), dtype=np.int64).astype(np.int32)
+    sc = rng.uniform(1e-3, 2e-2, size=(oracle.num_groups(K, G), N)).astype(np.float16)
+    la = (rng.standard_normal((r, K)) / np.sqrt(K)).astype(np.float16)
+    lb = (rng.standard_normal((N, r)) * 0.05).astype(np.float16)
+    zc = rng.integers(0, 16, size=(oracle.num_groups(K, G), N)).astype(np.uint8)
+    qz = oracle.pack_zeros(zc)
+    ms = np.array([0, 2, 4], dtype=np.int64)
+    ns = rng.integers(0, N, size=40).astype(np.int64)
+    mm = rng.integers(0, M, size=40).astype(np.int64)
+
+    def run_all():
+        return (oracle.gemm(x, qw, sc, G), oracle.gemm_rows(x, qw, sc, G, ms),
+                oracle.gemm_entries(x, qw, sc, G, mm, ns), oracle.lora_down(x, la),
+                oracle.gemm_lora(x, qw, sc, G, la, lb), oracle.gemm_asym(x, qw, sc, qz, G),
+                oracle.dequant(qw, sc, G))
+
+    saved = oracle.get_threads()
+    many = max(4, os.cpu_count() or 4)
+    try:
+        oracle.set_threads(1)
+        assert oracle.get_threads() == 1
+        one = run_all()
+        oracle.set_threads(many)
+        assert oracle.get_threads() == many
+        lots = run_all()
+    finally:
+        oracle.set_threads(saved)
+    for a, b in zip(one, lots):
+        assert a.dtype == b.dtype and a.shape == b.shape
+        assert a.tobytes() == b.tobytes()

@@ -415,6 +415,24 @@ def test_lora_parity(M, K, N, G, r):
     assert err <= TOL
 
 
+# K not a multiple of 256: the down-projection's last 256-k piece is short in
+# both small-M forms (per-lane up to 8 tokens, staged rows from 9 to 32), and
+# ranks 48 / 80 leave a ragged last 128-rank piece in the decode's adapter stage.
+@pytest.mark.parametrize("M", [1, 5, 8, 9, 16, 32])
+@pytest.mark.parametrize("K,r", [(528, 48), (1040, 80), (2064, 16)])
+def test_lora_small_m_ragged_k(M, K, r):
+    N, G = 264, 16 if K == 528 else 128
+    p = W.make_problem(M, K, N, G, seed=M * 3 + K + r)
+    ad = W.make_adapter(K, N, r, seed=M * 3 + K + r)
+    y, t = run_lora(p, ad, t_out=True)
+    check_t(t, p.x, ad.lora_a)
+    ref = oracle.gemm_lora(p.x, p.qweight, p.scales, G, ad.lora_a, ad.lora_b)
+    err = rel_err(y, ref)
+    print(f"[parity] lora small M={M} K={K} N={N} G={G} r={r}: {err:.3e}")
+    assert np.all(np.isfinite(y))
+    assert err <= TOL
+
+
 @pytest.mark.parametrize("M", [1, 40, 300])
 def test_lora_integer_exact_inputs_bitwise(M):
     """Integer x and codes, power-of-two scales, sparse +-1 lora_a and lora_b

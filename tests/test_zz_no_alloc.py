@@ -51,3 +51,21 @@ def test_static_buffer_matches_caller_buffer_on_two_calls():
         torch.cuda.synchronize()
         assert B.device_error() == 0
         assert torch.equal(y_static.view(torch.int16), y_work.view(torch.int16))
+
+
+@pytest.mark.gpu
+def test_mis_shaped_tensors_are_refused_before_the_library_is_called():
+    """The C ABI cannot see buffer sizes: the binding refuses tensors whose
+    shapes do not match the sizes it would pass (out, lora_b, qweight, scales)."""
+    x, qw, s, G, a, b = _inputs(4, 512, 256, 128, 32, 3)
+    cases = [
+        dict(out=torch.empty((4, 248), dtype=torch.float16, device="cuda")),
+        dict(lora_b=b[:248]),
+        dict(qweight=qw[:56]),
+        dict(scales=s[:2]),
+    ]
+    for kw in cases:
+        args = dict(x=x, qweight=qw, scales=s, group=G, lora_a=a, lora_b=b)
+        args.update(kw)
+        with pytest.raises(ValueError):
+            B.gemm_lora_noalloc(**args)
