@@ -67,6 +67,43 @@ __device__ __forceinline__ void dequant_word_paired(uint32_t w, uint32_t s2, uin
   for (int j = 0; j < 4; ++j) p[j] = hmul2_rn(p[j], s2);
 }
 
+// The same four half2 for a scale with |s| < 2^-4, with two FP16 operations
+// fewer.  Codes at bits 4..7 of each 16-bit half, masked out of the word, are
+// the FP16 subnormals q * 2^-20; one fused multiply-add with b2 = s * 2^20 and
+// c2 = -8 s computes q * s - 8 s = (q - 8) * s exactly and rounds it once, the
+// same value as the subtract-then-multiply of dequant_word_paired.  b2 and c2
+// are exact (scaling by powers of two), and b2 stays finite because |s| < 2^-4.
+// Pairs (k1, k5) and (k3, k7) take this form; (k0, k4) and (k2, k6) keep the
+// magic-number form, which balances the FP16 and integer pipes.  Only for
+// 0 < s < 2^-4: with s <= 0 the sum q * s - 8 s can give +0 where the
+// definition's product gives -0.
+__device__ __forceinline__ bool scale_fits_subnormal_form(uint32_t s2) {
+  return (s2 & 0xFFFFu) - 1u < 0x2BFFu;  // the low half's bits in 0x0001 .. 0x2BFF
+}
+
+__device__ __forceinline__ void subnormal_form_constants(uint32_t s2, uint32_t& b2, uint32_t& c2) {
+  constexpr uint32_t k1024 = 0x64006400u;     // half2(1024, 1024)
+  constexpr uint32_t kMinus8 = 0xC800C800u;   // half2(-8, -8)
+  b2 = hmul2_rn(hmul2_rn(s2, k1024), k1024);  // s * 2^20, exact
+  c2 = hmul2_rn(s2, kMinus8);                 // -8 s, exact
+}
+
+__device__ __forceinline__ uint32_t and_b32(uint32_t a, uint32_t m) {
+  uint32_t r;
+  asm("and.b32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(m));
+  return r;
+}
+
+__device__ __forceinline__ void dequant_word_paired_small_scale(uint32_t w, uint32_t s2,
+                                                                uint32_t b2, uint32_t c2,
+                                                                uint32_t p[4]) {
+  const uint32_t w8 = w >> 8;
+  p[0] = hmul2_rn(hsub2_rn(lop3_and_or(w, 0x000F000Fu, kMagic1024), kMinus1032), s2);
+  p[1] = hfma2_rn(and_b32(w, 0x00F000F0u), b2, c2);
+  p[2] = hmul2_rn(hsub2_rn(lop3_and_or(w8, 0x000F000Fu, kMagic1024), kMinus1032), s2);
+  p[3] = hfma2_rn(and_b32(w8, 0x00F000F0u), b2, c2);
+}
+
 // Same, in natural k order: n[j] = (k_{2j}, k_{2j+1}).
 __device__ __forceinline__ void dequant_word_natural(uint32_t w, uint32_t s2, uint32_t n[4]) {
   uint32_t p[4];

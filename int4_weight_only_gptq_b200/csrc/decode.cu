@@ -542,6 +542,30 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint8_t* sc = st + S_OFF + col * 2;
           uint32_t cells[4 * WPT];
           uint32_t s2 = 0, zlo = 0, zhi = 0;
+          if constexpr (!ASYM && WPS >= 4) {
+            // symmetric weights, a scale per four or more words: the
+            // six-operation form where the scale allows it (same values)
+#pragma unroll
+            for (int g = 0; g < WPT / WPS; ++g) {
+              const int row = (8 * (row0 + WPS * g)) >> gs;
+              s2 = half2_broadcast(*reinterpret_cast<const uint16_t*>(sc + row * S_ROW_BYTES));
+              uint32_t w[WPS];
+#pragma unroll
+              for (int i = 0; i < WPS; ++i)
+                w[i] = *reinterpret_cast<const uint32_t*>(qw + (WPS * g + i) * (BW * 4));
+              if (scale_fits_subnormal_form(s2)) {
+                uint32_t b2, c2;
+                subnormal_form_constants(s2, b2, c2);
+#pragma unroll
+                for (int i = 0; i < WPS; ++i)
+                  dequant_word_paired_small_scale(w[i], s2, b2, c2, cells + 4 * (WPS * g + i));
+              } else {
+#pragma unroll
+                for (int i = 0; i < WPS; ++i)
+                  dequant_word_paired(w[i], s2, cells + 4 * (WPS * g + i));
+              }
+            }
+          } else {
 #pragma unroll
           for (int i = 0; i < WPT; ++i) {
             if (i % WPS == 0) {
@@ -564,6 +588,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               dequant_word_paired(w, s2, p);
 #pragma unroll
             for (int j = 0; j < 4; ++j) cells[4 * i + j] = p[j];
+          }
           }
           if (hf == HALVES - 1 && c == CHUNKS - 1) {
             __syncwarp();

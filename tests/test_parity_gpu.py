@@ -204,6 +204,37 @@ def test_one_hot_x_reproduces_dequantised_rows_bitwise(kernel):
         assert np.array_equal(y[m].view(np.uint16), w[k].view(np.uint16)), (m, k)
 
 
+@pytest.mark.parametrize("kernel", [B.KERNEL_DECODE, B.KERNEL_PREFILL])
+@pytest.mark.parametrize("M", [1, 16])
+def test_one_hot_x_every_scale_range_bitwise(kernel, M):
+    """Scales from subnormal to 8, negative and zero, mixed within every group of
+    columns: the decode kernel takes a six-operation form for 0 < s < 2^-4
+    and the magic-number form otherwise; both must give the definition's
+    rounded weight, so one-hot X reproduces the dequantised rows (bitwise
+    where the weight is not zero; a zero weight must come out as a zero)."""
+    K, N, G = 1024, 264, 128
+    p = W.make_problem(M, K, N, G, seed=40 + M)
+    rng = np.random.default_rng(40 + M)
+    ranges = [(2.0 ** -24, 2.0 ** -14), (2.0 ** -14, 2.0 ** -4), (2.0 ** -4, 2.0 ** -4),
+              (2.0 ** -4, 1.0), (1.0, 8.0)]
+    pick = rng.integers(0, len(ranges), size=p.scales.shape)
+    lo = np.array([r[0] for r in ranges])[pick]
+    hi = np.array([r[1] for r in ranges])[pick]
+    mag = np.exp(rng.uniform(np.log(lo), np.log(hi)))
+    sign = np.where(rng.random(p.scales.shape) < 0.15, -1.0, 1.0)
+    s = (sign * mag).astype(np.float16)
+    s[rng.random(p.scales.shape) < 0.03] = 0
+    p.scales[:] = s
+    ks = rng.integers(0, K, size=M)
+    p.x[:] = 0
+    p.x[np.arange(M), ks] = 1
+    y = run(p, kernel)
+    w = oracle.dequant(p.qweight, p.scales, G)[ks]
+    nz = w != 0
+    assert np.array_equal(y[nz].view(np.uint16), w[nz].view(np.uint16))
+    assert np.all(y[~nz] == 0)
+
+
 def test_one_hot_x_pair_tile_bitwise():
     """256 tokens = both halves of a CTA-pair tile (rows 0..127 loaded by
     the even CTA, 128..255 by the odd one), 264 columns = two pairs, the
