@@ -252,6 +252,14 @@ def copies_for(p, l2_bytes: int) -> int:
     return max(1, math.ceil(2 * l2_bytes / per) + 1)
 
 
+def hold_device(torch, us: float = 50.0):
+    """A short device-side wait enqueued before the start event, outside the
+    timed region: the graph replay behind it is already submitted when the
+    start event is reached, so the timed region holds the device's work and
+    not the host's submission latency (the end-to-end line keeps that)."""
+    torch.cuda._sleep(int(us * 2000))
+
+
 def time_loop(torch, fn, make_argv, steps, warmup, graph=True):
     """Device time per call (ms) of `steps` back-to-back calls fn(*argv[i % n]),
     argv = make_argv(stream handle), after `warmup` untimed calls.
@@ -282,6 +290,7 @@ def time_loop(torch, fn, make_argv, steps, warmup, graph=True):
                     raise RuntimeError(f"status {st} while capturing")
         g.replay()
         torch.cuda.synchronize()
+        hold_device(torch)
         e0.record(stream)
         g.replay()
         e1.record(stream)
@@ -442,6 +451,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank, str(getattr(props, "uuid", "")) or None) as clk:
+        hold_device(torch)
         e0.record(stream)
         graph.replay()
         e1.record(stream)
@@ -508,7 +518,7 @@ def run_ours(args):
             "config": {"workload": desc, "M": p.M, "K": p.K, "N": p.N, "group": p.group,
                        "bytes_per_step": bytes_per_step,
                        "l2": f"rotating {copies} input copies ({copies * bytes_per_step / 1e6:.0f} MB > 2x L2 {l2 / 1e6:.0f} MB)",
-                       "timing": "the steps captured once as a CUDA graph of library calls, replayed once untimed and once timed (CUDA events on the replay stream)",
+                       "timing": "the steps captured once as a CUDA graph of library calls, replayed once untimed and once timed (CUDA events on the replay stream; a 50 us device-side wait is queued before the start event, so the timed region holds no host submission latency)",
                        "parallelism": f"replicas x{world} (no exchange)",
                        "kernel": {1: "decode", 2: "prefill"}.get(kernel_id, kernel_id),
                        "split_k_ctas": split},
