@@ -61,14 +61,15 @@ typedef enum {
 /* Kernel identifiers reported by gptq_w4a16_select and accepted by
  * gptq_w4a16_gemm_kernel. */
 #define GPTQ_KERNEL_AUTO 0
-#define GPTQ_KERNEL_DECODE 1   /* M <= 32: streams qweight, split-K, tcgen05 MMA   */
+#define GPTQ_KERNEL_DECODE 1   /* M <= 64: streams qweight, split-K, tcgen05 MMA   */
 #define GPTQ_KERNEL_PREFILL 2  /* any M: TMA + tcgen05 MMA with TMEM accumulators  */
 
 /* Size limits (inclusive). */
 #define GPTQ_MAX_K 65536
 #define GPTQ_MAX_N 1048576
 #define GPTQ_MAX_M 8388608
-#define GPTQ_DECODE_MAX_M 32
+#define GPTQ_DECODE_MAX_M 64
+#define GPTQ_LORA_DECODE_MAX_M 32 /* gptq_w4a16_gemm_lora: decode kernel up to here */
 #define GPTQ_MAX_GROUPED 8     /* linears per gptq_w4a16_gemm_grouped call */
 #define GPTQ_MAX_LORA_RANK 256 /* largest adapter rank of gptq_w4a16_gemm_lora */
 #define GPTQ_LORA_SCRATCH_BYTES (8 << 20) /* T buffer of gptq_w4a16_gemm_lora_noalloc */
@@ -177,8 +178,8 @@ GPTQ_API int gptq_w4a16_gemm_asym(const uint16_t* x, const int32_t* qweight,
  * T is summed in FP32 and rounded to FP16; T . lora_b^T is added to the
  * layer's FP32 accumulator (the adapter's rank is extra K of the same
  * tensor-core product) and Y is rounded once.  Two launches on `stream`: T,
- * then the layer, which follows M as in gptq_w4a16_gemm (decode up to
- * GPTQ_DECODE_MAX_M, prefill above) and may start while T is computed (it
+ * then the layer, which runs on the decode kernel up to
+ * GPTQ_LORA_DECODE_MAX_M tokens and on the prefill kernel above and may start while T is computed (it
  * waits for T only before reading it).  Other arguments, checks
  * and errors as gptq_w4a16_gemm, plus GPTQ_ERR_NULL for a NULL lora_a, lora_b
  * or t_work (when M > 0), GPTQ_ERR_SHAPE for a rank out of range, and

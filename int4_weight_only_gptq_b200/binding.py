@@ -18,7 +18,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libgptq_w4a16.so")
 
 KERNEL_AUTO, KERNEL_DECODE, KERNEL_PREFILL = 0, 1, 2
-DECODE_MAX_M = 32
+DECODE_MAX_M = 64
+LORA_DECODE_MAX_M = 32
 MAX_GROUPED = 8
 MAX_LORA_RANK = 256
 LORA_SCRATCH_BYTES = 8 << 20

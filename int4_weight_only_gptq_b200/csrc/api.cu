@@ -104,7 +104,7 @@ bool overlaps(const void* a, int64_t abytes, const void* b, int64_t bbytes) {
 
 int select_kernel(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev, int32_t* split) {
   if (M <= GPTQ_DECODE_MAX_M) {
-    if (split) *split = decode_pick_splits(M, K, N, dev);
+    if (split) *split = decode_pick_splits(M, K, N, false, dev);
     return GPTQ_KERNEL_DECODE;
   }
   if (split) *split = 1;
@@ -179,16 +179,16 @@ int lora_impl(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
   if (st != GPTQ_OK) return st;
   if (static_t) t_work = dev->lora_scratch;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // up to 32 tokens the layer runs on the decode kernel, one CTA per SM: the
-  // T launch may use the SMs it leaves free
+  // up to GPTQ_LORA_DECODE_MAX_M tokens the layer runs on the decode kernel,
+  // one CTA per SM: the T launch may use the SMs it leaves free
   int free_sms = 0;
-  if (M <= GPTQ_DECODE_MAX_M) {
-    const int64_t ctas = decode_ctas(M, K, N, *dev);
+  if (M <= GPTQ_LORA_DECODE_MAX_M) {
+    const int64_t ctas = decode_ctas(M, K, N, true, *dev);
     free_sms = ctas < dev->num_sms ? (int)(dev->num_sms - ctas) : 0;
   }
   cudaError_t e = launch_lora_down(x, lora_a, t_work, M, K, rank, free_sms, s, *dev);
   if (e == cudaSuccess)
-    e = M <= GPTQ_DECODE_MAX_M
+    e = M <= GPTQ_LORA_DECODE_MAX_M
             ? launch_decode_lora(x, qweight, scales, y, M, K, N, group_shift_of(group), t_work,
                                  lora_b, rank, s, *dev)
             : launch_prefill_pair_lora(x, qweight, scales, y, M, K, N, group_shift_of(group),

@@ -1,4 +1,4 @@
-// Decode kernel: Y[M, N] = X[M, K] . dequant(qweight, scales) for M <= 32,
+// Decode kernel: Y[M, N] = X[M, K] . dequant(qweight, scales) for M <= 64,
 // on the 5th-generation tensor cores (tcgen05) with TMEM accumulators.
 //
 // Operation: GPTQ-Pro README, "Runtime contract" and "Ampere kernel
@@ -10,12 +10,16 @@
 //
 // * The product is computed transposed, Y^T = W^T . X^T: a CTA owns 128 weight
 //   columns (the MMA's M, one TMEM lane each) and a range of K; the tokens are
-//   the MMA's N = BT, 16 or 32 (rows at or beyond M read as zero).
-// * One TMA producer thread streams, per 512-k stage, the qweight tile [64
-//   packed rows x 128 columns] (32 KB), the scale rows of the stage and the X
-//   tile [BT tokens x 512 k] (FP16, 128-byte swizzle: the B operand; one 3-D
-//   box when K is a multiple of 64) into a ring of stages in shared memory
-//   (three or four fit in the 224 KB budget).
+//   the MMA's N = BT, 16, 32, 48 or 64 (rows at or beyond M read as zero).
+// * One TMA producer thread streams, per stage of 512 or 256 k, the qweight
+//   tile [64 or 32 packed rows x 128 columns] (32 or 16 KB), the scale rows of
+//   the stage and the X tile [BT tokens x the stage's k] (FP16, 128-byte
+//   swizzle: the B operand; one 3-D box when K is a multiple of 64) into a
+//   ring of stages in shared memory (224 KB: two to eight stages, depending
+//   on BT and the stage's k).  512-k stages serve the 16-token tile when a
+//   CTA streams the whole K of its columns, and adapters; 256-k stages
+//   everything else (a split K range, or a token tile whose X leaves room for
+//   only two or three 512-k stages).
 // * Sixteen dequantisation warps in two groups of eight take alternate stages
 //   (so one group's waits overlap the other's arithmetic); in a group, two
 //   k-slices x four TMEM lane quarters each turn eight words of their column
@@ -69,10 +73,7 @@ namespace {
 
 constexpr int BW = 128;                  // weight columns per CTA (MMA M)
 constexpr int BKA = 256;                 // k per A slot fill (16 MMAs of k16)
-constexpr int HALVES = 2;                // A slot fills per ring stage
-constexpr int BKS = BKA * HALVES;        // k per ring stage
 constexpr int PRA = BKA / 8;             // packed rows per A slot fill
-constexpr int PRS = BKS / 8;             // packed rows per ring stage
 constexpr int GROUPS = 2;                // dequantisation groups, taking alternate stages
 constexpr int SLICES = 2;                // k slices of an A slot fill within a group
 constexpr int WPT = 8;                   // words per TMEM store (32 columns)
@@ -80,12 +81,9 @@ constexpr int CHUNKS = PRA / (SLICES * WPT);  // TMEM stores per thread per fill
 constexpr int GROUP_WARPS = 4 * SLICES;  // four TMEM lane quarters per slice
 constexpr int DQ_WARPS = GROUPS * GROUP_WARPS;
 constexpr int THREADS = (2 + DQ_WARPS) * 32;
-constexpr int X_ATOMS = BKS / 64;
-constexpr int QW_STAGE_BYTES = PRS * BW * 4;
 // A LoRA stage's lora_b tile: 128 rows x 64 ranks (128-byte rows, 128-byte
 // swizzle) per half, two halves in the qweight area.
 constexpr int LORA_HALF_BYTES = BW * 64 * 2;
-static_assert(2 * LORA_HALF_BYTES <= QW_STAGE_BYTES, "a LoRA stage fits the qweight area");
 constexpr int S_ROW_BYTES = BW * 2;
 constexpr int Z_ROW_BYTES = BW / 8 * 4;  // one row of packed zero points (asymmetric weights)
 constexpr int kMaxStages = 8;
@@ -100,12 +98,20 @@ constexpr uint64_t kDrainLimitNs = 200000000ull;
 
 static_assert(A_COL0 + A_SLOTS * A_SLOT_COLS <= TMEM_COLS, "TMEM budget");
 
-// Geometry that depends on the token tile BT (the MMA's N): a stage holds X
-// as X_ATOMS atoms of [BT tokens x 64 k] (128-byte swizzle), then qweight,
-// then the scale rows.
-template <int BT_>
+// Geometry that depends on the token tile BT (the MMA's N) and on the packed
+// rows per ring stage PRS (64: 512 k, two A slot fills; 32: 256 k, one
+// fill): a stage holds X as X_ATOMS atoms of [BT tokens x 64 k] (128-byte
+// swizzle), then qweight, then the scale rows.
+template <int BT_, int PRS_>
 struct TokGeo {
   static constexpr int BT = BT_;
+  static constexpr int PRS = PRS_;                   // packed rows per ring stage
+  static constexpr int BKS = 8 * PRS;                // k per ring stage
+  static constexpr int HALVES = BKS / BKA;           // A slot fills per ring stage
+  static constexpr int X_ATOMS = BKS / 64;
+  static constexpr int QW_STAGE_BYTES = PRS * BW * 4;
+  // adapter stages need room for two lora_b halves in the qweight area
+  static constexpr bool LORA_OK = 2 * LORA_HALF_BYTES <= QW_STAGE_BYTES;
   static constexpr int X_ATOM_BYTES = BT * 128;
   static constexpr int X_STAGE_BYTES = X_ATOMS * X_ATOM_BYTES;
   static constexpr int QW_OFF = X_STAGE_BYTES;
@@ -113,6 +119,7 @@ struct TokGeo {
   // independent accumulators (the k16 steps go round-robin), NACC x BT <= 128
   static constexpr int NACC = 128 / BT < 4 ? 128 / BT : 4;
   static_assert(BT % 16 == 0 && BT >= 16 && BT <= 64, "token tile");
+  static_assert(PRS == PRA || PRS == 2 * PRA, "a stage is one or two A slot fills");
   static_assert(D_COL + NACC * BT <= A_COL0, "accumulators below the A slots");
   static_assert(BT * BW * 4 <= X_STAGE_BYTES + QW_STAGE_BYTES, "reduction buffer fits a stage");
 };
@@ -127,14 +134,17 @@ struct DecodeShape {
 
 inline int align1024(int v) { return (v + 1023) & ~1023; }
 
-// Stages start on multiples of 512 k and groups are powers of two, so a
-// stage touches 512 / group scale rows (one for groups of 512 and more).
+// Stages start on multiples of their k extent BKS (512 or 256) and groups
+// are powers of two, so a stage touches BKS / group scale rows (one for
+// groups of BKS and more).
 // With zero points (asym) each stage also holds their rows after the scales.
-template <int BT>
+template <int BT, int PRS>
 inline DecodeShape decode_shape(int group_shift, bool asym = false) {
   DecodeShape d;
-  d.scale_rows = group_shift >= 9 ? 1 : (BKS >> group_shift);
-  d.stage_bytes = align1024(TokGeo<BT>::S_OFF +
+  constexpr int BKS = TokGeo<BT, PRS>::BKS;
+  const int gs = group_shift < 30 ? group_shift : 30;  // group -1 has shift 62
+  d.scale_rows = (BKS >> gs) > 1 ? (BKS >> gs) : 1;
+  d.stage_bytes = align1024(TokGeo<BT, PRS>::S_OFF +
                             d.scale_rows * (S_ROW_BYTES + (asym ? Z_ROW_BYTES : 0)));
   const int s = kRingBudget / d.stage_bytes;
   d.stages = s > kMaxStages ? kMaxStages : s;
@@ -209,18 +219,23 @@ __device__ __forceinline__ void permute_x_chunk(uint8_t* p) {
 // swizzle), T's rows to the X area (two 64-rank atoms); one fill per stage
 // copies lora_b into the A slot in the paired k order (T is permuted like X),
 // and the MMAs add T . lora_b^T to the same accumulators.
-template <int WPS, int BT, bool ASYM>
+template <int WPS, int BT, int PRS_, bool ASYM>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ LinearSet ls,
                   const __grid_constant__ CUtensorMap qz_map,
                   const __grid_constant__ CUtensorMap t_map,
                   const __grid_constant__ CUtensorMap b_map, int M, int K, int group_shift,
                   int stages, int stage_bytes, int scale_rows, int x3d, int lora_rank, int* err) {
-  constexpr int X_ATOM_BYTES = TokGeo<BT>::X_ATOM_BYTES;
-  constexpr int X_STAGE_BYTES = TokGeo<BT>::X_STAGE_BYTES;
-  constexpr int QW_OFF = TokGeo<BT>::QW_OFF;
-  constexpr int S_OFF = TokGeo<BT>::S_OFF;
-  constexpr int NACC = TokGeo<BT>::NACC;
+  constexpr int X_ATOM_BYTES = TokGeo<BT, PRS_>::X_ATOM_BYTES;
+  constexpr int X_STAGE_BYTES = TokGeo<BT, PRS_>::X_STAGE_BYTES;
+  constexpr int QW_OFF = TokGeo<BT, PRS_>::QW_OFF;
+  constexpr int S_OFF = TokGeo<BT, PRS_>::S_OFF;
+  constexpr int NACC = TokGeo<BT, PRS_>::NACC;
+  constexpr int PRS = TokGeo<BT, PRS_>::PRS;
+  constexpr int BKS = TokGeo<BT, PRS_>::BKS;
+  constexpr int HALVES = TokGeo<BT, PRS_>::HALVES;
+  constexpr int X_ATOMS = TokGeo<BT, PRS_>::X_ATOMS;
+  constexpr int QW_STAGE_BYTES = TokGeo<BT, PRS_>::QW_STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array itself so that the
   // compiler keeps the shared address space (plain LDS, no generic loads)
@@ -243,7 +258,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int st_end = (int)((int64_t)(blockIdx.y + 1) * NS / splits);
   const int n_st = st_end - st_begin;
   // LoRA stages of this CTA (the last of the column block's split), then all
-  const int n_lora = (lora_rank > 0 && (int)blockIdx.y == splits - 1) ? (lora_rank + 127) / 128 : 0;
+  const int n_lora = (TokGeo<BT, PRS_>::LORA_OK && lora_rank > 0 && (int)blockIdx.y == splits - 1)
+                         ? (lora_rank + 127) / 128 : 0;
   const int n_tot = n_st + n_lora;
   const int gs = min(group_shift, 30);        // group -1 (shift 62): row 0 throughout
   const int z_off = S_OFF + scale_rows * S_ROW_BYTES;  // zero-point rows (ASYM)
@@ -476,11 +492,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar->full[s], ph, abort_flag, kWaitLimitNs));
       if (!ok) break;
       uint8_t* st = smem + s * stage_bytes;
-      // chunk j: token row j / 64, 64-k atom (j % 64) / 8, chunk (j % 8) of
-      // the 128-byte row (every chunk of the row is permuted, so the swizzle
-      // does not matter); rows >= M are zero and stay so
+      // chunk j: token row j / CPR, 64-k atom (j % CPR) / 8, chunk (j % 8) of
+      // the 128-byte row, CPR = BKS / 8 chunks per row (every chunk of the
+      // row is permuted, so the swizzle does not matter); rows >= M are zero
+      // and stay so
+      constexpr int CPR = BKS / 8;
       for (int j = gid; j < x_chunks; j += GROUP_WARPS * 32)
-        permute_x_chunk(st + ((j & 63) >> 3) * X_ATOM_BYTES + (j >> 6) * 128 + (j & 7) * 16);
+        permute_x_chunk(st + ((j % CPR) >> 3) * X_ATOM_BYTES + (j / CPR) * 128 + (j & 7) * 16);
 
       if (t >= n_st) {
         // LoRA stage: one fill.  Row rho (eight ranks) of this slice's chunks
@@ -684,7 +702,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int WPS, int BT, bool ASYM>
+template <int WPS, int BT, int PRS, bool ASYM>
 cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtensorMap& qz_map,
                      const CUtensorMap& t_map, const CUtensorMap& b_map, int lora_rank, int M,
                      int K, int group_shift, int splits, int x3d, const DecodeShape& d,
@@ -693,7 +711,7 @@ cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtens
   static cudaError_t attr_err[64];
   const int di = dev.device & 63;
   std::call_once(once[di], [&] {
-    attr_err[di] = cudaFuncSetAttribute(decode_kernel<WPS, BT, ASYM>,
+    attr_err[di] = cudaFuncSetAttribute(decode_kernel<WPS, BT, PRS, ASYM>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         1024 + kRingBudget + 256);
   });
@@ -717,7 +735,7 @@ cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtens
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT, ASYM>, x_map, ls, qz_map, t_map, b_map,
+  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT, PRS, ASYM>, x_map, ls, qz_map, t_map, b_map,
                             M, K, group_shift, d.stages, d.stage_bytes, d.scale_rows, x3d,
                             lora_rank, dev.error_word);
 }
@@ -741,14 +759,15 @@ struct LinearExtras {
   int64_t rank = 0;
 };
 
-template <int BT>
+template <int BT, int PRS>
 cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count,
                       const LinearExtras& ex, int64_t M, int64_t K, int group_shift, int splits,
                       cudaStream_t stream, const DeviceInfo& dev) {
   const int32_t* qzeros = ex.qzeros;
   const bool asym = qzeros != nullptr;
   if ((asym || ex.rank > 0) && count != 1) return cudaErrorInvalidValue;
-  const DecodeShape d = decode_shape<BT>(group_shift, asym);
+  if (ex.rank > 0 && !TokGeo<BT, PRS>::LORA_OK) return cudaErrorInvalidValue;
+  const DecodeShape d = decode_shape<BT, PRS>(group_shift, asym);
   if (d.stages < GROUPS || d.smem_bytes > 1024 + kRingBudget + 256) return cudaErrorInvalidValue;
   if (count < 1 || count > kMaxLinears) return cudaErrorInvalidValue;
   const int64_t n_groups = (group_shift == 62 || (int64_t(1) << group_shift) >= K)
@@ -783,7 +802,7 @@ cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count,
   if (K % 64 == 0) {
     const uint64_t dims[3] = {64, (uint64_t)M, (uint64_t)(K / 64)};
     const uint64_t strides[2] = {(uint64_t)K * 2, 128};
-    const uint32_t box[3] = {64, BT, X_ATOMS};
+    const uint32_t box[3] = {64, BT, TokGeo<BT, PRS>::X_ATOMS};
     x3d = tensor_map_3d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, dims, strides, box,
                         CU_TENSOR_MAP_SWIZZLE_128B) ? 1 : 0;
   }
@@ -809,7 +828,7 @@ cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count,
                        (uint64_t)lora_rank * 2, 64, BW, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
-  if (splits <= 0) splits = decode_pick_splits_blocks(ls.blk0[count], K, dev);
+  if (splits <= 0) splits = decode_pick_splits_blocks(ls.blk0[count], K, PRS, dev);
   // with an adapter, the last split's CTA (which runs the LoRA stages after
   // its K stages) must own at least one K stage: the first MMAs of its K
   // stages are what initialise its accumulators
@@ -820,39 +839,49 @@ cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count,
   const int iM = (int)M, iK = (int)K;
   if (asym) {
     if (group_shift == 4)
-      return launch_t<2, BT, true>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
+      return launch_t<2, BT, PRS, true>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
                                    group_shift, splits, x3d, d, stream, dev);
     if (group_shift == 5)
-      return launch_t<4, BT, true>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
+      return launch_t<4, BT, PRS, true>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
                                    group_shift, splits, x3d, d, stream, dev);
-    return launch_t<WPT, BT, true>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
+    return launch_t<WPT, BT, PRS, true>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
                                    group_shift, splits, x3d, d, stream, dev);
   }
   if (group_shift == 4)
-    return launch_t<2, BT, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
+    return launch_t<2, BT, PRS, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
                                   splits, x3d, d, stream, dev);
   if (group_shift == 5)
-    return launch_t<4, BT, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
+    return launch_t<4, BT, PRS, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
                                   splits, x3d, d, stream, dev);
-  return launch_t<WPT, BT, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
+  return launch_t<WPT, BT, PRS, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
                                   splits, x3d, d, stream, dev);
 }
 
 cudaError_t launch_set(const uint16_t* x, const LinearArgs* lin, int count,
                        const LinearExtras& ex, int64_t M, int64_t K, int group_shift, int splits,
                        cudaStream_t stream, const DeviceInfo& dev) {
-  // token tile: 16 tokens up to M = 16, else 32
-  if (M <= 16) return launch_bt<16>(x, lin, count, ex, M, K, group_shift, splits, stream, dev);
-  return launch_bt<32>(x, lin, count, ex, M, K, group_shift, splits, stream, dev);
+  int64_t nblk = 0;
+  for (int i = 0; i < count; ++i) nblk += (lin[i].n + BW - 1) / BW;
+  const bool wide = decode_stage_rows(M, nblk, K, splits, ex.rank > 0, dev) == 2 * PRA;
+  // token tile: the smallest of 16, 32, 48 and 64 that holds M
+  if (M <= 16)
+    return wide ? launch_bt<16, 2 * PRA>(x, lin, count, ex, M, K, group_shift, splits, stream, dev)
+                : launch_bt<16, PRA>(x, lin, count, ex, M, K, group_shift, splits, stream, dev);
+  if (M <= 32)
+    return wide ? launch_bt<32, 2 * PRA>(x, lin, count, ex, M, K, group_shift, splits, stream, dev)
+                : launch_bt<32, PRA>(x, lin, count, ex, M, K, group_shift, splits, stream, dev);
+  if (ex.rank > 0) return cudaErrorInvalidValue;  // adapters: up to 32 tokens
+  if (M <= 48) return launch_bt<48, PRA>(x, lin, count, ex, M, K, group_shift, splits, stream, dev);
+  return launch_bt<64, PRA>(x, lin, count, ex, M, K, group_shift, splits, stream, dev);
 }
 
 }  // namespace
 
-int decode_pick_splits_blocks(int64_t nblk, int64_t K, const DeviceInfo& dev) {
+int decode_pick_splits_blocks(int64_t nblk, int64_t K, int prs, const DeviceInfo& dev) {
   // One CTA per SM.  Pick the split that minimises (waves of CTAs) x (stages
   // per CTA) plus one stage for the cluster reduction, among splits whose
   // CTAs are all resident at once.  Ties go to the smaller split.
-  const int64_t ns = ((K >> 3) + PRS - 1) / PRS;
+  const int64_t ns = ((K >> 3) + prs - 1) / prs;
   const int64_t sms = dev.num_sms;
   int best = 1;
   int64_t best_cost = -1;
@@ -868,13 +897,28 @@ int decode_pick_splits_blocks(int64_t nblk, int64_t K, const DeviceInfo& dev) {
   return best;
 }
 
-int decode_pick_splits(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev) {
-  (void)M;
-  return decode_pick_splits_blocks((N + BW - 1) / BW, K, dev);
+int decode_stage_rows(int64_t M, int64_t nblk, int64_t K, int splits, bool lora,
+                      const DeviceInfo& dev) {
+  // An adapter's stages need the 512-k stage's qweight area (two 64-rank
+  // lora_b halves).  Otherwise the 16-token tile streams 512-k stages (four
+  // fit the ring) when each CTA takes the whole K range of its columns, where
+  // fewer, larger copies cost less per byte, and 256-k stages (eight) when the
+  // K range is split, where a CTA's share is short and the ring's fill and
+  // drain weigh more.  Larger tiles take 256-k stages: their X tiles leave
+  // room for only two or three 512-k stages.
+  if (lora) return 2 * PRA;
+  if (M > 16) return PRA;
+  const int s = splits > 0 ? splits : decode_pick_splits_blocks(nblk, K, 2 * PRA, dev);
+  return s == 1 ? 2 * PRA : PRA;
 }
 
-int64_t decode_ctas(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev) {
-  return (N + BW - 1) / BW * decode_pick_splits(M, K, N, dev);
+int decode_pick_splits(int64_t M, int64_t K, int64_t N, bool lora, const DeviceInfo& dev) {
+  const int64_t nblk = (N + BW - 1) / BW;
+  return decode_pick_splits_blocks(nblk, K, decode_stage_rows(M, nblk, K, 0, lora, dev), dev);
+}
+
+int64_t decode_ctas(int64_t M, int64_t K, int64_t N, bool lora, const DeviceInfo& dev) {
+  return (N + BW - 1) / BW * decode_pick_splits(M, K, N, lora, dev);
 }
 
 cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,

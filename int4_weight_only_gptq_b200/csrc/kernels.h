@@ -32,10 +32,14 @@ cudaError_t launch_dequant(const int32_t* qweight, const uint16_t* scales, int64
                            int group_shift, uint16_t* w_out, cudaStream_t stream,
                            const DeviceInfo& dev);
 
-// Decode (M <= 32).  splits = number of CTAs that share one column block along
+// Decode (M <= 64).  splits = number of CTAs that share one column block along
 // K (the cluster size, 1..8); 0 picks it from the shape.
-int decode_pick_splits(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev);
-int decode_pick_splits_blocks(int64_t column_blocks, int64_t K, const DeviceInfo& dev);
+int decode_pick_splits(int64_t M, int64_t K, int64_t N, bool lora, const DeviceInfo& dev);
+// Packed rows per ring stage of a decode launch (64: 512 k, 32: 256 k) for M
+// tokens over nblk column blocks; splits = 0 when the launch picks it.
+int decode_stage_rows(int64_t M, int64_t nblk, int64_t K, int splits, bool lora,
+                      const DeviceInfo& dev);
+int decode_pick_splits_blocks(int64_t column_blocks, int64_t K, int prs, const DeviceInfo& dev);
 cudaError_t launch_decode(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                           uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
                           int splits, cudaStream_t stream, const DeviceInfo& dev);
@@ -90,6 +94,6 @@ cudaError_t launch_lora_down(const uint16_t* x, const uint16_t* lora_a, uint16_t
                              int64_t K, int64_t r, int free_sms, cudaStream_t stream,
                              const DeviceInfo& dev);
 // CTAs of one decode launch of this shape (column blocks x K split).
-int64_t decode_ctas(int64_t M, int64_t K, int64_t N, const DeviceInfo& dev);
+int64_t decode_ctas(int64_t M, int64_t K, int64_t N, bool lora, const DeviceInfo& dev);
 
 }  // namespace gptq

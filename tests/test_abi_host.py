@@ -64,7 +64,7 @@ def call(lib, x=X, qw=QW, s=S, M=4, K=512, N=256, g=128, y=Y, kernel=None):
     (dict(qw=0), 1), (dict(s=0), 1), (dict(x=0), 1), (dict(y=0), 1),
     (dict(x=X + 2), 4), (dict(qw=QW + 4), 4), (dict(s=S + 8), 4), (dict(y=Y + 2), 4),
     (dict(y=X), 8), (dict(y=QW + 16), 8), (dict(y=S), 8),
-    (dict(kernel=3), 9), (dict(kernel=-1), 9), (dict(kernel=1, M=33), 9),
+    (dict(kernel=3), 9), (dict(kernel=-1), 9), (dict(kernel=1, M=65), 9),
 ])
 def test_gemm_argument_checks(lib, kw, status):
     assert call(lib, **kw) == status

@@ -5,7 +5,7 @@ whose bytes are a seeded random pattern.  After the call, the bytes before and
 after the output must still hold the pattern, and the inputs must be unchanged:
 no kernel may write outside the output it was given, also on ragged shapes
 (M, N and K that are not multiples of the tiles, a ragged last group) and in
-every kernel path (decode 16- and 32-token tiles, K splits reduced over a
+every kernel path (decode 16- to 64-token tiles, K splits reduced over a
 cluster, forced single-CTA prefill, pair prefill with 128- and 256-token tiles,
 grouped linears, asymmetric zeros, the LoRA adapter in both kernels, the
 dequantisation entry).  Fail-closed execution is part of the contract (GPTQ-Pro
@@ -82,6 +82,8 @@ LAYER_CASES = [  # (label, M, K, N, G, kernel, splits)
     ("decode 32-token tile", 27, 1040, 264, 16, B.KERNEL_DECODE, 0),
     ("decode K split over a cluster", 3, 5120, 136, 128, B.KERNEL_AUTO, 4),
     ("decode K split, ragged K", 16, 2064, 72, 32, B.KERNEL_AUTO, 3),
+    ("decode 48-token tile", 41, 1040, 136, 32, B.KERNEL_AUTO, 0),
+    ("decode 64-token tile, K split", 63, 2064, 264, 128, B.KERNEL_AUTO, 2),
     ("forced single-CTA prefill", 20, 528, 136, 64, B.KERNEL_PREFILL, 0),
     ("pair prefill 128-token tile", 100, 528, 392, 128, B.KERNEL_AUTO, 0),
     ("pair prefill 256-token tile", 300, 1040, 264, -1, B.KERNEL_AUTO, 0),

@@ -120,12 +120,15 @@ def test_tiny(M, kernel):
 EDGE = [  # (M, K, N, G)
     (1, 16, 8, -1), (3, 48, 40, 16), (5, 528, 24, 128), (7, 96, 72, 32), (8, 160, 264, 64),
     (9, 64, 8, 16), (13, 1040, 136, 1024), (16, 272, 520, 16), (2, 5120, 8, 512),
-    # K-stages that straddle group boundaries (stages of 768 k for M <= 8,
-    # 512 k for M <= 16), ragged last stages
+    # K-stages that straddle group boundaries (stages of 512 k, or 256 k when
+    # K is split), ragged last stages
     (4, 3072, 64, 1024), (3, 2304, 16, 512), (8, 6144, 24, 256), (1, 1600, 72, 512),
     (12, 2560, 40, 1024), (16, 1536, 200, 512),
     # the 32-token tile (17 <= M <= 32)
     (17, 528, 136, 128), (24, 2048, 72, 16), (32, 1040, 264, -1), (29, 6144, 40, 32),
+    # the 48- and 64-token tiles (33 <= M <= 64, 256-k stages)
+    (33, 528, 136, 128), (40, 2048, 72, 16), (48, 1040, 264, -1), (57, 6144, 40, 32),
+    (64, 1536, 200, 512), (49, 3072, 64, 1024), (64, 96, 8, 64),
 ]
 
 
@@ -152,16 +155,19 @@ def test_edge_shapes_small_m(M, K, N, G, kernel):
                                      (385, 96, 136, 32), (160, 64, 8, -1), (255, 1024, 24, 64)])
 def test_edge_shapes_prefill(M, K, N, G):
     p = W.make_problem(M, K, N, G, seed=M + K + N)
-    y = run(p)
+    y = run(p, B.KERNEL_PREFILL)
     ref = oracle.gemm(p.x, p.qweight, p.scales, G)
     err = rel_err(y, ref)
     print(f"[parity] prefill M={M} K={K} N={N} G={G}: {err:.3e}")
     assert err <= TOL
 
 
+@pytest.mark.parametrize("M", [6, 40, 64])
 @pytest.mark.parametrize("splits", [1, 2, 3, 4, 5, 6, 7, 8])
-def test_decode_every_split(splits):
-    p = W.make_problem(6, 2048, 200, 32, seed=splits)
+def test_decode_every_split(M, splits):
+    # M = 6: 512-k stages without a split, 256-k stages with one; M = 40 and
+    # 64: 256-k stages of the 48- and 64-token tiles
+    p = W.make_problem(M, 2048, 200, 32, seed=splits + M)
     y = run(p, splits=splits)
     ref = oracle.gemm(p.x, p.qweight, p.scales, 32)
     assert rel_err(y, ref) <= TOL
@@ -319,6 +325,15 @@ def test_decode_down_projection_sweep(M):
     check_rows(p, run(p), sample_rows(M, 3), f"decode down-projection M={M}")
 
 
+@pytest.mark.parametrize("M", [33, 48, 64, 65])
+def test_mid_m_full(M):
+    # 48- and 64-token decode tiles up to M = 64, the pair prefill above
+    p = W.prefill(M)
+    kernel = B.select(M, 5120, 17408, 128)[0]
+    assert kernel == (B.KERNEL_DECODE if M <= B.DECODE_MAX_M else B.KERNEL_PREFILL)
+    check_rows(p, run(p), sample_rows(M, 3), f"mid-M up-projection M={M}")
+
+
 @pytest.mark.parametrize("M", [512, 2048, 8192])
 def test_prefill_full(M):
     p = W.prefill(M)
@@ -360,7 +375,8 @@ def run_grouped(ps):
 
 @pytest.mark.parametrize("M,K,Ns,G", [
     (1, 2048, (264, 136, 8), 128), (5, 1040, (72, 200), 32), (16, 2560, (128, 128, 40, 8), 16),
-    (32, 1536, (136, 264), -1), (33, 528, (64, 24), 128),   # M = 33: one prefill launch each
+    (32, 1536, (136, 264), -1), (33, 528, (64, 24), 128), (64, 2064, (136, 40, 8), 32),
+    (65, 528, (64, 24), 128),                               # M = 65: one prefill launch each
     (3, 512, (8, 8, 8, 8, 8, 8, 8, 8), 64),                  # the most linears per call
 ])
 def test_grouped_parity(M, K, Ns, G):
@@ -552,10 +568,10 @@ def run_asym(p, qzeros):
 
 
 @pytest.mark.parametrize("M,K,N,G", [
-    # decode kernel (M <= 32): 16- and 32-token tiles, groups of 16 and 32
+    # decode kernel (M <= 64): 16- to 64-token tiles, groups of 16 and 32
     (1, 512, 256, 128), (5, 512, 256, 16), (7, 1024, 160, 32), (16, 2048, 288, -1),
-    (24, 1040, 224, 128), (32, 6144, 96, 64),
-    (33, 528, 128, 16),                 # 128-token pair tile, ragged K and last group
+    (24, 1040, 224, 128), (32, 6144, 96, 64), (33, 528, 128, 16), (64, 2064, 160, 32),
+    (65, 528, 128, 16),                 # 128-token pair tile, ragged K and last group
     (130, 1040, 416, 64),               # 256-token pair tile, odd number of column tiles
     (300, 96, 224, 32),                 # a single k stage
     (2048, 5120, 512, 128),             # several token tiles per cluster
