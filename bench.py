@@ -371,6 +371,22 @@ def time_asym(lib, torch, p, qzeros, steps, warmup, l2_bytes):
     return ms
 
 
+def time_gidx(lib, torch, p, g_idx, steps, warmup, l2_bytes):
+    """Device time per call (ms) of back-to-back gptq_w4a16_gemm_gidx calls
+    (act-order weights), rotating weight copies past the L2 like time_gemm."""
+    copies = copies_for(p, l2_bytes) if l2_bytes else 1
+    sets = to_device(p, torch, copies)
+    gi = torch.from_numpy(g_idx).cuda()
+    v = ctypes.c_void_p
+    ng = p.scales.shape[0]
+
+    def make(sh):
+        return [(v(x.data_ptr()), v(qw.data_ptr()), v(s.data_ptr()), v(gi.data_ptr()), p.M, p.K,
+                 p.N, ng, v(y.data_ptr()), sh) for (x, qw, s, y) in sets]
+    ms, _ = time_loop(torch, lib.gptq_w4a16_gemm_gidx, make, steps, warmup)
+    return ms
+
+
 def time_lora(lib, torch, p, ad, steps, warmup, l2_bytes):
     """Device time per call (ms) of back-to-back gptq_w4a16_gemm_lora calls
     (the adapter's down-projection launch and the layer launch), rotating
@@ -580,7 +596,7 @@ def run_sweep(lib, torch, l2, hbm, tf):
 
     for M in (1, 2, 4, 8, 16, 32):
         hbm_case(f"decode_down_M{M}", W.decode_down(M))
-    # between the kernels: decode up to M = 32, pair prefill above
+    # between the kernels: decode up to M = 64, pair prefill above
     for M in (24, 32, 48, 64, 96, 128):
         hbm_case(f"midm_up_M{M}", W.make_problem(M, 5120, 17408, 128, seed=0), steps=100)
     for M in (512, 2048, 8192):
@@ -635,6 +651,25 @@ def run_sweep(lib, torch, l2, hbm, tf):
             tfl = p.flops / (ms * 1e-3) / 1e12
             entry.update({"TFLOP/s": round(tfl, 1), "frac_tensor": round(tfl / tf, 3)})
         res[f"asym_up_M{M}"] = entry
+    # act order (a group index per input channel, GPTQ's desc_act order) on
+    # the up- and down-projections; the plain layer beside it
+    for name, mk, Ms in (("up", lambda M: W.make_problem(M, 5120, 17408, 128, seed=0),
+                          (1, 16, 64, 2048)),
+                         ("down", W.decode_down, (1, 16))):
+        for M in Ms:
+            p = mk(M)
+            g = W.make_gidx(p.K, p.group, seed=0, kind="perm")
+            steps = 200 if M <= 64 else 20
+            ms = time_gidx(lib, torch, p, g, steps, 10, l2)
+            plain, _ = time_gemm(lib, torch, p, steps, 10, l2_bytes=l2)
+            entry = {"ms": round(ms, 5), "plain_ms": round(plain, 5)}
+            if M <= 64:
+                gbs = (p.algorithmic_bytes + g.size * 4) / (ms * 1e-3) / 1e9
+                entry.update({"GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)})
+            else:
+                tfl = p.flops / (ms * 1e-3) / 1e12
+                entry.update({"TFLOP/s": round(tfl, 1), "frac_tensor": round(tfl / tf, 3)})
+            res[f"gidx_{name}_M{M}"] = entry
     return res
 
 

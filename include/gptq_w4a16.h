@@ -55,7 +55,8 @@ typedef enum {
     GPTQ_ERR_CUDA = 6,     /* the CUDA runtime reported an error at launch             */
     GPTQ_ERR_TIMEOUT = 7,  /* a kernel gave up a bounded wait (see gptq_device_error)  */
     GPTQ_ERR_ALIAS = 8,    /* the output overlaps an input                            */
-    GPTQ_ERR_KERNEL = 9    /* kernel_id names no kernel, or one that cannot take M     */
+    GPTQ_ERR_KERNEL = 9,   /* kernel_id names no kernel, or one that cannot take M     */
+    GPTQ_ERR_INDEX = 10    /* a g_idx entry outside 0 .. n_groups-1 (device-reported) */
 } gptq_status;
 
 /* Kernel identifiers reported by gptq_w4a16_select and accepted by
@@ -73,6 +74,7 @@ typedef enum {
 #define GPTQ_MAX_GROUPED 8     /* linears per gptq_w4a16_gemm_grouped call */
 #define GPTQ_MAX_LORA_RANK 256 /* largest adapter rank of gptq_w4a16_gemm_lora */
 #define GPTQ_LORA_SCRATCH_BYTES (8 << 20) /* T buffer of gptq_w4a16_gemm_lora_noalloc */
+#define GPTQ_GIDX_MAX_GROUPS 640 /* scale rows of gptq_w4a16_gemm_gidx (a tile per CTA) */
 
 /*
  * Y = X . dequant(qweight, scales).
@@ -212,6 +214,34 @@ GPTQ_API int gptq_w4a16_gemm_lora_noalloc(const uint16_t* x, const int32_t* qwei
                                           int64_t N, int32_t group, const uint16_t* lora_a,
                                           const uint16_t* lora_b, int64_t rank, uint16_t* y,
                                           void* stream);
+
+/*
+ * The layer with act-order weights (GPTQ's desc_act=True checkpoints), whose
+ * input channels each carry their own group index:
+ *   Y = X . W,  W[k,n] = fp16((q[k,n] - 8) * scales[g_idx[k], n])
+ * The GPTQ-Pro README ("Runtime contract") runs desc_act=False only and puts
+ * act order outside its contract; the GPTQModel wiki names desc_act as
+ * activation ordering.  Neither gives its storage; read as GPTQ's:
+ *   g_idx    [K] int32, device, 16-byte aligned, 0 <= g_idx[k] < n_groups;
+ *            any assignment of channels to groups (group sizes need not be
+ *            equal); qweight keeps the channels in their own order
+ *   scales   [n_groups, N] FP16 bits, device
+ *   n_groups 1 .. GPTQ_GIDX_MAX_GROUPS (each CTA keeps the scale rows of its
+ *            128 columns in shared memory)
+ * With g_idx[k] = floor(k / G) the layer is gptq_w4a16_gemm's with group G,
+ * and for M <= GPTQ_DECODE_MAX_M the result is the same bit for bit.  Runs on
+ * the decode kernel for every M (tiles of at most 64 tokens; above that the
+ * weights are streamed once per tile).  An index out of range is clamped
+ * into 0 .. n_groups-1 for reading (no access outside scales) and reported
+ * as GPTQ_ERR_INDEX by gptq_device_error; the output is then undefined.
+ * Other arguments, checks and errors as gptq_w4a16_gemm (no group argument),
+ * plus GPTQ_ERR_NULL for a NULL g_idx, GPTQ_ERR_SHAPE for n_groups out of
+ * range, and GPTQ_ERR_ALIAS when y overlaps g_idx.
+ */
+GPTQ_API int gptq_w4a16_gemm_gidx(const uint16_t* x, const int32_t* qweight,
+                                  const uint16_t* scales, const int32_t* g_idx, int64_t M,
+                                  int64_t K, int64_t N, int64_t n_groups, uint16_t* y,
+                                  void* stream);
 
 /*
  * W[K, N] = dequant(qweight, scales) as FP16 bits, each value rounded once from

@@ -9,10 +9,11 @@ and fails loudly if it is missing.
 """
 __version__ = "0.1.0"
 
-_BINDING_NAMES = {"gemm", "gemm_grouped", "gemm_asym", "gemm_lora", "gemm_lora_noalloc",
-                  "dequant", "select", "device_error", "version", "load", "GptqError",
-                  "KERNEL_AUTO", "KERNEL_DECODE", "KERNEL_PREFILL", "DECODE_MAX_M", "LORA_DECODE_MAX_M",
-                  "MAX_GROUPED", "MAX_LORA_RANK", "LORA_SCRATCH_BYTES", "GROUP_SIZES"}
+_BINDING_NAMES = {"gemm", "gemm_grouped", "gemm_asym", "gemm_gidx", "gemm_lora",
+                  "gemm_lora_noalloc", "dequant", "select", "device_error", "version", "load",
+                  "GptqError", "KERNEL_AUTO", "KERNEL_DECODE", "KERNEL_PREFILL", "DECODE_MAX_M",
+                  "LORA_DECODE_MAX_M", "MAX_GROUPED", "MAX_LORA_RANK", "LORA_SCRATCH_BYTES",
+                  "GIDX_MAX_GROUPS", "GROUP_SIZES"}
 
 
 def __getattr__(name):

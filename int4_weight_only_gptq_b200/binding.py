@@ -23,16 +23,18 @@ LORA_DECODE_MAX_M = 32
 MAX_GROUPED = 8
 MAX_LORA_RANK = 256
 LORA_SCRATCH_BYTES = 8 << 20
+GIDX_MAX_GROUPS = 640
 GROUP_SIZES = (-1, 16, 32, 64, 128, 256, 512, 1024)
 
 STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_NULL", 2: "GPTQ_ERR_SHAPE", 3: "GPTQ_ERR_GROUP",
           4: "GPTQ_ERR_ALIGN", 5: "GPTQ_ERR_DEVICE", 6: "GPTQ_ERR_CUDA",
-          7: "GPTQ_ERR_TIMEOUT", 8: "GPTQ_ERR_ALIAS", 9: "GPTQ_ERR_KERNEL"}
+          7: "GPTQ_ERR_TIMEOUT", 8: "GPTQ_ERR_ALIAS", 9: "GPTQ_ERR_KERNEL",
+          10: "GPTQ_ERR_INDEX"}
 
 # Every entry point declared in include/gptq_w4a16.h.
 EXPORTS = ("gptq_w4a16_gemm", "gptq_w4a16_gemm_kernel", "gptq_w4a16_gemm_decode_splits",
-           "gptq_w4a16_gemm_grouped", "gptq_w4a16_gemm_asym", "gptq_w4a16_gemm_lora",
-           "gptq_w4a16_gemm_lora_noalloc",
+           "gptq_w4a16_gemm_grouped", "gptq_w4a16_gemm_asym", "gptq_w4a16_gemm_gidx",
+           "gptq_w4a16_gemm_lora", "gptq_w4a16_gemm_lora_noalloc",
            "gptq_dequant",
            "gptq_w4a16_select", "gptq_status_string", "gptq_device_error", "gptq_version")
 
@@ -70,6 +72,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.gptq_w4a16_gemm_lora.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32, _p, _p,
                                                  _i64, _p, _p, _p]
             lib.gptq_w4a16_gemm_asym.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32, _p, _p]
+            lib.gptq_w4a16_gemm_gidx.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p]
             lib.gptq_w4a16_gemm_lora_noalloc.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i32,
                                                          _p, _p, _i64, _p, _p]
             lib.gptq_dequant.argtypes = [_p, _p, _i64, _i64, _i32, _p, _p]
@@ -81,7 +84,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.gptq_version.restype = ctypes.c_char_p
             for name in ("gptq_w4a16_gemm", "gptq_w4a16_gemm_kernel",
                          "gptq_w4a16_gemm_decode_splits", "gptq_w4a16_gemm_grouped",
-                         "gptq_w4a16_gemm_asym", "gptq_w4a16_gemm_lora",
+                         "gptq_w4a16_gemm_asym", "gptq_w4a16_gemm_gidx", "gptq_w4a16_gemm_lora",
                          "gptq_w4a16_gemm_lora_noalloc",
                          "gptq_dequant",
                          "gptq_w4a16_select", "gptq_device_error"):
@@ -266,6 +269,42 @@ def gemm_asym(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
     with torch.cuda.device(dev):
         _check(lib.gptq_w4a16_gemm_asym(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(qzeros), M,
                                         K, N, group, _ptr(out), _stream_handle(stream, dev)))
+    return out
+
+
+def gidx_shapes(x, qweight, scales, g_idx) -> tuple[int, int, int, int]:
+    """(M, K, N, n_groups) of an act-order call, after checking x [M, K],
+    qweight [K/8, N], scales [n_groups, N] and g_idx [K]."""
+    M, K, N = layer_shapes(x, qweight, scales, 0)  # 0: scales checked below
+    if int(scales.shape[1]) != N:
+        raise ValueError(f"scales has shape {tuple(scales.shape)}, expected (n_groups, {N})")
+    if g_idx.dim() != 1 or int(g_idx.shape[0]) != K:
+        raise ValueError(f"g_idx has shape {tuple(g_idx.shape)}, expected ({K},)")
+    return M, K, N, int(scales.shape[0])
+
+
+def gemm_gidx(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
+              g_idx: torch.Tensor, out: torch.Tensor | None = None,
+              stream=None) -> torch.Tensor:
+    """Y = x . W, W[k, n] = fp16((q[k, n] - 8) * scales[g_idx[k], n]) (act
+    order): g_idx [K] int32 with entries in 0 .. n_groups - 1, scales
+    [n_groups, N], n_groups <= GIDX_MAX_GROUPS.  An out-of-range index is
+    reported by device_error() as GPTQ_ERR_INDEX."""
+    lib = load()
+    dev = qweight.device
+    _require(qweight, "qweight", lambda d: d == torch.int32, None)
+    _require(scales, "scales", lambda d: d == torch.float16, dev)
+    _require(g_idx, "g_idx", lambda d: d == torch.int32, dev)
+    _require(x, "x", lambda d: d == torch.float16, dev)
+    M, K, N, ng = gidx_shapes(x, qweight, scales, g_idx)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=dev)
+    else:
+        _require(out, "out", lambda d: d == torch.float16, dev)
+        _check_shape(out, "out", (M, N))
+    with torch.cuda.device(dev):
+        _check(lib.gptq_w4a16_gemm_gidx(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(g_idx), M, K,
+                                        N, ng, _ptr(out), _stream_handle(stream, dev)))
     return out
 
 

@@ -275,6 +275,34 @@ int gptq_w4a16_gemm_grouped(const uint16_t* x, const int32_t* const* qweights,
   return GPTQ_OK;
 }
 
+int gptq_w4a16_gemm_gidx(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                         const int32_t* g_idx, int64_t M, int64_t K, int64_t N, int64_t n_groups,
+                         uint16_t* y, void* stream) {
+  int st = check_shape(M, K, N, -1);
+  if (st != GPTQ_OK) return st;
+  if (n_groups < 1 || n_groups > GPTQ_GIDX_MAX_GROUPS) return GPTQ_ERR_SHAPE;
+  if (!qweight || !scales || !g_idx) return GPTQ_ERR_NULL;
+  if (M == 0) return GPTQ_OK;
+  if (!x || !y) return GPTQ_ERR_NULL;
+  if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(g_idx) ||
+      !aligned16(y))
+    return GPTQ_ERR_ALIGN;
+  const int64_t yb = M * N * 2;
+  if (overlaps(y, yb, x, M * K * 2) || overlaps(y, yb, qweight, K / 8 * N * 4) ||
+      overlaps(y, yb, scales, n_groups * N * 2) || overlaps(y, yb, g_idx, K * 4))
+    return GPTQ_ERR_ALIAS;
+  const DeviceInfo* dev = nullptr;
+  st = query_device(&dev);
+  if (st != GPTQ_OK) return st;
+  const cudaError_t e = launch_decode_gidx(x, qweight, scales, g_idx, y, M, K, N, n_groups,
+                                           static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  return GPTQ_OK;
+}
+
 int gptq_w4a16_gemm_asym(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                          const int32_t* qzeros, int64_t M, int64_t K, int64_t N, int32_t group,
                          uint16_t* y, void* stream) {
@@ -372,6 +400,7 @@ const char* gptq_status_string(int status) {
     case GPTQ_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
     case GPTQ_ERR_ALIAS: return "output overlaps an input";
     case GPTQ_ERR_KERNEL: return "kernel id or split count not valid for this call";
+    case GPTQ_ERR_INDEX: return "a g_idx entry outside 0 .. n_groups - 1";
     default: return "unknown status";
   }
 }

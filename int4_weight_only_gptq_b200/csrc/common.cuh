@@ -67,6 +67,16 @@ __device__ __forceinline__ void dequant_word_paired(uint32_t w, uint32_t s2, uin
   for (int j = 0; j < 4; ++j) p[j] = hmul2_rn(p[j], s2);
 }
 
+// Dequantised weights of one word with a scale per pair (act-order weights,
+// whose k can each take a different group): s2[j] holds the scales of k_j
+// (low half) and k_{j+4} (high half).  One rounding per weight, as above.
+__device__ __forceinline__ void dequant_word_paired_per_pair(uint32_t w, const uint32_t s2[4],
+                                                             uint32_t p[4]) {
+  unpack_centered(w, p);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) p[j] = hmul2_rn(p[j], s2[j]);
+}
+
 // The same four half2 for a scale with |s| < 2^-4, with two FP16 operations
 // fewer.  Codes at bits 4..7 of each 16-bit half, masked out of the word, are
 // the FP16 subnormals q * 2^-20; one fused multiply-add with b2 = s * 2^20 and

@@ -130,6 +130,12 @@ struct DecodeShape {
   int stage_bytes;  // X + qweight + scales of one stage (1024-aligned)
   int stages;       // ring depth
   int smem_bytes;   // whole dynamic allocation
+  // act order: the resident scale tile and the token tiles of the grid
+  int n_groups = 0;
+  int tile_bytes = 0;
+  int tile_boxes = 0;
+  int tile_box_rows = 0;
+  int tok_tiles = 1;
 };
 
 inline int align1024(int v) { return (v + 1023) & ~1023; }
@@ -152,12 +158,32 @@ inline DecodeShape decode_shape(int group_shift, bool asym = false) {
   return d;
 }
 
+// Act order: the scale tile of every group in front of the ring, loaded as
+// the fewest boxes of at most 256 rows; each stage carries its BKS entries of
+// g_idx in place of scale rows.
+template <int BT, int PRS>
+inline DecodeShape decode_shape_gidx(int64_t n_groups) {
+  using G = TokGeo<BT, PRS>;
+  DecodeShape d;
+  d.scale_rows = 0;
+  d.n_groups = (int)n_groups;
+  d.tile_boxes = (int)((n_groups + 255) / 256);
+  d.tile_box_rows = (int)((n_groups + d.tile_boxes - 1) / d.tile_boxes);
+  d.tile_bytes = align1024(d.tile_boxes * d.tile_box_rows * S_ROW_BYTES);
+  d.stage_bytes = align1024(G::S_OFF + G::BKS * 4);
+  const int s = d.tile_bytes < kRingBudget ? (kRingBudget - d.tile_bytes) / d.stage_bytes : 0;
+  d.stages = s > kMaxStages ? kMaxStages : s;
+  d.smem_bytes = 1024 + d.tile_bytes + d.stages * d.stage_bytes + 256;
+  return d;
+}
+
 struct DecodeBars {
   uint64_t full[kMaxStages];   // stage landed (TMA transaction count)
   uint64_t empty[kMaxStages];  // stage read by every dequantisation warp and the MMAs
   uint64_t afull[A_SLOTS];     // A slot written (and X permuted) by every dequantisation thread
   uint64_t aempty[A_SLOTS];    // MMAs reading the A slot done
   uint64_t dfull;              // all MMAs done
+  uint64_t tile_full;          // act order: the CTA's scale tile landed
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -219,13 +245,22 @@ __device__ __forceinline__ void permute_x_chunk(uint8_t* p) {
 // swizzle), T's rows to the X area (two 64-rank atoms); one fill per stage
 // copies lora_b into the A slot in the paired k order (T is permuted like X),
 // and the MMAs add T . lora_b^T to the same accumulators.
-template <int WPS, int BT, int PRS_, bool ASYM>
+// GIDX (act order): every k has its own group g_idx[k].  The CTA's whole
+// scale tile [n_groups x 128 columns] is loaded once into shared memory in
+// front of the ring (tile_boxes boxes of tile_box_rows rows, tile_bytes in
+// all; s_map's box is that high); each stage carries its slice of g_idx (in
+// place of scale rows, through qz_map) and the dequantisation gathers one
+// scale per k from the tile.  Token tiles: blockIdx.z takes tokens
+// BT * blockIdx.z onwards (more than one tile only for act order).
+template <int WPS, int BT, int PRS_, bool ASYM, bool GIDX>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ LinearSet ls,
                   const __grid_constant__ CUtensorMap qz_map,
                   const __grid_constant__ CUtensorMap t_map,
                   const __grid_constant__ CUtensorMap b_map, int M, int K, int group_shift,
-                  int stages, int stage_bytes, int scale_rows, int x3d, int lora_rank, int* err) {
+                  int stages, int stage_bytes, int scale_rows, int x3d, int lora_rank,
+                  int n_groups, int tile_bytes, int tile_boxes, int tile_box_rows, int* err) {
+  static_assert(!(GIDX && ASYM), "act order with symmetric weights only");
   constexpr int X_ATOM_BYTES = TokGeo<BT, PRS_>::X_ATOM_BYTES;
   constexpr int X_STAGE_BYTES = TokGeo<BT, PRS_>::X_STAGE_BYTES;
   constexpr int QW_OFF = TokGeo<BT, PRS_>::QW_OFF;
@@ -240,7 +275,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   // 1024-byte aligned base, derived from the shared array itself so that the
   // compiler keeps the shared address space (plain LDS, no generic loads)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  DecodeBars* bar = reinterpret_cast<DecodeBars*>(smem + stages * stage_bytes);
+  // act order: the scale tile, then the ring (tile_bytes is a multiple of 1024)
+  uint8_t* ring = smem + (GIDX ? tile_bytes : 0);
+  DecodeBars* bar = reinterpret_cast<DecodeBars*>(ring + stages * stage_bytes);
   volatile int* abort_flag = &bar->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -252,6 +289,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint16_t* __restrict__ y = ls.y[li];
   const int N = ls.n[li];
   const int n0 = ((int)blockIdx.x - ls.blk0[li]) * BW;
+  const int tok0 = (int)blockIdx.z * BT;      // this CTA's first token
+  const int Mt = min(M - tok0, BT);           // its tokens (1 .. BT)
   const int NS = ((K >> 3) + PRS - 1) / PRS;  // stages over all of K
   const int splits = gridDim.y;
   const int st_begin = (int)((int64_t)blockIdx.y * NS / splits);
@@ -274,6 +313,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&bar->aempty[a], 1);
     }
     mbar_init(&bar->dfull, 1);
+    mbar_init(&bar->tile_full, 1);
     bar->abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -312,6 +352,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       int s = 0;
       uint32_t ph = 0;
       bool t_waited = false;
+      if constexpr (GIDX) {
+        // the scale tile of this CTA's columns: every group
+        mbar_arrive_expect_tx(&bar->tile_full,
+                              (uint32_t)(tile_boxes * tile_box_rows * S_ROW_BYTES));
+        for (int b = 0; b < tile_boxes; ++b)
+          tma_load_2d(smem + b * tile_box_rows * S_ROW_BYTES, s_map, n0, b * tile_box_rows,
+                      &bar->tile_full);
+      }
       for (int t = 0; t < n_tot; ++t) {
         if (!mbar_wait_bounded(&bar->empty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
           record_timeout(err, bar);
@@ -323,7 +371,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           record_timeout(err, bar);
           break;
         }
-        uint8_t* st = smem + s * stage_bytes;
+        uint8_t* st = ring + s * stage_bytes;
         if (t >= n_st) {
           // LoRA stage: ranks 128 l .. 128 l + 127, as two 64-rank halves
           // (a half wholly past the rank is neither loaded nor multiplied)
@@ -337,7 +385,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (uint32_t h = 0; h < halves; ++h) {
             tma_load_2d(st + QW_OFF + h * LORA_HALF_BYTES, &b_map, r0 + 64 * (int)h, n0,
                         &bar->full[s]);
-            tma_load_2d(st + h * X_ATOM_BYTES, &t_map, r0 + 64 * (int)h, 0, &bar->full[s]);
+            tma_load_2d(st + h * X_ATOM_BYTES, &t_map, r0 + 64 * (int)h, tok0, &bar->full[s]);
           }
           ++issued;
           if (++s == stages) {
@@ -349,16 +397,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int k0 = (st_begin + t) * BKS;
         mbar_arrive_expect_tx(&bar->full[s],
                               X_STAGE_BYTES + QW_STAGE_BYTES +
-                                  scale_rows * (S_ROW_BYTES + (ASYM ? Z_ROW_BYTES : 0)));
+                                  (GIDX ? BKS * 4
+                                        : scale_rows * (S_ROW_BYTES + (ASYM ? Z_ROW_BYTES : 0))));
         tma_load_2d(st + QW_OFF, qw_map, n0, k0 >> 3, &bar->full[s]);
-        tma_load_2d(st + S_OFF, s_map, n0, k0 >> gs, &bar->full[s]);
-        if (ASYM) tma_load_2d(st + z_off, &qz_map, n0 / 8, k0 >> gs, &bar->full[s]);
+        if constexpr (GIDX) {
+          // g_idx[k0 .. k0 + BKS) as [BKS / 16 rows x 16]
+          tma_load_2d(st + S_OFF, &qz_map, 0, k0 >> 4, &bar->full[s]);
+        } else {
+          tma_load_2d(st + S_OFF, s_map, n0, k0 >> gs, &bar->full[s]);
+          if (ASYM) tma_load_2d(st + z_off, &qz_map, n0 / 8, k0 >> gs, &bar->full[s]);
+        }
         if (x3d) {
-          tma_load_3d(st, &x_map, 0, 0, k0 >> 6, &bar->full[s]);
+          tma_load_3d(st, &x_map, 0, tok0, k0 >> 6, &bar->full[s]);
         } else {
 #pragma unroll 1
           for (int a = 0; a < X_ATOMS; ++a)
-            tma_load_2d(st + a * X_ATOM_BYTES, &x_map, k0 + 64 * a, 0, &bar->full[s]);
+            tma_load_2d(st + a * X_ATOM_BYTES, &x_map, k0 + 64 * a, tok0, &bar->full[s]);
         }
         ++issued;
         if (++s == stages) {
@@ -372,6 +426,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int j = issued - 1; j >= 0 && j >= issued - stages; --j)
           mbar_wait_bounded(&bar->full[j % stages], (uint32_t)(j / stages) & 1u, &never,
                             kDrainLimitNs);
+        if (GIDX) mbar_wait_bounded(&bar->tile_full, 0u, &never, kDrainLimitNs);
       }
       // a CTA with adapter stages completes only after the launch computing T
       // (so this grid's completion implies T's, also when it gave up early)
@@ -391,7 +446,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t ph = 0, aph = 0;
     for (int t = 0; t < n_tot && ok; ++t) {
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar->full[s], ph, abort_flag, kWaitLimitNs));
-      const uint64_t x_desc = smem_desc_sw128(smem_u32(smem + s * stage_bytes));
+      const uint64_t x_desc = smem_desc_sw128(smem_u32(ring + s * stage_bytes));
+      if constexpr (GIDX) {
+        // every group index of the stage in range (the dequantisation clamps
+        // them, so a bad one reads inside the tile; it is reported here)
+        if (ok) {
+          const uint32_t* gi = reinterpret_cast<const uint32_t*>(ring + s * stage_bytes + S_OFF);
+          bool bad = false;
+#pragma unroll 4
+          for (int i = lane; i < BKS; i += 32) bad |= gi[i] >= (uint32_t)n_groups;
+          if (__any_sync(0xffffffffu, bad) && lane == 0) atomicCAS(err, 0, kDeviceErrIndex);
+        }
+      }
       if (t >= n_st) {
         // LoRA stage: one fill, one k16 step per 16 ranks of the stage
         if (ok)
@@ -476,11 +542,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int n = n0 + col;
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
     const int gid = (dw % GROUP_WARPS) * 32 + lane;
-    const int x_chunks = M * (BKS / 8);  // 16-byte chunks of the real X rows of a stage
+    const int x_chunks = Mt * (BKS / 8);  // 16-byte chunks of the real X rows of a stage
     // warps that rewrite X rows (whole warps: x_chunks is a multiple of 32)
     const bool x_writer = (dw % GROUP_WARPS) * 32 < x_chunks;
 
     bool ok = true;
+    if constexpr (GIDX) {
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar->tile_full, 0u, abort_flag, kWaitLimitNs));
+      if (!ok && lane == 0) record_timeout(err, bar);
+    }
+    // this thread's column of the scale tile (act order)
+    const uint8_t* tile_col = smem + col * 2;
+    const uint32_t g_max = (uint32_t)n_groups - 1u;
     // ring slot and phase of stage t, advanced incrementally (GROUPS <= stages)
     int s = grp % stages;
     uint32_t ph = (uint32_t)(grp / stages) & 1u;
@@ -491,7 +564,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar->full[s], ph, abort_flag, kWaitLimitNs));
       if (!ok) break;
-      uint8_t* st = smem + s * stage_bytes;
+      uint8_t* st = ring + s * stage_bytes;
       // chunk j: token row j / CPR, 64-k atom (j % CPR) / 8, chunk (j % 8) of
       // the 128-byte row, CPR = BKS / 8 chunks per row (every chunk of the
       // row is permuted, so the swizzle does not matter); rows >= M are zero
@@ -560,7 +633,23 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint8_t* sc = st + S_OFF + col * 2;
           uint32_t cells[4 * WPT];
           uint32_t s2 = 0, zlo = 0, zhi = 0;
-          if constexpr (!ASYM && WPS >= 4) {
+          if constexpr (GIDX) {
+            // act order: the group of each k from the stage's g_idx slice,
+            // its scale from the tile (indices clamped into the tile)
+            const uint32_t* gi = reinterpret_cast<const uint32_t*>(st + S_OFF) + 8 * row0;
+#pragma unroll
+            for (int i = 0; i < WPT; ++i) {
+              const uint4 ga = *reinterpret_cast<const uint4*>(gi + 8 * i);
+              const uint4 gb = *reinterpret_cast<const uint4*>(gi + 8 * i + 4);
+              const uint32_t w = *reinterpret_cast<const uint32_t*>(qw + i * (BW * 4));
+              auto sc = [&](uint32_t g) -> uint32_t {
+                return *reinterpret_cast<const uint16_t*>(tile_col + min(g, g_max) * S_ROW_BYTES);
+              };
+              const uint32_t sp[4] = {sc(ga.x) | (sc(gb.x) << 16), sc(ga.y) | (sc(gb.y) << 16),
+                                      sc(ga.z) | (sc(gb.z) << 16), sc(ga.w) | (sc(gb.w) << 16)};
+              dequant_word_paired_per_pair(w, sp, cells + 4 * i);
+            }
+          } else if constexpr (!ASYM && WPS >= 4) {
             // symmetric weights, a scale per four or more words: the
             // six-operation form where the scale allows it (same values)
 #pragma unroll
@@ -639,7 +728,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (h == 0) {
       // the four warps of slice 0 hold the four lane quarters: column `col`,
       // tokens in blocks of 16; an empty K range contributes zero
-      float* part = reinterpret_cast<float*>(smem);  // [token][column], splits > 1
+      float* part = reinterpret_cast<float*>(ring);  // [token][column], splits > 1
       if (ok && n_st > 0) tc_fence_after();
 #pragma unroll 1
       for (int tb = 0; tb < BT / 16; ++tb) {
@@ -665,8 +754,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (ok && n < N) {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (16 * tb + j < M)
-                y[(int64_t)(16 * tb + j) * N + n] = __half_as_ushort(__float2half_rn(r[j]));
+              if (16 * tb + j < Mt)
+                y[(int64_t)(tok0 + 16 * tb + j) * N + n] =
+                    __half_as_ushort(__float2half_rn(r[j]));
           }
         } else {
           // partial tile in the (fully consumed) ring
@@ -684,15 +774,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     // fixed-order reduction over the cluster's CTAs (consecutive K ranges)
     cluster_sync_all();
     const int rank = (int)cluster_ctarank();
-    const int E = M * BW;
+    const int E = Mt * BW;
     const int begin = rank * E / splits, end = (rank + 1) * E / splits;
-    const uint32_t base = smem_u32(smem);
+    const uint32_t base = smem_u32(ring);
     for (int idx = begin + (int)threadIdx.x; idx < end; idx += THREADS) {
       const int tok = idx / BW, c = idx - tok * BW;
       if (n0 + c >= N) continue;
       float sum = 0.f;
       for (int r = 0; r < splits; ++r) sum += ld_dsmem_f32(map_to_rank(base + 4u * idx, r));
-      y[(int64_t)tok * N + n0 + c] = __half_as_ushort(__float2half_rn(sum));
+      y[(int64_t)(tok0 + tok) * N + n0 + c] = __half_as_ushort(__float2half_rn(sum));
     }
     cluster_sync_all();
   }
@@ -702,7 +792,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int WPS, int BT, int PRS, bool ASYM>
+template <int WPS, int BT, int PRS, bool ASYM, bool GIDX>
 cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtensorMap& qz_map,
                      const CUtensorMap& t_map, const CUtensorMap& b_map, int lora_rank, int M,
                      int K, int group_shift, int splits, int x3d, const DecodeShape& d,
@@ -711,13 +801,13 @@ cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtens
   static cudaError_t attr_err[64];
   const int di = dev.device & 63;
   std::call_once(once[di], [&] {
-    attr_err[di] = cudaFuncSetAttribute(decode_kernel<WPS, BT, PRS, ASYM>,
+    attr_err[di] = cudaFuncSetAttribute(decode_kernel<WPS, BT, PRS, ASYM, GIDX>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         1024 + kRingBudget + 256);
   });
   if (attr_err[di] != cudaSuccess) return attr_err[di];
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)ls.blk0[ls.count], (unsigned)splits, 1);
+  cfg.gridDim = dim3((unsigned)ls.blk0[ls.count], (unsigned)splits, (unsigned)d.tok_tiles);
   cfg.blockDim = dim3(THREADS, 1, 1);
   cfg.dynamicSmemBytes = (size_t)d.smem_bytes;
   cfg.stream = stream;
@@ -735,9 +825,10 @@ cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtens
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT, PRS, ASYM>, x_map, ls, qz_map, t_map, b_map,
-                            M, K, group_shift, d.stages, d.stage_bytes, d.scale_rows, x3d,
-                            lora_rank, dev.error_word);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT, PRS, ASYM, GIDX>, x_map, ls, qz_map,
+                            t_map, b_map, M, K, group_shift, d.stages, d.stage_bytes,
+                            d.scale_rows, x3d, lora_rank, d.n_groups, d.tile_bytes, d.tile_boxes,
+                            d.tile_box_rows, dev.error_word);
 }
 
 // One linear of a launch, as the host sees it.
@@ -758,6 +849,23 @@ struct LinearExtras {
   const uint16_t* lora_b = nullptr;
   int64_t rank = 0;
 };
+
+// X as [K/64 atoms][M tokens][64 k] (one box per stage) when K is a multiple
+// of 64, else as [M][K] in one box per 64-k atom; rows at or beyond M and k at
+// or beyond K read as zero either way.  x3d: which of the two.
+template <int BT, int PRS>
+bool x_tensor_map(const uint16_t* x, int64_t M, int64_t K, CUtensorMap* x_map, int* x3d) {
+  *x3d = 0;
+  if (K % 64 == 0) {
+    const uint64_t dims[3] = {64, (uint64_t)M, (uint64_t)(K / 64)};
+    const uint64_t strides[2] = {(uint64_t)K * 2, 128};
+    const uint32_t box[3] = {64, BT, TokGeo<BT, PRS>::X_ATOMS};
+    *x3d = tensor_map_3d(x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, dims, strides, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ? 1 : 0;
+  }
+  return *x3d || tensor_map_2d(x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K,
+                               (uint64_t)M, (uint64_t)K * 2, 64, BT, CU_TENSOR_MAP_SWIZZLE_128B);
+}
 
 template <int BT, int PRS>
 cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count,
@@ -794,21 +902,9 @@ cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count,
     ls.n[i] = 0;
     ls.blk0[i + 1] = ls.blk0[count];
   }
-  // X as [K/64 atoms][M tokens][64 k] (one box per stage) when K is a
-  // multiple of 64, else as [M][K] in one box per 64-k atom; rows at or beyond
-  // M and k at or beyond K read as zero either way
   CUtensorMap x_map;
   int x3d = 0;
-  if (K % 64 == 0) {
-    const uint64_t dims[3] = {64, (uint64_t)M, (uint64_t)(K / 64)};
-    const uint64_t strides[2] = {(uint64_t)K * 2, 128};
-    const uint32_t box[3] = {64, BT, TokGeo<BT, PRS>::X_ATOMS};
-    x3d = tensor_map_3d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, dims, strides, box,
-                        CU_TENSOR_MAP_SWIZZLE_128B) ? 1 : 0;
-  }
-  if (!x3d && !tensor_map_2d(&x_map, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K,
-                             (uint64_t)M, (uint64_t)K * 2, 64, BT, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
+  if (!x_tensor_map<BT, PRS>(x, M, K, &x_map, &x3d)) return cudaErrorInvalidValue;
   CUtensorMap qz_map = ls.qw[0];  // read only for asymmetric weights
   if (asym) {
     const uint64_t N = (uint64_t)lin[0].n;
@@ -839,21 +935,21 @@ cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count,
   const int iM = (int)M, iK = (int)K;
   if (asym) {
     if (group_shift == 4)
-      return launch_t<2, BT, PRS, true>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
+      return launch_t<2, BT, PRS, true, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
                                    group_shift, splits, x3d, d, stream, dev);
     if (group_shift == 5)
-      return launch_t<4, BT, PRS, true>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
+      return launch_t<4, BT, PRS, true, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
                                    group_shift, splits, x3d, d, stream, dev);
-    return launch_t<WPT, BT, PRS, true>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
+    return launch_t<WPT, BT, PRS, true, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
                                    group_shift, splits, x3d, d, stream, dev);
   }
   if (group_shift == 4)
-    return launch_t<2, BT, PRS, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
+    return launch_t<2, BT, PRS, false, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
                                   splits, x3d, d, stream, dev);
   if (group_shift == 5)
-    return launch_t<4, BT, PRS, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
+    return launch_t<4, BT, PRS, false, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
                                   splits, x3d, d, stream, dev);
-  return launch_t<WPT, BT, PRS, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
+  return launch_t<WPT, BT, PRS, false, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
                                   splits, x3d, d, stream, dev);
 }
 
@@ -873,6 +969,51 @@ cudaError_t launch_set(const uint16_t* x, const LinearArgs* lin, int count,
   if (ex.rank > 0) return cudaErrorInvalidValue;  // adapters: up to 32 tokens
   if (M <= 48) return launch_bt<48, PRA>(x, lin, count, ex, M, K, group_shift, splits, stream, dev);
   return launch_bt<64, PRA>(x, lin, count, ex, M, K, group_shift, splits, stream, dev);
+}
+
+// Act order on a token tile of BT: false if the scale tile leaves no room
+// for two ring stages.
+template <int BT, int PRS>
+bool gidx_fits(int64_t n_groups) {
+  return decode_shape_gidx<BT, PRS>(n_groups).stages >= GROUPS;
+}
+
+template <int BT, int PRS>
+cudaError_t launch_gidx_bt(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                           const int32_t* g_idx, uint16_t* y, int64_t M, int64_t K, int64_t N,
+                           int64_t n_groups, cudaStream_t stream, const DeviceInfo& dev) {
+  DecodeShape d = decode_shape_gidx<BT, PRS>(n_groups);
+  if (d.stages < GROUPS) return cudaErrorInvalidValue;
+  d.tok_tiles = (int)((M + BT - 1) / BT);
+  LinearSet ls;
+  ls.count = 1;
+  ls.blk0[0] = 0;
+  if (!tensor_map_2d(&ls.qw[0], qweight, CU_TENSOR_MAP_DATA_TYPE_INT32, (uint64_t)N,
+                     (uint64_t)(K / 8), (uint64_t)N * 4, BW, PRS, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !tensor_map_2d(&ls.sc[0], scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, (uint64_t)N,
+                     (uint64_t)n_groups, (uint64_t)N * 2, BW, (uint32_t)d.tile_box_rows,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  ls.y[0] = y;
+  ls.n[0] = (int)N;
+  ls.blk0[1] = (int)((N + BW - 1) / BW);
+  for (int i = 1; i < kMaxLinears; ++i) {
+    ls.qw[i] = ls.qw[0];
+    ls.sc[i] = ls.sc[0];
+    ls.y[i] = nullptr;
+    ls.n[i] = 0;
+    ls.blk0[i + 1] = ls.blk0[1];
+  }
+  CUtensorMap x_map, gi_map;
+  int x3d = 0;
+  if (!x_tensor_map<BT, PRS>(x, M, K, &x_map, &x3d)) return cudaErrorInvalidValue;
+  // g_idx [K] as [K / 16 rows x 16]: one box of a stage's BKS entries
+  if (!tensor_map_2d(&gi_map, g_idx, CU_TENSOR_MAP_DATA_TYPE_INT32, 16, (uint64_t)(K / 16), 64,
+                     16, TokGeo<BT, PRS>::BKS / 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  const int splits = decode_pick_splits_blocks((int64_t)ls.blk0[1] * d.tok_tiles, K, PRS, dev);
+  return launch_t<WPT, BT, PRS, false, true>(x_map, ls, gi_map, x_map, x_map, 0, (int)M, (int)K,
+                                             62, splits, x3d, d, stream, dev);
 }
 
 }  // namespace
@@ -948,6 +1089,30 @@ cudaError_t launch_decode_lora(const uint16_t* x, const int32_t* qweight, const 
   ex.lora_b = lora_b;
   ex.rank = rank;
   return launch_set(x, &one, 1, ex, M, K, group_shift, 0, stream, dev);
+}
+
+cudaError_t launch_decode_gidx(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                               const int32_t* g_idx, uint16_t* y, int64_t M, int64_t K,
+                               int64_t N, int64_t n_groups, cudaStream_t stream,
+                               const DeviceInfo& dev) {
+  // Token tile as for plain weights (64 at most; more tokens take several
+  // tiles along the grid's z), and the stage size of the plain layer where
+  // the scale tile leaves room for it, so that consecutive group indices give
+  // the plain layer's result bit for bit.  Otherwise 256-k stages, else a
+  // smaller token tile.
+  const int64_t nblk = (N + BW - 1) / BW;
+  const int64_t mt = M < 64 ? M : 64;
+  const bool wide = decode_stage_rows(mt, nblk, K, 0, false, dev) == 2 * PRA;
+  const auto args = [&](auto launch) {
+    return launch(x, qweight, scales, g_idx, y, M, K, N, n_groups, stream, dev);
+  };
+  if (mt <= 16 && wide && gidx_fits<16, 2 * PRA>(n_groups))
+    return args(launch_gidx_bt<16, 2 * PRA>);
+  if (mt > 48 && gidx_fits<64, PRA>(n_groups)) return args(launch_gidx_bt<64, PRA>);
+  if (mt > 32 && gidx_fits<48, PRA>(n_groups)) return args(launch_gidx_bt<48, PRA>);
+  if (mt > 16 && gidx_fits<32, PRA>(n_groups)) return args(launch_gidx_bt<32, PRA>);
+  if (gidx_fits<16, PRA>(n_groups)) return args(launch_gidx_bt<16, PRA>);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode_grouped(const uint16_t* x, const int32_t* const* qweights,

@@ -19,6 +19,7 @@ struct DeviceInfo {
 
 // Error codes written to the device error word (match gptq_status values).
 constexpr int kDeviceErrTimeout = 7;
+constexpr int kDeviceErrIndex = 10;  // a g_idx entry outside 0 .. n_groups - 1
 
 // log2(group), or 62 for group == -1 (then (8*i) >> 62 == 0 for every row).
 inline int group_shift_of(int32_t group) {
@@ -58,6 +59,12 @@ cudaError_t launch_decode_lora(const uint16_t* x, const int32_t* qweight, const 
                                cudaStream_t stream, const DeviceInfo& dev);
 // Decode of `count` linears that share X (1..GPTQ_MAX_GROUPED), one launch;
 // the split is picked from the total number of column blocks.
+// Act order: W[k,n] = fp16((q[k,n] - 8) * scales[g_idx[k], n]), g_idx [K]
+// int32, scales [n_groups, N]; any M (tiles of at most 64 tokens).
+cudaError_t launch_decode_gidx(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                               const int32_t* g_idx, uint16_t* y, int64_t M, int64_t K,
+                               int64_t N, int64_t n_groups, cudaStream_t stream,
+                               const DeviceInfo& dev);
 cudaError_t launch_decode_grouped(const uint16_t* x, const int32_t* const* qweights,
                                   const uint16_t* const* scales, const int64_t* ns,
                                   uint16_t* const* ys, int count, int64_t M, int64_t K,

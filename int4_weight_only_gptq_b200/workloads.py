@@ -138,6 +138,29 @@ def make_qzeros(n_groups: int, N: int, *, seed: int = 0) -> np.ndarray:
     return words.view(np.int32)
 
 
+def make_gidx(K: int, group: int, *, seed: int = 0, kind: str = "perm") -> np.ndarray:
+    """Group index per input channel, int32 [K], for act-order weights.
+    kind "perm": GPTQ's act order, the channels taken in a seeded random
+    order and the i-th of that order put in group i // group (every group
+    holds `group` channels, the last the rest); "random": each channel in a
+    uniformly drawn group of the ceil(K / group) (group sizes unequal);
+    "consecutive": k // group (the plain layer).  Own stream: PCG64 seeded
+    with (seed, 3)."""
+    rng = np.random.Generator(np.random.PCG64([seed, 3]))
+    ng = num_groups(K, group)
+    G = K if group == -1 or group >= K else group
+    if kind == "consecutive":
+        return (np.arange(K) // G).astype(np.int32)
+    if kind == "perm":
+        order = rng.permutation(K)
+        g = np.empty(K, dtype=np.int32)
+        g[order] = np.arange(K) // G
+        return g
+    if kind == "random":
+        return rng.integers(0, ng, size=K).astype(np.int32)
+    raise ValueError(kind)
+
+
 # The five synthetic workloads, restated from their prose descriptions.
 def tiny(M: int = 1, seed: int = 0) -> Problem:
     """W4A16 GEMM, M in {1, 4}, K=512, N=256, group=128, scales U[1e-3, 2e-2]."""

@@ -38,8 +38,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_version_and_status_strings(lib):
     assert binding.version() == "0.1.0"
-    for st in range(10):
-        assert binding.status_string(st)
+    for st in range(11):
+        assert binding.status_string(st) != "unknown status"
     assert binding.status_string(12345) == "unknown status"
 
 
@@ -229,6 +229,37 @@ def test_asym_empty_m_and_no_device(lib):
         assert call_asym(lib) == 5
 
 
+# ---- gptq_w4a16_gemm_gidx: host-side checks ----------------------------------
+# Fake g_idx [512] (2 KB) for K=512, N=256 and four groups.
+
+GI = 0x2800000
+
+
+def call_gidx(lib, x=X, qw=QW, s=S, gi=GI, M=4, K=512, N=256, ng=4, y=Y):
+    v = ctypes.c_void_p
+    return lib.gptq_w4a16_gemm_gidx(v(x), v(qw), v(s), v(gi), M, K, N, ng, v(y), None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(M=-1), 2), (dict(K=520), 2), (dict(N=252), 2), (dict(K=65536 + 16), 2),
+    (dict(ng=0), 2), (dict(ng=-1), 2), (dict(ng=641), 2),
+    (dict(gi=0), 1), (dict(qw=0), 1), (dict(s=0), 1), (dict(x=0), 1), (dict(y=0), 1),
+    (dict(gi=GI + 4), 4), (dict(x=X + 2), 4), (dict(y=Y + 2), 4),
+    (dict(y=GI), 8), (dict(y=X), 8), (dict(y=S + 32), 8), (dict(y=QW), 8),
+])
+def test_gidx_argument_checks(lib, kw, status):
+    assert call_gidx(lib, **kw) == status
+
+
+def test_gidx_empty_m_and_no_device(lib):
+    import torch
+    assert call_gidx(lib, M=0, x=0, y=0) == 0
+    assert call_gidx(lib, M=0, x=0, y=0, gi=0) == 1
+    assert call_gidx(lib, M=0, x=0, y=0, ng=640) == 0
+    if not torch.cuda.is_available():
+        assert call_gidx(lib) == 5
+
+
 # ---- binding: shape checks before the library is called ----------------------
 # The C ABI sees pointers and the sizes it is given; a tensor smaller than those
 # sizes would be read or written past its end, so the binding checks shapes.
@@ -276,3 +307,16 @@ def test_adapter_shapes_accept_and_reject():
                  (_t(32 * 512), _t(256, 32))):   # lora_a not 2-D
         with pytest.raises(ValueError):
             binding.adapter_shapes(a, b, 512, 256)
+
+
+def test_gidx_shapes_accept_and_reject():
+    import torch
+    x, qw = _t(4, 512), _t(64, 256, dtype=torch.int32)
+    gi = _t(512, dtype=torch.int32)
+    assert binding.gidx_shapes(x, qw, _t(7, 256), gi) == (4, 512, 256, 7)
+    for s, g in ((_t(7, 248), gi),                             # scales columns != N
+                 (_t(7, 256), _t(520, dtype=torch.int32)),     # g_idx length != K
+                 (_t(7, 256), _t(1, 512, dtype=torch.int32)),  # g_idx not 1-D
+                 (_t(7 * 256), gi)):                           # scales not 2-D
+        with pytest.raises(ValueError):
+            binding.gidx_shapes(x, qw, s, g)

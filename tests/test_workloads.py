@@ -54,3 +54,19 @@ def test_algorithmic_bytes():
     p = W.decode_up()
     assert p.algorithmic_bytes == 46_002_176
     assert W.prefill(512).flops == 2 * 512 * 5120 * 17408
+
+
+def test_gidx_generator():
+    # consecutive indices are the plain layer's groups
+    assert np.array_equal(W.make_gidx(40, 16, kind="consecutive"), np.arange(40) // 16)
+    # act order: every group holds exactly `group` channels (the last the rest)
+    g = W.make_gidx(528, 128, seed=5, kind="perm")
+    assert g.dtype == np.int32 and g.shape == (528,)
+    assert np.bincount(g).tolist() == [128, 128, 128, 128, 16]
+    assert not np.array_equal(g, np.arange(528) // 128)
+    # random: indices in range, seeded
+    r = W.make_gidx(1040, 32, seed=1, kind="random")
+    assert r.min() >= 0 and r.max() < 33
+    assert np.array_equal(r, W.make_gidx(1040, 32, seed=1, kind="random"))
+    # one group (group -1): every index 0
+    assert not W.make_gidx(64, -1, kind="perm").any()
