@@ -184,6 +184,8 @@ struct DecodeBars {
   uint64_t aempty[A_SLOTS];    // MMAs reading the A slot done
   uint64_t dfull;              // all MMAs done
   uint64_t tile_full;          // act order: the CTA's scale tile landed
+  uint64_t dblk[2];            // persistent: MMAs of a column block done (set j % 2)
+  uint64_t dempty[2];          // persistent: accumulator set read out
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -252,7 +254,12 @@ __device__ __forceinline__ void permute_x_chunk(uint8_t* p) {
 // place of scale rows, through qz_map) and the dequantisation gathers one
 // scale per k from the tile.  Token tiles: blockIdx.z takes tokens
 // BT * blockIdx.z onwards (more than one tile only for act order).
-template <int WPS, int BT, int PRS_, bool ASYM, bool GIDX>
+// PERSIST (16-token tile, no split, plain weights): a grid smaller than the
+// column blocks; CTA c takes blocks c, c + gridDim.x, ... one after another
+// through the same ring, its MMAs alternating between two accumulator sets so
+// that block j is read out (by the four slice-0 warps of group 0, between
+// their stages) while block j + 1 streams.
+template <int WPS, int BT, int PRS_, bool ASYM, bool GIDX, bool PERSIST>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ LinearSet ls,
                   const __grid_constant__ CUtensorMap qz_map,
@@ -261,6 +268,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                   int stages, int stage_bytes, int scale_rows, int x3d, int lora_rank,
                   int n_groups, int tile_bytes, int tile_boxes, int tile_box_rows, int* err) {
   static_assert(!(GIDX && ASYM), "act order with symmetric weights only");
+  static_assert(!PERSIST || (!ASYM && !GIDX && 2 * TokGeo<BT, PRS_>::NACC * BT <= A_COL0),
+                "persistent: plain weights, two accumulator sets below the A slots");
   constexpr int X_ATOM_BYTES = TokGeo<BT, PRS_>::X_ATOM_BYTES;
   constexpr int X_STAGE_BYTES = TokGeo<BT, PRS_>::X_STAGE_BYTES;
   constexpr int QW_OFF = TokGeo<BT, PRS_>::QW_OFF;
@@ -299,7 +308,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   // LoRA stages of this CTA (the last of the column block's split), then all
   const int n_lora = (TokGeo<BT, PRS_>::LORA_OK && lora_rank > 0 && (int)blockIdx.y == splits - 1)
                          ? (lora_rank + 127) / 128 : 0;
-  const int n_tot = n_st + n_lora;
+  // persistent: this CTA's column blocks (PERSIST launches have no split and
+  // no adapter, so each block is n_st stages)
+  const int n_blk = PERSIST ? (ls.blk0[ls.count] - (int)blockIdx.x + (int)gridDim.x - 1) /
+                                  (int)gridDim.x
+                            : 1;
+  const int n_tot = PERSIST ? n_blk * n_st : n_st + n_lora;
   const int gs = min(group_shift, 30);        // group -1 (shift 62): row 0 throughout
   const int z_off = S_OFF + scale_rows * S_ROW_BYTES;  // zero-point rows (ASYM)
 
@@ -314,6 +328,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(&bar->dfull, 1);
     mbar_init(&bar->tile_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar->dblk[i], 1);
+      mbar_init(&bar->dempty[i], 4);  // the four read-out warps
+    }
     bar->abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -372,7 +390,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         uint8_t* st = ring + s * stage_bytes;
-        if (t >= n_st) {
+        if (!PERSIST && t >= n_st) {
           // LoRA stage: ranks 128 l .. 128 l + 127, as two 64-rank halves
           // (a half wholly past the rank is neither loaded nor multiplied)
           if (t == n_st) {
@@ -394,17 +412,29 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           continue;
         }
-        const int k0 = (st_begin + t) * BKS;
+        const int ts = PERSIST ? t % n_st : t;  // stage within the column block
+        const CUtensorMap* qwm = qw_map;
+        const CUtensorMap* scm = s_map;
+        int nb0 = n0;
+        if constexpr (PERSIST) {
+          const int b = (int)blockIdx.x + (t / n_st) * (int)gridDim.x;
+          int l = 0;
+          while (l + 1 < ls.count && b >= ls.blk0[l + 1]) ++l;
+          qwm = &ls.qw[l];
+          scm = &ls.sc[l];
+          nb0 = (b - ls.blk0[l]) * BW;
+        }
+        const int k0 = (st_begin + ts) * BKS;
         mbar_arrive_expect_tx(&bar->full[s],
                               X_STAGE_BYTES + QW_STAGE_BYTES +
                                   (GIDX ? BKS * 4
                                         : scale_rows * (S_ROW_BYTES + (ASYM ? Z_ROW_BYTES : 0))));
-        tma_load_2d(st + QW_OFF, qw_map, n0, k0 >> 3, &bar->full[s]);
+        tma_load_2d(st + QW_OFF, qwm, nb0, k0 >> 3, &bar->full[s]);
         if constexpr (GIDX) {
           // g_idx[k0 .. k0 + BKS) as [BKS / 16 rows x 16]
           tma_load_2d(st + S_OFF, &qz_map, 0, k0 >> 4, &bar->full[s]);
         } else {
-          tma_load_2d(st + S_OFF, s_map, n0, k0 >> gs, &bar->full[s]);
+          tma_load_2d(st + S_OFF, scm, nb0, k0 >> gs, &bar->full[s]);
           if (ASYM) tma_load_2d(st + z_off, &qz_map, n0 / 8, k0 >> gs, &bar->full[s]);
         }
         if (x3d) {
@@ -458,7 +488,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (__any_sync(0xffffffffu, bad) && lane == 0) atomicCAS(err, 0, kDeviceErrIndex);
         }
       }
-      if (t >= n_st) {
+      if (!PERSIST && t >= n_st) {
         // LoRA stage: one fill, one k16 step per 16 ranks of the stage
         if (ok)
           ok = __all_sync(0xffffffffu,
@@ -486,6 +516,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         continue;
       }
+      // persistent: column block j of this CTA, stage ts of it, and its
+      // accumulator set (free again once block j - 2 has been read out)
+      const int j = PERSIST ? t / n_st : 0;
+      const int ts = PERSIST ? t - j * n_st : t;
+      const uint32_t d_base = tmem + D_COL + (uint32_t)((j & 1) * NACC * BT);
+      if (PERSIST && ts == 0 && j >= 2) {
+        if (ok)
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar->dempty[j & 1],
+                                                         (uint32_t)((j - 2) >> 1) & 1u,
+                                                         abort_flag, kWaitLimitNs));
+        if (!ok) break;
+        tc_fence_after();
+      }
 #pragma unroll
       for (int hf = 0; hf < HALVES; ++hf) {
         if (ok)
@@ -497,15 +540,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         // k16 step kk of this fill reads X atom 4*hf + kk/4 at byte (kk % 4) * 32
         // (the descriptor's address field counts 16 bytes)
         const uint64_t b_desc0 = x_desc + (uint64_t)((hf * 4 * X_ATOM_BYTES) >> 4);
-        const uint32_t first = (t == 0 && hf == 0) ? 0u : 1u;
+        const uint32_t first = (ts == 0 && hf == 0) ? 0u : 1u;
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < BKA / 16; ++kk)
-            mma_f16_ts(tmem + D_COL + (kk % NACC) * BT, a_base + 8 * kk,
+            mma_f16_ts(d_base + (kk % NACC) * BT, a_base + 8 * kk,
                        b_desc0 + (uint64_t)(((kk >> 2) * X_ATOM_BYTES + (kk & 3) * 32) >> 4),
                        idesc, kk >= NACC ? 1u : first);
           mma_commit(&bar->aempty[a]);
           if (hf == HALVES - 1) mma_commit(&bar->empty[s]);
+          if (PERSIST && hf == HALVES - 1 && ts == n_st - 1) mma_commit(&bar->dblk[j & 1]);
         }
         __syncwarp();
         if (++a == A_SLOTS) {
@@ -554,6 +598,47 @@ __global__ void __launch_bounds__(THREADS, 1)
     // this thread's column of the scale tile (act order)
     const uint8_t* tile_col = smem + col * 2;
     const uint32_t g_max = (uint32_t)n_groups - 1u;
+    // persistent: reads out column block jd (accumulator set jd % 2) and
+    // stores its columns of Y; false if the wait expired
+    int drained = 0;
+    auto drain = [&](int jd) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bar->dblk[jd & 1], (uint32_t)(jd >> 1) & 1u,
+                                                     abort_flag, kWaitLimitNs)))
+        return false;
+      tc_fence_after();
+      const int b = (int)blockIdx.x + jd * (int)gridDim.x;
+      int l = 0;
+      while (l + 1 < ls.count && b >= ls.blk0[l + 1]) ++l;
+      const int nl = ls.n[l];
+      const int nc = (b - ls.blk0[l]) * BW + col;
+      uint16_t* __restrict__ yl = ls.y[l];
+      const uint32_t d_set = D_COL + (uint32_t)((jd & 1) * NACC * BT);
+      float r[BT];
+#pragma unroll
+      for (int tb = 0; tb < BT / 16; ++tb) {
+        uint32_t v[NACC][16];
+#pragma unroll
+        for (int c = 0; c < NACC; ++c)
+          tmem_ld_32x32b_x16(tmem + lane_addr + d_set + c * BT + 16 * tb, v[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float acc = __uint_as_float(v[0][q]);
+#pragma unroll
+          for (int c = 1; c < NACC; ++c) acc += __uint_as_float(v[c][q]);
+          r[16 * tb + q] = acc;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->dempty[jd & 1]);  // the set may be overwritten
+      if (nc < nl) {
+#pragma unroll
+        for (int q = 0; q < BT; ++q)
+          if (q < Mt) yl[(int64_t)(tok0 + q) * nl + nc] = __half_as_ushort(__float2half_rn(r[q]));
+      }
+      return true;
+    };
     // ring slot and phase of stage t, advanced incrementally (GROUPS <= stages)
     int s = grp % stages;
     uint32_t ph = (uint32_t)(grp / stages) & 1u;
@@ -561,6 +646,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (s >= stages) {
         s -= stages;
         ph ^= 1u;
+      }
+      if (PERSIST && h == 0) {
+        // read out the finished blocks before this stage's block j; those
+        // up to j - 2 first of all (block j's MMAs wait for their set)
+        const int j = t / n_st;
+        while (ok && drained < j) {
+          if (drained > j - 2 &&
+              !__shfl_sync(0xffffffffu,
+                           (int)mbar_test_wait(smem_u32(&bar->dblk[drained & 1]),
+                                               (uint32_t)(drained >> 1) & 1u),
+                           0))
+            break;
+          ok = drain(drained);
+          ++drained;
+        }
+        if (!ok) break;
       }
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar->full[s], ph, abort_flag, kWaitLimitNs));
       if (!ok) break;
@@ -573,7 +674,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int j = gid; j < x_chunks; j += GROUP_WARPS * 32)
         permute_x_chunk(st + ((j % CPR) >> 3) * X_ATOM_BYTES + (j / CPR) * 128 + (j & 7) * 16);
 
-      if (t >= n_st) {
+      if (!PERSIST && t >= n_st) {
         // LoRA stage: one fill.  Row rho (eight ranks) of this slice's chunks
         // comes from lora_b row `col` in the swizzled qweight area and is
         // paired (k, k+4) like X and the dequantised weights.
@@ -719,13 +820,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_arrive(&bar->afull[a]);
       }
     }
+    // persistent: the blocks not read out yet
+    if (PERSIST && h == 0) {
+      while (ok && drained < n_blk) {
+        ok = drain(drained);
+        ++drained;
+      }
+    }
     if (!ok && lane == 0) record_timeout(err, bar);
 
     if (ok) {
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar->dfull, 0, abort_flag, kWaitLimitNs));
       if (!ok && lane == 0) record_timeout(err, bar);
     }
-    if (h == 0) {
+    if (!PERSIST && h == 0) {
       // the four warps of slice 0 hold the four lane quarters: column `col`,
       // tokens in blocks of 16; an empty K range contributes zero
       float* part = reinterpret_cast<float*>(ring);  // [token][column], splits > 1
@@ -792,7 +900,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int WPS, int BT, int PRS, bool ASYM, bool GIDX>
+template <int WPS, int BT, int PRS, bool ASYM, bool GIDX, bool PERSIST = false>
 cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtensorMap& qz_map,
                      const CUtensorMap& t_map, const CUtensorMap& b_map, int lora_rank, int M,
                      int K, int group_shift, int splits, int x3d, const DecodeShape& d,
@@ -801,13 +909,16 @@ cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtens
   static cudaError_t attr_err[64];
   const int di = dev.device & 63;
   std::call_once(once[di], [&] {
-    attr_err[di] = cudaFuncSetAttribute(decode_kernel<WPS, BT, PRS, ASYM, GIDX>,
+    attr_err[di] = cudaFuncSetAttribute(decode_kernel<WPS, BT, PRS, ASYM, GIDX, PERSIST>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         1024 + kRingBudget + 256);
   });
   if (attr_err[di] != cudaSuccess) return attr_err[di];
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)ls.blk0[ls.count], (unsigned)splits, (unsigned)d.tok_tiles);
+  // persistent: one CTA per SM, each walking several column blocks
+  const int blocks = ls.blk0[ls.count];
+  const int grid_x = PERSIST && blocks > dev.num_sms ? dev.num_sms : blocks;
+  cfg.gridDim = dim3((unsigned)grid_x, (unsigned)splits, (unsigned)d.tok_tiles);
   cfg.blockDim = dim3(THREADS, 1, 1);
   cfg.dynamicSmemBytes = (size_t)d.smem_bytes;
   cfg.stream = stream;
@@ -825,7 +936,7 @@ cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtens
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT, PRS, ASYM, GIDX>, x_map, ls, qz_map,
+  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT, PRS, ASYM, GIDX, PERSIST>, x_map, ls, qz_map,
                             t_map, b_map, M, K, group_shift, d.stages, d.stage_bytes,
                             d.scale_rows, x3d, lora_rank, d.n_groups, d.tile_bytes, d.tile_boxes,
                             d.tile_box_rows, dev.error_word);
@@ -933,24 +1044,39 @@ cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count,
     if (splits > ns) splits = ns;
   }
   const int iM = (int)M, iK = (int)K;
+  const int gsh = group_shift;
   if (asym) {
-    if (group_shift == 4)
-      return launch_t<2, BT, PRS, true, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
-                                   group_shift, splits, x3d, d, stream, dev);
-    if (group_shift == 5)
-      return launch_t<4, BT, PRS, true, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
-                                   group_shift, splits, x3d, d, stream, dev);
-    return launch_t<WPT, BT, PRS, true, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
-                                   group_shift, splits, x3d, d, stream, dev);
+    if (gsh == 4)
+      return launch_t<2, BT, PRS, true, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM,
+                                               iK, gsh, splits, x3d, d, stream, dev);
+    if (gsh == 5)
+      return launch_t<4, BT, PRS, true, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM,
+                                               iK, gsh, splits, x3d, d, stream, dev);
+    return launch_t<WPT, BT, PRS, true, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM,
+                                               iK, gsh, splits, x3d, d, stream, dev);
   }
-  if (group_shift == 4)
-    return launch_t<2, BT, PRS, false, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
-                                  splits, x3d, d, stream, dev);
-  if (group_shift == 5)
-    return launch_t<4, BT, PRS, false, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
-                                  splits, x3d, d, stream, dev);
-  return launch_t<WPT, BT, PRS, false, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK, group_shift,
-                                  splits, x3d, d, stream, dev);
+  // more column blocks than SMs (wide or grouped linears) at up to 16 tokens
+  // without a split: one persistent wave instead of several
+  if constexpr (BT == 16 && PRS == 2 * PRA) {
+    if (splits == 1 && lora_rank == 0 && ls.blk0[count] > dev.num_sms) {
+      if (gsh == 4)
+        return launch_t<2, BT, PRS, false, false, true>(x_map, ls, qz_map, t_map, b_map, 0, iM,
+                                                        iK, gsh, splits, x3d, d, stream, dev);
+      if (gsh == 5)
+        return launch_t<4, BT, PRS, false, false, true>(x_map, ls, qz_map, t_map, b_map, 0, iM,
+                                                        iK, gsh, splits, x3d, d, stream, dev);
+      return launch_t<WPT, BT, PRS, false, false, true>(x_map, ls, qz_map, t_map, b_map, 0, iM,
+                                                        iK, gsh, splits, x3d, d, stream, dev);
+    }
+  }
+  if (gsh == 4)
+    return launch_t<2, BT, PRS, false, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
+                                              gsh, splits, x3d, d, stream, dev);
+  if (gsh == 5)
+    return launch_t<4, BT, PRS, false, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
+                                              gsh, splits, x3d, d, stream, dev);
+  return launch_t<WPT, BT, PRS, false, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
+                                              gsh, splits, x3d, d, stream, dev);
 }
 
 cudaError_t launch_set(const uint16_t* x, const LinearArgs* lin, int count,

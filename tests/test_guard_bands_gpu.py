@@ -84,6 +84,7 @@ LAYER_CASES = [  # (label, M, K, N, G, kernel, splits)
     ("decode K split, ragged K", 16, 2064, 72, 32, B.KERNEL_AUTO, 3),
     ("decode 48-token tile", 41, 1040, 136, 32, B.KERNEL_AUTO, 0),
     ("decode 64-token tile, K split", 63, 2064, 264, 128, B.KERNEL_AUTO, 2),
+    ("decode persistent (more column blocks than SMs)", 7, 528, 20488, 64, B.KERNEL_AUTO, 0),
     ("forced single-CTA prefill", 20, 528, 136, 64, B.KERNEL_PREFILL, 0),
     ("pair prefill 128-token tile", 100, 528, 392, 128, B.KERNEL_AUTO, 0),
     ("pair prefill 256-token tile", 300, 1040, 264, -1, B.KERNEL_AUTO, 0),

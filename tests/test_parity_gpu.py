@@ -373,6 +373,42 @@ def run_grouped(ps):
     return [y.cpu().numpy() for y in ys]
 
 
+# More column blocks than SMs at up to 16 tokens: one persistent wave, each CTA
+# walking blocks c, c + 148, ... with two alternating accumulator sets.
+PERSISTENT = [  # (M, K, Ns, G)
+    (1, 512, (17408, 17408), 128),            # gate+up shape: 272 blocks, two per CTA
+    (16, 528, (20480,), 32),                  # one wide linear, 160 blocks, ragged K
+    (5, 1040, (40968,), 16),                  # 321 blocks (three for some CTAs), ragged N
+    (3, 2048, (17408,) * 8, 64),              # 1088 blocks: seven or eight per CTA
+    (9, 512, (8, 20480, 24, 136), -1),        # narrow and wide linears mixed, one group
+]
+
+
+@pytest.mark.parametrize("M,K,Ns,G", PERSISTENT)
+def test_persistent_decode_parity(M, K, Ns, G):
+    ps = grouped_problem(M, K, Ns, G, seed=M + K + len(Ns))
+    ys = run_grouped(ps)
+    for i, (p, y) in enumerate(zip(ps, ys)):
+        ref = oracle.gemm(p.x, p.qweight, p.scales, G)
+        err = rel_err(y, ref)
+        print(f"[parity] persistent M={M} K={K} linear {i} N={p.N} G={G}: {err:.3e}")
+        assert np.all(np.isfinite(y))
+        assert err <= TOL
+    assert B.device_error() == 0
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_persistent_gate_up_equals_separate_calls_bitwise(M):
+    # the same stages and accumulation order per column as one launch per linear
+    ps = grouped_problem(M, 5120, (17408, 17408), 128, seed=M)
+    ys = run_grouped(ps)
+    for p, y in zip(ps, ys):
+        assert np.array_equal(y.view(np.uint16), run(p).view(np.uint16))
+    rows = sorted({0, M - 1})
+    for p, y in zip(ps, ys):
+        check_rows(p, y, rows, f"persistent gate+up M={M}")
+
+
 @pytest.mark.parametrize("M,K,Ns,G", [
     (1, 2048, (264, 136, 8), 128), (5, 1040, (72, 200), 32), (16, 2560, (128, 128, 40, 8), 16),
     (32, 1536, (136, 264), -1), (33, 528, (64, 24), 128), (64, 2064, (136, 40, 8), 32),
