@@ -179,10 +179,18 @@ GPTQ_API int gptq_w4a16_gemm_asym(const uint16_t* x, const int32_t* qweight,
  *            own output); must not overlap any other argument
  * T is summed in FP32 and rounded to FP16; T . lora_b^T is added to the
  * layer's FP32 accumulator (the adapter's rank is extra K of the same
- * tensor-core product) and Y is rounded once.  Two launches on `stream`: T,
- * then the layer, which runs on the decode kernel up to
- * GPTQ_LORA_DECODE_MAX_M tokens and on the prefill kernel above and may start while T is computed (it
- * waits for T only before reading it).  Other arguments, checks
+ * tensor-core product) and Y is rounded once.  Up to GPTQ_LORA_DECODE_MAX_M
+ * tokens the layer runs on the decode kernel, and when its column blocks
+ * leave SMs free T is computed by CTAs of that same launch, on those SMs,
+ * and handed over through a counter in the library's static device memory
+ * (one of 1024 slots, taken in turn by successive calls on the device; the
+ * last reader clears it): one launch.  Otherwise two launches on `stream`: T,
+ * then the layer (decode kernel, or the prefill kernel above
+ * GPTQ_LORA_DECODE_MAX_M tokens), which may start while T is computed and
+ * waits for T only before reading it.  Calls that may run at the same time
+ * on different streams take different slots; a CUDA graph that holds such a
+ * call keeps its slot, so one graph must not be replayed on two streams at
+ * once.  Other arguments, checks
  * and errors as gptq_w4a16_gemm, plus GPTQ_ERR_NULL for a NULL lora_a, lora_b
  * or t_work (when M > 0), GPTQ_ERR_SHAPE for a rank out of range, and
  * GPTQ_ERR_ALIAS when t_work or y overlaps any other buffer.
@@ -266,9 +274,12 @@ GPTQ_API const char* gptq_status_string(int status);
 
 /*
  * Reads and clears the device-side error word of the current device: 0 when
- * no kernel gave up a bounded wait since the last call, else GPTQ_ERR_TIMEOUT.
- * Synchronises the current device.  Kernels never trap: a wait that exceeds
- * its bound records the error here, abandons the output tile and exits.
+ * no kernel gave up a bounded wait or met a bad index since the last call,
+ * else GPTQ_ERR_TIMEOUT or GPTQ_ERR_INDEX.  Synchronises the current device.
+ * Kernels never trap: a wait that exceeds its bound records the error here,
+ * abandons the output tile and exits.  After an error it also clears the
+ * library's adapter hand-over counters (static device memory), which a kernel
+ * that gave up may have left set.
  */
 GPTQ_API int gptq_device_error(void);
 

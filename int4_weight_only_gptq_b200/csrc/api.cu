@@ -22,6 +22,11 @@ __device__ int g_error_word;
 // library, one per device, shared by every such call on that device.
 __device__ __align__(256) uint16_t g_lora_scratch[GPTQ_LORA_SCRATCH_BYTES / 2];
 
+// Hand-over flags of adapters computed inside the layer's launch: slot
+// (call number % kTFlagSlots) counts the T CTAs done (low half) and the layer
+// CTAs past their wait (high half); the last of those clears it.
+__device__ unsigned long long g_t_flags[kTFlagSlots];
+
 constexpr int kMaxDevices = 64;
 std::once_flag g_dev_once[kMaxDevices];
 DeviceInfo g_dev[kMaxDevices];
@@ -65,6 +70,13 @@ int query_device(const DeviceInfo** out) {
       return;
     }
     info.lora_scratch = static_cast<uint16_t*>(q);
+    void* f = nullptr;
+    if (cudaGetSymbolAddress(&f, g_t_flags) != cudaSuccess) {
+      cudaGetLastError();
+      g_dev_status[d] = GPTQ_ERR_DEVICE;
+      return;
+    }
+    info.t_flags = static_cast<unsigned long long*>(f);
     g_dev[d] = info;
     g_dev_status[d] = GPTQ_OK;
   });
@@ -179,6 +191,18 @@ int lora_impl(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
   if (st != GPTQ_OK) return st;
   if (static_t) t_work = dev->lora_scratch;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // up to GPTQ_LORA_DECODE_MAX_M tokens, when the decode launch leaves SMs
+  // free: T on CTAs of the layer's own launch, handed over through a flag
+  if (M <= GPTQ_LORA_DECODE_MAX_M && decode_lora_fused_fits(M, K, N, rank, *dev)) {
+    const cudaError_t e = launch_decode_lora_fused(x, qweight, scales, y, M, K, N,
+                                                   group_shift_of(group), t_work, lora_a, lora_b,
+                                                   rank, s, *dev);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return GPTQ_ERR_CUDA;
+    }
+    return GPTQ_OK;
+  }
   // up to GPTQ_LORA_DECODE_MAX_M tokens the layer runs on the decode kernel,
   // one CTA per SM: the T launch may use the SMs it leaves free
   int free_sms = 0;
@@ -417,6 +441,12 @@ int gptq_device_error(void) {
   const int zero = 0;
   if (cudaMemcpy(&v, dev->error_word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
       cudaMemcpy(dev->error_word, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  // a kernel that gave up may have left an adapter hand-over slot uncleared
+  if (v != 0 && cudaMemset(dev->t_flags, 0, sizeof(unsigned long long) * kTFlagSlots) !=
+                    cudaSuccess) {
     cudaGetLastError();
     return GPTQ_ERR_CUDA;
   }

@@ -67,6 +67,24 @@ __device__ __forceinline__ void dequant_word_paired(uint32_t w, uint32_t s2, uin
   for (int j = 0; j < 4; ++j) p[j] = hmul2_rn(p[j], s2);
 }
 
+// sm += the FP32 dot product of eight FP16 x (one 16-byte chunk) with eight
+// weights already widened to four float2, in k order.
+__device__ __forceinline__ void fma8(float& sm, const uint4 xv, const float2 a0, const float2 a1,
+                                     const float2 a2, const float2 a3) {
+  const float2 x0 = __half22float2(*reinterpret_cast<const __half2*>(&xv.x));
+  const float2 x1 = __half22float2(*reinterpret_cast<const __half2*>(&xv.y));
+  const float2 x2 = __half22float2(*reinterpret_cast<const __half2*>(&xv.z));
+  const float2 x3 = __half22float2(*reinterpret_cast<const __half2*>(&xv.w));
+  sm = fmaf(x0.x, a0.x, sm);
+  sm = fmaf(x0.y, a0.y, sm);
+  sm = fmaf(x1.x, a1.x, sm);
+  sm = fmaf(x1.y, a1.y, sm);
+  sm = fmaf(x2.x, a2.x, sm);
+  sm = fmaf(x2.y, a2.y, sm);
+  sm = fmaf(x3.x, a3.x, sm);
+  sm = fmaf(x3.y, a3.y, sm);
+}
+
 // Dequantised weights of one word with a scale per pair (act-order weights,
 // whose k can each take a different group): s2[j] holds the scales of k_j
 // (low half) and k_{j+4} (high half).  One rounding per weight, as above.

@@ -59,6 +59,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -232,6 +234,120 @@ __device__ __forceinline__ void permute_x_chunk(uint8_t* p) {
   *reinterpret_cast<uint4*>(p) = o;
 }
 
+// The LoRA adapter's T computed by CTAs of the layer's own launch (the fused
+// form, up to 32 tokens): `ctas` CTAs appended to the grid's column blocks
+// (blockIdx.y == 0 of each computes; the others of its cluster only exit)
+// each compute T for a balanced share of the ranks over all of K, store it,
+// and add one to the low half of this call's hand-over slot.  Each of the
+// `consumers` CTAs that run adapter stages waits for that count to reach
+// `ctas` before its first read of T, then adds one to the high half; the last
+// of them clears the slot, so that the slot starts at zero for its next use
+// (the next call given it, or the same call replayed from a CUDA graph).
+// ctas == 0: T comes from the launch before this one.
+struct LoraFused {
+  const uint16_t* x;           // X [M, K]
+  const uint16_t* a;           // lora_a [rank, K]
+  uint16_t* t;                 // T [M, rank]
+  unsigned long long* flag;    // this call's slot
+  int ctas;
+  int consumers;
+  int rank;
+};
+
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Global-memory writes that this thread has observed (through an acquire)
+// become visible to its later TMA reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Waits until the low half of *flag reaches `count`; false after limit_ns or
+// once *abort is set.
+__device__ __forceinline__ bool flag_wait_bounded(const unsigned long long* flag, uint32_t count,
+                                                  volatile int* abort, uint64_t limit_ns) {
+  if ((uint32_t)ld_acquire_gpu_u64(flag) >= count) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if ((uint32_t)ld_acquire_gpu_u64(flag) >= count) return true;
+    if ((n & 63u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+  }
+}
+
+// One CTA of the fused form: T[m, j] = fp16(sum_k X[m, k] lora_a[j, k]) for
+// its ranks j (i-th of `ctas` balanced shares) and every token m < M <= MB.
+// The ranks take the CTA's warps in equal groups that split K (a warp per
+// rank, several ranks in turn, when there are more ranks than warps); lane l
+// takes 8-k chunk l of every 256-k piece of its warp's range.  FP32 sums in a
+// fixed order: the lanes by shuffles, then the rank's warps in order.
+template <int MB>
+__device__ void lora_t_cta(const LoraFused& lf, int M, int K, int i, float* part) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // X may come from the previous kernel
+  constexpr int NW = THREADS / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = (int)((int64_t)i * lf.rank / lf.ctas);
+  const int nr = (int)((int64_t)(i + 1) * lf.rank / lf.ctas) - r0;
+  const int wpr = nr > 0 && nr < NW ? NW / nr : 1;  // warps per rank
+  const int ws = warp % wpr;                        // this warp's slice of K
+  const int pieces = (K + 255) / 256;
+  const int pb = ws * pieces / wpr, pe = (ws + 1) * pieces / wpr;
+  for (int rr = warp / wpr; rr < nr; rr += NW / wpr) {
+    float acc[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) acc[m] = 0.f;
+    const uint16_t* __restrict__ arow = lf.a + (int64_t)(r0 + rr) * K;
+    for (int pc = pb; pc < pe; ++pc) {
+      const int k = pc * 256 + 8 * lane;
+      if (k < K) {  // K % 8 == 0: the chunk is whole
+        const uint4 av = __ldg(reinterpret_cast<const uint4*>(arow + k));
+        const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&av.x));
+        const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&av.y));
+        const float2 a2 = __half22float2(*reinterpret_cast<const __half2*>(&av.z));
+        const float2 a3 = __half22float2(*reinterpret_cast<const __half2*>(&av.w));
+#pragma unroll
+        for (int m0 = 0; m0 < MB; m0 += 8) {
+          if (m0 >= M) break;
+          uint4 xv[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            xv[q] = m0 + q < M
+                        ? __ldg(reinterpret_cast<const uint4*>(lf.x + (int64_t)(m0 + q) * K + k))
+                        : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) fma8(acc[m0 + q], xv[q], a0, a1, a2, a3);
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      float v = acc[m];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+      if (lane == 0) part[(rr * wpr + ws) * MB + m] = v;
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < nr * M; idx += THREADS) {
+    const int rr = idx / M, m = idx - rr * M;
+    float sum = 0.f;
+    for (int w = 0; w < wpr; ++w) sum += part[(rr * wpr + w) * MB + m];
+    lf.t[(int64_t)m * lf.rank + r0 + rr] = __half_as_ushort(__float2half_rn(sum));
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // every thread's stores of T, then this CTA's count (release at GPU scope)
+    __threadfence();
+    atomicAdd(lf.flag, 1ull);
+  }
+}
+
 // WPS: consecutive words of a thread (8 k each) that share one scale: 2 for
 // group 16, 4 for group 32, 8 (the thread's whole slice) for 64 and more.
 // x3d: X arrives as one 3-D box per stage (K a multiple of 64) instead of
@@ -266,7 +382,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                   const __grid_constant__ CUtensorMap t_map,
                   const __grid_constant__ CUtensorMap b_map, int M, int K, int group_shift,
                   int stages, int stage_bytes, int scale_rows, int x3d, int lora_rank,
-                  int n_groups, int tile_bytes, int tile_boxes, int tile_box_rows, int* err) {
+                  int n_groups, int tile_bytes, int tile_boxes, int tile_box_rows,
+                  const __grid_constant__ LoraFused lf, int* err) {
   static_assert(!(GIDX && ASYM), "act order with symmetric weights only");
   static_assert(!PERSIST || (!ASYM && !GIDX && 2 * TokGeo<BT, PRS_>::NACC * BT <= A_COL0),
                 "persistent: plain weights, two accumulator sets below the A slots");
@@ -284,6 +401,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   // 1024-byte aligned base, derived from the shared array itself so that the
   // compiler keeps the shared address space (plain LDS, no generic loads)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  if constexpr (!PERSIST && !GIDX && !ASYM && BT <= 32) {
+    // fused adapter form: the CTAs past the column blocks compute T
+    if (lf.ctas > 0 && (int)blockIdx.x >= ls.blk0[ls.count]) {
+      if (blockIdx.y == 0 && blockIdx.z == 0)
+        lora_t_cta<BT>(lf, M, K, (int)blockIdx.x - ls.blk0[ls.count],
+                       reinterpret_cast<float*>(smem));
+      return;
+    }
+  }
   // act order: the scale tile, then the ring (tile_bytes is a multiple of 1024)
   uint8_t* ring = smem + (GIDX ? tile_bytes : 0);
   DecodeBars* bar = reinterpret_cast<DecodeBars*>(ring + stages * stage_bytes);
@@ -356,12 +482,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
-  // Without an adapter the previous kernel in the stream may still be running
-  // and may write X: every thread waits for it here.  With one, the previous
-  // launch computes T and itself started only after all earlier work had
-  // completed, so X, the weights and Y are safe now and only the producer's
-  // first read of T waits for that launch (below).
-  if (lora_rank == 0) grid_dependency_wait();
+  // Without an adapter, or with T computed in this launch, the previous
+  // kernel in the stream may still be running and may write X: every thread
+  // waits for it here.  With T from a separate launch, that launch started
+  // only after all earlier work had completed, so X, the weights and Y are
+  // safe now and only the producer's first read of T waits for it (below).
+  if (lora_rank == 0 || lf.ctas > 0) grid_dependency_wait();
 
   if (warp == 0) {
     // ---------------- TMA producer (one lane) ----------------
@@ -394,7 +520,19 @@ __global__ void __launch_bounds__(THREADS, 1)
           // LoRA stage: ranks 128 l .. 128 l + 127, as two 64-rank halves
           // (a half wholly past the rank is neither loaded nor multiplied)
           if (t == n_st) {
-            grid_dependency_wait();  // T is complete and visible
+            if (lf.ctas > 0) {
+              // T from this launch's T CTAs: all of them done, then visible to
+              // TMA; the last CTA past this point clears the slot
+              if (!flag_wait_bounded(lf.flag, (uint32_t)lf.ctas, abort_flag, kWaitLimitNs)) {
+                record_timeout(err, bar);
+                break;
+              }
+              fence_proxy_async_global();
+              const unsigned long long seen = atomicAdd(lf.flag, 1ull << 32);
+              if ((seen >> 32) == (unsigned long long)(lf.consumers - 1)) atomicExch(lf.flag, 0ull);
+            } else {
+              grid_dependency_wait();  // T is complete and visible
+            }
             t_waited = true;
           }
           const int r0 = 128 * (t - n_st);
@@ -904,7 +1042,8 @@ template <int WPS, int BT, int PRS, bool ASYM, bool GIDX, bool PERSIST = false>
 cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtensorMap& qz_map,
                      const CUtensorMap& t_map, const CUtensorMap& b_map, int lora_rank, int M,
                      int K, int group_shift, int splits, int x3d, const DecodeShape& d,
-                     cudaStream_t stream, const DeviceInfo& dev) {
+                     cudaStream_t stream, const DeviceInfo& dev,
+                     const LoraFused& lf = LoraFused{}) {
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
   const int di = dev.device & 63;
@@ -917,7 +1056,7 @@ cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtens
   cudaLaunchConfig_t cfg = {};
   // persistent: one CTA per SM, each walking several column blocks
   const int blocks = ls.blk0[ls.count];
-  const int grid_x = PERSIST && blocks > dev.num_sms ? dev.num_sms : blocks;
+  const int grid_x = (PERSIST && blocks > dev.num_sms ? dev.num_sms : blocks) + lf.ctas;
   cfg.gridDim = dim3((unsigned)grid_x, (unsigned)splits, (unsigned)d.tok_tiles);
   cfg.blockDim = dim3(THREADS, 1, 1);
   cfg.dynamicSmemBytes = (size_t)d.smem_bytes;
@@ -939,7 +1078,7 @@ cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtens
   return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT, PRS, ASYM, GIDX, PERSIST>, x_map, ls, qz_map,
                             t_map, b_map, M, K, group_shift, d.stages, d.stage_bytes,
                             d.scale_rows, x3d, lora_rank, d.n_groups, d.tile_bytes, d.tile_boxes,
-                            d.tile_box_rows, dev.error_word);
+                            d.tile_box_rows, lf, dev.error_word);
 }
 
 // One linear of a launch, as the host sees it.
@@ -959,6 +1098,11 @@ struct LinearExtras {
   const uint16_t* t = nullptr;
   const uint16_t* lora_b = nullptr;
   int64_t rank = 0;
+  // fused form: T computed in the launch from lora_a; `call` numbers the
+  // call on its device (its hand-over slot is call % kTFlagSlots)
+  const uint16_t* lora_a = nullptr;
+  bool fused = false;
+  unsigned long long call = 0;
 };
 
 // X as [K/64 atoms][M tokens][64 k] (one box per stage) when K is a multiple
@@ -1043,6 +1187,16 @@ cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count,
     const int ns = (int)(((K >> 3) + PRS - 1) / PRS);
     if (splits > ns) splits = ns;
   }
+  // fused form: T CTAs on the SMs the column blocks leave free (each CTA of
+  // the layer's grid takes an SM), at most one per rank
+  LoraFused lf{};
+  if (ex.fused) {
+    const int ctas = std::min<int>((dev.num_sms - ls.blk0[count] * splits) / splits, lora_rank);
+    if (ctas < 1 || !ex.lora_a) return cudaErrorInvalidValue;
+    // the CTAs with adapter stages: the last split of every column block
+    lf = LoraFused{x, ex.lora_a, const_cast<uint16_t*>(ex.t), dev.t_flags + ex.call % kTFlagSlots,
+                   ctas, ls.blk0[count], lora_rank};
+  }
   const int iM = (int)M, iK = (int)K;
   const int gsh = group_shift;
   if (asym) {
@@ -1071,12 +1225,12 @@ cudaError_t launch_bt(const uint16_t* x, const LinearArgs* lin, int count,
   }
   if (gsh == 4)
     return launch_t<2, BT, PRS, false, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
-                                              gsh, splits, x3d, d, stream, dev);
+                                              gsh, splits, x3d, d, stream, dev, lf);
   if (gsh == 5)
     return launch_t<4, BT, PRS, false, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
-                                              gsh, splits, x3d, d, stream, dev);
+                                              gsh, splits, x3d, d, stream, dev, lf);
   return launch_t<WPT, BT, PRS, false, false>(x_map, ls, qz_map, t_map, b_map, lora_rank, iM, iK,
-                                              gsh, splits, x3d, d, stream, dev);
+                                              gsh, splits, x3d, d, stream, dev, lf);
 }
 
 cudaError_t launch_set(const uint16_t* x, const LinearArgs* lin, int count,
@@ -1239,6 +1393,46 @@ cudaError_t launch_decode_gidx(const uint16_t* x, const int32_t* qweight, const 
   if (mt > 16 && gidx_fits<32, PRA>(n_groups)) return args(launch_gidx_bt<32, PRA>);
   if (gidx_fits<16, PRA>(n_groups)) return args(launch_gidx_bt<16, PRA>);
   return cudaErrorInvalidValue;
+}
+
+bool decode_lora_fused_fits(int64_t M, int64_t K, int64_t N, int64_t rank,
+                            const DeviceInfo& dev) {
+  if (M < 1 || M > 32 || rank < 1) return false;
+  // the adapter's launch geometry: 512-k stages, the split decode_pick_splits
+  // gives them, at most one per K stage
+  const int64_t nblk = (N + BW - 1) / BW;
+  int splits = decode_pick_splits_blocks(nblk, K, 2 * PRA, dev);
+  const int ns = (int)(((K >> 3) + 2 * PRA - 1) / (2 * PRA));
+  if (splits > ns) splits = ns;
+  const int64_t ctas = std::min<int64_t>((dev.num_sms - nblk * splits) / splits, rank);
+  if (ctas < 1) return false;
+  // A T CTA's time is a chain of load latencies: its busiest warp takes
+  // ceil(ranks per CTA x 256-k pieces / warps) pieces, each in rounds of
+  // eight tokens.  Measured on the up-projection: up to 16 rounds the T CTAs
+  // finish under the layer's K stages (rank 32 at 1 to 32 tokens, rank 128
+  // at up to 8); beyond that the separate T launch is faster.
+  constexpr int64_t kWarps = THREADS / 32;
+  const int64_t ranks = (rank + ctas - 1) / ctas;
+  const int64_t pieces = (K + 255) / 256;
+  const int64_t rounds = (ranks * pieces + kWarps - 1) / kWarps * ((M + 7) / 8);
+  return rounds <= 16;
+}
+
+cudaError_t launch_decode_lora_fused(const uint16_t* x, const int32_t* qweight,
+                                     const uint16_t* scales, uint16_t* y, int64_t M, int64_t K,
+                                     int64_t N, int group_shift, uint16_t* t,
+                                     const uint16_t* lora_a, const uint16_t* lora_b,
+                                     int64_t rank, cudaStream_t stream, const DeviceInfo& dev) {
+  static std::atomic<unsigned long long> calls[64];
+  const LinearArgs one{qweight, scales, y, N};
+  LinearExtras ex;
+  ex.t = t;
+  ex.lora_b = lora_b;
+  ex.rank = rank;
+  ex.lora_a = lora_a;
+  ex.fused = true;
+  ex.call = ++calls[dev.device & 63];
+  return launch_set(x, &one, 1, ex, M, K, group_shift, 0, stream, dev);
 }
 
 cudaError_t launch_decode_grouped(const uint16_t* x, const int32_t* const* qweights,

@@ -15,7 +15,13 @@ struct DeviceInfo {
   int l2_bytes = 0;
   int* error_word = nullptr;  // device address of this device's error word
   uint16_t* lora_scratch = nullptr;  // device address of the static T buffer
+  unsigned long long* t_flags = nullptr;  // device address of the T hand-over flags
 };
+
+// Slots of the flags through which the CTAs computing a LoRA adapter's T
+// inside the layer's launch hand it over (one slot per call, reused after
+// this many calls on the device).
+constexpr int kTFlagSlots = 1024;
 
 // Error codes written to the device error word (match gptq_status values).
 constexpr int kDeviceErrTimeout = 7;
@@ -53,6 +59,15 @@ cudaError_t launch_decode_asym(const uint16_t* x, const int32_t* qweight, const 
 // Decode with a LoRA adapter: t = fp16(x . lora_a^T) [M, rank] (from
 // launch_lora_down), lora_b [N, rank]; rank/128 extra stages in the last
 // split of each column block.
+// The adapter's T computed inside the layer's decode launch (on CTAs beside
+// the column blocks) when the SMs that launch leaves free allow it; false if
+// the two-launch form must be used (then nothing is enqueued).
+bool decode_lora_fused_fits(int64_t M, int64_t K, int64_t N, int64_t rank, const DeviceInfo& dev);
+cudaError_t launch_decode_lora_fused(const uint16_t* x, const int32_t* qweight,
+                                     const uint16_t* scales, uint16_t* y, int64_t M, int64_t K,
+                                     int64_t N, int group_shift, uint16_t* t,
+                                     const uint16_t* lora_a, const uint16_t* lora_b,
+                                     int64_t rank, cudaStream_t stream, const DeviceInfo& dev);
 cudaError_t launch_decode_lora(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                                uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
                                const uint16_t* t, const uint16_t* lora_b, int64_t rank,

@@ -84,22 +84,6 @@ __device__ __forceinline__ void small_finish(float (&acc)[MB], float (*part)[MB]
     t[(int64_t)m * r + jj] = __half_as_ushort(__float2half_rn(sum));
 }
 
-__device__ __forceinline__ void fma8(float& sm, const uint4 xv, const float2 a0, const float2 a1,
-                                     const float2 a2, const float2 a3) {
-  const float2 x0 = __half22float2(*reinterpret_cast<const __half2*>(&xv.x));
-  const float2 x1 = __half22float2(*reinterpret_cast<const __half2*>(&xv.y));
-  const float2 x2 = __half22float2(*reinterpret_cast<const __half2*>(&xv.z));
-  const float2 x3 = __half22float2(*reinterpret_cast<const __half2*>(&xv.w));
-  sm = fmaf(x0.x, a0.x, sm);
-  sm = fmaf(x0.y, a0.y, sm);
-  sm = fmaf(x1.x, a1.x, sm);
-  sm = fmaf(x1.y, a1.y, sm);
-  sm = fmaf(x2.x, a2.x, sm);
-  sm = fmaf(x2.y, a2.y, sm);
-  sm = fmaf(x3.x, a3.x, sm);
-  sm = fmaf(x3.y, a3.y, sm);
-}
-
 // Lanes form, M <= LANES_M.
 __global__ void __launch_bounds__(SMALL_WARPS * 32)
     lora_down_lanes_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a,

@@ -516,6 +516,58 @@ def test_lora_small_m_ragged_k(M, K, r):
     assert err <= TOL
 
 
+# Up to 32 tokens T is computed by CTAs of the layer's own launch on the SMs
+# its column blocks leave free; with no SM free (148 column blocks or more) it
+# comes from a launch of its own before the layer's.
+@pytest.mark.parametrize("M,K,N,r", [(4, 512, 18944, 32), (20, 528, 19200, 16),
+                                     (1, 1040, 20480, 128)])
+def test_lora_without_free_sms_takes_the_separate_t_launch(M, K, N, r):
+    p = W.make_problem(M, K, N, 64, seed=M + N)
+    ad = W.make_adapter(K, N, r, seed=M + N)
+    y, t = run_lora(p, ad, t_out=True)
+    check_t(t, p.x, ad.lora_a)
+    rows = sorted({0, M - 1})
+    ref = oracle.gemm_lora_rows(p.x, p.qweight, p.scales, 64, ad.lora_a, ad.lora_b, rows)
+    err = rel_err(y[rows], ref)
+    print(f"[parity] lora, no free SM, M={M} K={K} N={N} r={r}: {err:.3e}")
+    assert err <= TOL
+
+
+@pytest.mark.parametrize("noalloc", [False, True])
+def test_lora_fused_form_replayed_from_a_cuda_graph(noalloc):
+    # the hand-over slot of T must start at zero on every replay
+    M, K, N, G, r = 16, 2048, 1024, 128, 32
+    p = W.make_problem(M, K, N, G, seed=5)
+    ad = W.make_adapter(K, N, r, seed=5)
+    x, qw, s = dev(p)
+    a = torch.from_numpy(ad.lora_a.view(np.int16)).view(torch.float16).cuda()
+    b = torch.from_numpy(ad.lora_b.view(np.int16)).view(torch.float16).cuda()
+    t = torch.empty((M, r), dtype=torch.float16, device="cuda")
+    ys = [torch.empty((M, N), dtype=torch.float16, device="cuda") for _ in range(3)]
+
+    def call(y):
+        if noalloc:
+            B.gemm_lora_noalloc(x, qw, s, G, a, b, out=y)
+        else:
+            B.gemm_lora(x, qw, s, G, a, b, t_work=t, out=y)
+
+    call(ys[0])
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for y in ys:
+            call(y)
+    for _ in range(4):
+        for y in ys:
+            y.zero_()
+        graph.replay()
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    ref = oracle.gemm_lora(p.x, p.qweight, p.scales, G, ad.lora_a, ad.lora_b)
+    for y in ys:
+        assert rel_err(y.cpu().numpy(), ref) <= TOL
+
+
 @pytest.mark.parametrize("M", [1, 40, 300])
 def test_lora_integer_exact_inputs_bitwise(M):
     """Integer x and codes, power-of-two scales, sparse +-1 lora_a and lora_b
