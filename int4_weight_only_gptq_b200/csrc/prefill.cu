@@ -10,7 +10,7 @@
 // Above 32 tokens the dispatcher below sends every call to the persistent
 // CTA-pair kernel (prefill_pair.cu).  This kernel takes the prefill path at
 // M <= 32, which only a caller that forces the prefill kernel reaches (the
-// automatic choice there is the decode kernel); it runs 64-token tiles (the
+// automatic choice up to 64 tokens is the decode kernel); it runs 64-token tiles (the
 // template also builds 128 and 256):
 //
 // * The product is computed transposed, Y^T = W^T . X^T, so that the weights
@@ -348,7 +348,7 @@ cudaError_t launch_t(const uint16_t* x, const int32_t* qweight, const uint16_t* 
 }  // namespace
 
 // Up to 32 tokens (reached only when prefill is forced: the dispatcher sends
-// M <= 32 to the decode kernel) one CTA per 128 columns x 64 tokens; above
+// M <= 64 to the decode kernel) one CTA per 128 columns x 64 tokens; above
 // that the pair kernel, whose token tile (128 or 256) follows M.
 cudaError_t launch_prefill(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                            uint16_t* y, int64_t M, int64_t K, int64_t N, int group_shift,
