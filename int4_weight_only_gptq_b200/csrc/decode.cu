@@ -285,8 +285,11 @@ __device__ __forceinline__ bool flag_wait_bounded(const unsigned long long* flag
 // its ranks j (i-th of `ctas` balanced shares) and every token m < M <= MB.
 // The ranks take the CTA's warps in equal groups that split K (a warp per
 // rank, several ranks in turn, when there are more ranks than warps); lane l
-// takes 8-k chunk l of every 256-k piece of its warp's range.  FP32 sums in a
-// fixed order: the lanes by shuffles, then the rank's warps in order.
+// takes 8-k chunk l of every 256-k piece of its warp's range, X read in
+// rounds of eight tokens.  FP32 sums in a fixed order: the lanes by shuffles,
+// then the rank's warps in order.  X and lora_a are read with plain global
+// loads after the grid-dependency wait (not through the read-only path: this
+// grid may start while the previous one still runs).
 template <int MB>
 __device__ void lora_t_cta(const LoraFused& lf, int M, int K, int i, float* part) {
   asm volatile("griddepcontrol.wait;" ::: "memory");  // X may come from the previous kernel
@@ -302,11 +305,11 @@ __device__ void lora_t_cta(const LoraFused& lf, int M, int K, int i, float* part
     float acc[MB];
 #pragma unroll
     for (int m = 0; m < MB; ++m) acc[m] = 0.f;
-    const uint16_t* __restrict__ arow = lf.a + (int64_t)(r0 + rr) * K;
+    const uint16_t* arow = lf.a + (int64_t)(r0 + rr) * K;
     for (int pc = pb; pc < pe; ++pc) {
       const int k = pc * 256 + 8 * lane;
       if (k < K) {  // K % 8 == 0: the chunk is whole
-        const uint4 av = __ldg(reinterpret_cast<const uint4*>(arow + k));
+        const uint4 av = *reinterpret_cast<const uint4*>(arow + k);
         const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&av.x));
         const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&av.y));
         const float2 a2 = __half22float2(*reinterpret_cast<const __half2*>(&av.z));
@@ -317,9 +320,8 @@ __device__ void lora_t_cta(const LoraFused& lf, int M, int K, int i, float* part
           uint4 xv[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            xv[q] = m0 + q < M
-                        ? __ldg(reinterpret_cast<const uint4*>(lf.x + (int64_t)(m0 + q) * K + k))
-                        : make_uint4(0, 0, 0, 0);
+            xv[q] = m0 + q < M ? *reinterpret_cast<const uint4*>(lf.x + (int64_t)(m0 + q) * K + k)
+                               : make_uint4(0, 0, 0, 0);
 #pragma unroll
           for (int q = 0; q < 8; ++q) fma8(acc[m0 + q], xv[q], a0, a1, a2, a3);
         }
@@ -401,7 +403,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   // 1024-byte aligned base, derived from the shared array itself so that the
   // compiler keeps the shared address space (plain LDS, no generic loads)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  if constexpr (!PERSIST && !GIDX && !ASYM && BT <= 32) {
+  if constexpr (!PERSIST && !GIDX && !ASYM && TokGeo<BT, PRS_>::LORA_OK) {
     // fused adapter form: the CTAs past the column blocks compute T
     if (lf.ctas > 0 && (int)blockIdx.x >= ls.blk0[ls.count]) {
       if (blockIdx.y == 0 && blockIdx.z == 0)
