@@ -349,7 +349,8 @@ int gptq_w4a16_gemm_asym(const uint16_t* x, const int32_t* qweight, const uint16
   const int gs = group_shift_of(group);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const cudaError_t e = M <= GPTQ_DECODE_MAX_M
-                            ? launch_decode_asym(x, qweight, scales, qzeros, y, M, K, N, gs, s, *dev)
+                            ? launch_decode_asym(x, qweight, scales, qzeros, y, M, K, N, gs, s,
+                                                 *dev)
                             : launch_prefill_pair_asym(x, qweight, scales, qzeros, y, M, K, N, gs,
                                                        s, *dev);
   if (e != cudaSuccess) {

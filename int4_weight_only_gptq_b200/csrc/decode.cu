@@ -732,7 +732,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     bool ok = true;
     if constexpr (GIDX) {
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar->tile_full, 0u, abort_flag, kWaitLimitNs));
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_bounded(&bar->tile_full, 0u, abort_flag, kWaitLimitNs));
       if (!ok && lane == 0) record_timeout(err, bar);
     }
     // this thread's column of the scale tile (act order)
@@ -1077,7 +1078,8 @@ cudaError_t launch_t(const CUtensorMap& x_map, const LinearSet& ls, const CUtens
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT, PRS, ASYM, GIDX, PERSIST>, x_map, ls, qz_map,
+  return cudaLaunchKernelEx(&cfg, decode_kernel<WPS, BT, PRS, ASYM, GIDX, PERSIST>, x_map, ls,
+                            qz_map,
                             t_map, b_map, M, K, group_shift, d.stages, d.stage_bytes,
                             d.scale_rows, x3d, lora_rank, d.n_groups, d.tile_bytes, d.tile_boxes,
                             d.tile_box_rows, lf, dev.error_word);

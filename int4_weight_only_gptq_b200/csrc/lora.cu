@@ -178,7 +178,8 @@ cudaError_t launch_small(bool lanes, const uint16_t* x, const uint16_t* lora_a, 
   int splits = lanes && free_sms >= (int)gr ? free_sms / (int)gr : dev.num_sms / (int)gr;
   splits = std::max(1, std::min(kMaxSplits, splits));
   splits = std::min<int>(splits, (int)std::max<int64_t>(1, (K + PIECE - 1) / PIECE));
-  const void* fn = lanes ? (const void*)lora_down_lanes_kernel : (const void*)lora_down_staged_kernel;
+  const void* fn =
+      lanes ? (const void*)lora_down_lanes_kernel : (const void*)lora_down_staged_kernel;
   if (splits > 8) {
     static std::once_flag once[2][64];
     static cudaError_t attr_err[2][64];
