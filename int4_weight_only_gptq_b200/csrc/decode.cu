@@ -364,7 +364,10 @@ __device__ void lora_t_cta(const LoraFused& lf, int M, int K, int i, float* part
 // 128 rows x 128 ranks go to the qweight area (two 64-rank boxes, 128-byte
 // swizzle), T's rows to the X area (two 64-rank atoms); one fill per stage
 // copies lora_b into the A slot in the paired k order (T is permuted like X),
-// and the MMAs add T . lora_b^T to the same accumulators.
+// and the MMAs add T . lora_b^T to the same accumulators.  lf.ctas > 0 (the
+// fused form, LoraFused above): the CTAs past the column blocks compute T,
+// and the producer's first read of T waits on the hand-over counter instead
+// of the grid dependency.
 // GIDX (act order): every k has its own group g_idx[k].  The CTA's whole
 // scale tile [n_groups x 128 columns] is loaded once into shared memory in
 // front of the ring (tile_boxes boxes of tile_box_rows rows, tile_bytes in
